@@ -299,8 +299,8 @@ void orc_select(int kind, const void* K, const float* ks, int Hkv, int d, const 
       int64_t nsel = nc < k ? nc : k;
       int64_t* sel = (int64_t*)malloc(sizeof(int64_t) * (size_t)(nsel > 0 ? nsel : 1));
       kth[r * Hkv + g] = NAN;
-      if (nc <= k) {
-        for (int64_t j = 0; j < nc; ++j) sel[j] = j;
+      if (nc <= k || k == 0) { /* all candidates, or none when k = 0 (no k-th score) */
+        for (int64_t j = 0; j < nsel; ++j) sel[j] = j;
       } else {
         double* q = (double*)malloc(sizeof(double) * d * G);
         for (int hh = 0; hh < G; ++hh) fetch_q(Qr, r, g * G + hh, Hq, d, q + hh * d);

@@ -245,7 +245,8 @@ def test_sparse_with_k0_equals_sliding_window(orc):
     kv, sc = orc.KV(K, V), 1 / math.sqrt(d)
     rows = np.arange(T)
     _, lse = orc.full_attn(kv, Q, rows, sc)
-    idx, _ = orc.select(kv, Q, rows, sc, lse, 0, w)
+    idx, kth = orc.select(kv, Q, rows, sc, lse, 0, w)
+    assert np.all(np.isnan(kth)) and np.all(idx[:, :, :0] == 0)
     Os, ls = orc.sparse_attn(kv, Q, idx, sc)
     Oref, lref = _sdpa_ref(f(Q), f(K), f(V), sc, lambda i, j: (j <= i) & (j > i - w))
     np.testing.assert_allclose(Os, Oref, rtol=1e-10, atol=1e-12)
