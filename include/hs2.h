@@ -1,0 +1,201 @@
+/*
+ * hs2.h -- C ABI of the B200 (sm_100a) HySparse2 cross-decoder block library.
+ *
+ * HySparse2 ("Hybrid Sparse Attention with Two-Level KV Sharing") splits a
+ * model into a self-decoder and a cross-decoder.  Each cross-decoder block is
+ * one full-attention layer followed by several sparse-attention layers.  The
+ * block's K/V come from self-decoder hidden states (KV Bridging); the sparse
+ * layers reuse that K/V cache and the full layer's token list (KV Reuse).  The
+ * list holds, per query token, the 1024 earlier tokens the full layer's
+ * attention scores rank highest plus a forced window of the 128 most recent.
+ * Sources: javabetter.cn explainer "mimo-v3-hysparse2" (Cross-Decoder, KV Reuse,
+ * KV Bridging, selection-granularity and local-window paragraphs); siami.tw
+ * "小米 MiMo-V3 全新架構亮相：HySparse 2 把 1M Token 預填成本砍到 1/5",
+ * sections 一 and 四; zgeo.com.cn "小米MiMo-V3架构剧透：HySparse2稀疏注意力…",
+ * section 核心技术原理解析 and its comparison table; aitop.news "Xiaomi MiMo-V3
+ * to Adopt New Architecture with HySparse 2".
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Pointers are DEVICE pointers owned by the caller unless stated otherwise,
+ *   16-byte aligned, dense, in these layouts (row-major, last index fastest):
+ *     Q, O            [T, n_q_heads, head_dim]       bf16
+ *     K, V            [T, n_kv_heads, head_dim]      bf16
+ *     lse             [T, n_q_heads]                 fp32, natural log
+ *     idx             [T, n_kv_heads, k_global + window]  int32
+ *   Query head h uses KV head g = h / G with G = n_q_heads / n_kv_heads.
+ * - bf16 and e4m3 values are passed as their raw bits (hs2_bf16, hs2_fp8e4m3).
+ * - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *   default stream) and never synchronises, except hs2_get_device_status.
+ * - The library allocates no device memory.  Calls that need temporaries take
+ *   a caller-owned workspace of at least hs2_workspace_size() bytes.
+ * - Arguments are checked on the host before any launch.  A failed check
+ *   returns an error and launches nothing; outputs are then untouched.
+ * - Device-side waits are bounded.  A wait that runs out sets a sticky device
+ *   status word, the kernel returns early, and the next
+ *   hs2_get_device_status() reports HS2_ERR_TIMEOUT.
+ * - Supported: head_dim == 128; G in {1, 2, 4, 8, 16}; 0 <= k_global <= 2048;
+ *   1 <= window <= 2048; 1 <= T <= 2^31 - 1 (T * n_q_heads * 128 < 2^40).
+ * - Thread safety: calls on different streams may run concurrently; the only
+ *   global state is one-time kernel attribute set-up per device.
+ */
+#ifndef HS2_H_
+#define HS2_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HS2_OK = 0,
+  HS2_ERR_INVALID_ARG = 1, /* null/misaligned pointer, T <= 0, bad k/window   */
+  HS2_ERR_UNSUPPORTED = 2, /* head_dim != 128, G not in {1,2,4,8,16}, ...      */
+  HS2_ERR_WORKSPACE = 3,   /* workspace pointer null or smaller than required  */
+  HS2_ERR_CUDA = 4,        /* a CUDA runtime/driver call or launch failed      */
+  HS2_ERR_TIMEOUT = 5      /* a device-side bounded wait ran out               */
+} hs2_status;
+
+typedef uint16_t hs2_bf16;    /* raw bf16 bits */
+typedef uint8_t hs2_fp8e4m3;  /* raw OCP E4M3FN bits */
+
+typedef struct {
+  int64_t T;           /* tokens (prefill) or cache capacity (decode)          */
+  int32_t n_q_heads;   /* Hq                                                   */
+  int32_t n_kv_heads;  /* Hkv; Hq % Hkv == 0                                   */
+  int32_t head_dim;    /* d; must be 128                                       */
+  float scale;         /* logit scale, normally 1/sqrt(d)                      */
+  int32_t k_global;    /* k: globally selected tokens per (query, KV head)     */
+  int32_t window;      /* w: forced recent window, positions i-w+1 .. i        */
+} hs2_shape;
+
+/* Workspace queries (op codes for hs2_workspace_size). */
+enum {
+  HS2_OP_BRIDGE = 0,
+  HS2_OP_FULL_ATTN = 1,
+  HS2_OP_SELECT = 2,
+  HS2_OP_SPARSE = 3,
+  HS2_OP_BLOCK_PREFILL = 4,
+  HS2_OP_BLOCK_DECODE = 5
+};
+
+/*
+ * KV Bridging (step S1).  KV Bridging section of the javabetter.cn explainer
+ * and section 一 of the siami.tw article: the cross-decoder full-attention
+ * layer computes K and V from self-decoder hidden states with its own
+ * projection parameters.
+ *   K[t, :] = H[t, :] W_k,   V[t, :] = H[t, :] W_v
+ * H [T, d_model] bf16; W_k, W_v [d_model, n_kv_heads * 128] bf16 (row-major);
+ * K, V [T, n_kv_heads, 128] bf16, written with fp32 accumulation and one
+ * round-to-nearest-even to bf16.  No RoPE, norm or bias (the pages name none).
+ * d_model must be a positive multiple of 64.
+ */
+hs2_status hs2_bridge_kv(const hs2_bf16* H, int32_t d_model, const hs2_bf16* W_k,
+                         const hs2_bf16* W_v, hs2_bf16* K, hs2_bf16* V,
+                         const hs2_shape* shape, void* stream);
+
+/*
+ * Causal GQA full attention with per-row log-sum-exp (step S2).  The block's
+ * full-attention layer (Cross-Decoder paragraph of the javabetter.cn
+ * explainer); its complete attention scores later rank tokens (section
+ * 核心技术原理解析 of the zgeo.com.cn page).  For row i, head h, g = h / G:
+ *   s_j = scale * Q[i,h] . K[j,g]  (0 <= j <= i)
+ *   lse[i,h] = ln sum_j exp(s_j),  O[i,h] = sum_j exp(s_j - lse[i,h]) V[j,g]
+ * O is rounded once to bf16; lse is fp32.  No workspace.
+ */
+hs2_status hs2_full_attn_lse(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V,
+                             hs2_bf16* O, float* lse, const hs2_shape* shape, void* stream);
+
+/*
+ * Token-level selection with forced recent window (step S3).  Selection
+ * paragraphs of the javabetter.cn explainer (tokens picked one by one, e.g.
+ * 1024 from the whole context, by the full layer's attention scores; the 128
+ * most recent always kept), section 四 of the siami.tw article, and the
+ * 1024 + 128 entry of the zgeo.com.cn comparison table.
+ *   score[i,g,j] = sum over the G query heads h of g of exp(s_{h,i,j} - lse[i,h])
+ *   candidates j in [0, i - w]; all of them when there are at most k,
+ *   otherwise the k largest scores, equal scores going to the smaller j.
+ * idx[i,g,0..k-1]: the selected positions in ascending order, then -1 padding.
+ * idx[i,g,k+t] = i - w + 1 + t for t in [0, w), or -1 where that is negative.
+ * kth_score (nullable) [T, n_kv_heads] fp32: score of the k-th selected token,
+ * or -1 when every candidate is selected.
+ * lse is the full layer's lse (as written by hs2_full_attn_lse).
+ * Workspace: hs2_workspace_size(HS2_OP_SELECT, ...) bytes.
+ */
+hs2_status hs2_select_topk(const hs2_bf16* Q, const hs2_bf16* K, const float* lse,
+                           int32_t* idx, float* kth_score, const hs2_shape* shape,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Sparse attention over the shared K/V and index list (step S4, KV Reuse).
+ * KV Reuse paragraph of the javabetter.cn explainer and the aitop.news
+ * summary: each sparse layer has its own queries, reuses the full layer's K/V
+ * cache and selection indices, and stores no K/V.  For row i, head h:
+ *   s_j = scale * Q[i,h] . K[j,g] for j in idx[i,g,:] (entries < 0 skipped)
+ *   O[i,h] = sum_j softmax_j(s) V[j,g];  lse (nullable) = ln sum_j exp(s_j).
+ * Entries must satisfy -1 <= idx < T; lists hold no duplicates (as written by
+ * hs2_select_topk).  A row whose list is entirely -1 gets O = 0, lse = -inf.
+ * No workspace.
+ */
+hs2_status hs2_sparse_attn(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V,
+                           const int32_t* idx, hs2_bf16* O, float* lse,
+                           const hs2_shape* shape, void* stream);
+
+/*
+ * The whole block at prefill: bridge (if H != NULL), full attention, selection
+ * and n_sparse sparse layers sharing K/V and idx (all of the above, in order,
+ * on `stream`).  Q_sparse and O_sparse are HOST arrays of n_sparse DEVICE
+ * pointers.  With H == NULL, K and V are inputs and d_model, W_k, W_v are
+ * ignored.  Workspace: hs2_workspace_size(HS2_OP_BLOCK_PREFILL, ...).
+ */
+hs2_status hs2_block_prefill(const hs2_bf16* H, int32_t d_model, const hs2_bf16* W_k,
+                             const hs2_bf16* W_v, hs2_bf16* K, hs2_bf16* V,
+                             const hs2_bf16* Q_full, hs2_bf16* O_full, float* lse,
+                             int32_t* idx, int32_t n_sparse, const hs2_bf16* const* Q_sparse,
+                             hs2_bf16* const* O_sparse, const hs2_shape* shape,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * One decode step of the block over an FP8 KV cache (step S5).  The FP8 KV
+ * cache of the zgeo.com.cn comparison table and of the javabetter.cn
+ * explainer's 1M-token figures; the cross-decoder runs only while generating.
+ * For each sequence b the new token is the last cache entry, i = seq_len[b]-1,
+ * and the block (full attention, selection, n_sparse sparse layers) runs on
+ *   K^[t,g,:] = e4m3(Kc[b,t,g,:]) * k_scale[b,t,g],  likewise V with v_scale.
+ * seq_len: HOST array [batch], 1 <= seq_len[b] <= shape->T.
+ * Kc, Vc [batch, shape->T, n_kv_heads, 128] e4m3; k_scale, v_scale
+ * [batch, shape->T, n_kv_heads] fp32 (they may alias).
+ * q_full, o_full [batch, n_q_heads, 128] bf16; lse [batch, n_q_heads] fp32;
+ * idx [batch, n_kv_heads, k + w] int32; q_sparse/o_sparse: HOST arrays of
+ * n_sparse DEVICE pointers to [batch, n_q_heads, 128] bf16.
+ * Workspace: hs2_workspace_size(HS2_OP_BLOCK_DECODE, shape, batch, 0).
+ */
+hs2_status hs2_block_decode(int32_t batch, const int64_t* seq_len, const hs2_bf16* q_full,
+                            const hs2_fp8e4m3* Kc, const hs2_fp8e4m3* Vc,
+                            const float* k_scale, const float* v_scale, hs2_bf16* o_full,
+                            float* lse, int32_t* idx, int32_t n_sparse,
+                            const hs2_bf16* const* q_sparse, hs2_bf16* const* o_sparse,
+                            const hs2_shape* shape, void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/* Workspace bytes needed by `op` (an HS2_OP_* code) for these sizes; 0 when
+ * the op needs none.  Returns (size_t)-1 for invalid arguments. */
+size_t hs2_workspace_size(int32_t op, const hs2_shape* shape, int32_t batch, int32_t d_model);
+
+/* Synchronises `stream` and reports a sticky device-side error (a bounded
+ * wait that ran out) as HS2_ERR_TIMEOUT, clearing it; CUDA errors as
+ * HS2_ERR_CUDA. */
+hs2_status hs2_get_device_status(void* stream);
+
+/* Static English text for a status code. */
+const char* hs2_status_string(hs2_status status);
+
+/* Launch count of the library's kernels since load (all devices). */
+uint64_t hs2_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HS2_H_ */

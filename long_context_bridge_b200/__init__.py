@@ -1,0 +1,187 @@
+"""Python binding of libhs2 (the HySparse2 cross-decoder block for B200).
+
+Argument marshalling only: every function checks tensor dtypes, devices and
+contiguity, then calls the C entry point of the same name with raw device
+pointers and the current CUDA stream.  All computation runs in the library's
+CUDA kernels.  There is no fallback: if ``libhs2.so`` is missing or fails to
+load, importing this package raises.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libhs2.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(6)
+OP_BRIDGE, OP_FULL_ATTN, OP_SELECT, OP_SPARSE, OP_BLOCK_PREFILL, OP_BLOCK_DECODE = range(6)
+
+
+class HS2Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {_lib.hs2_status_string(status).decode()} (status {status})")
+        self.status = status
+
+
+class Shape(C.Structure):
+    """hs2_shape: T, n_q_heads, n_kv_heads, head_dim, scale, k_global, window."""
+    _fields_ = [("T", C.c_int64), ("n_q_heads", C.c_int32), ("n_kv_heads", C.c_int32),
+                ("head_dim", C.c_int32), ("scale", C.c_float), ("k_global", C.c_int32),
+                ("window", C.c_int32)]
+
+    @classmethod
+    def make(cls, T, n_q_heads, n_kv_heads, head_dim=128, scale=None, k_global=1024, window=128):
+        if scale is None:
+            scale = head_dim ** -0.5
+        return cls(int(T), int(n_q_heads), int(n_kv_heads), int(head_dim), float(scale),
+                   int(k_global), int(window))
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libhs2.so not built at {LIB_PATH}: run long_context_bridge_b200/build.py")
+    L = C.CDLL(LIB_PATH)
+    P, I32, I64, SZ = C.c_void_p, C.c_int32, C.c_int64, C.c_size_t
+    SP = C.POINTER(Shape)
+    PP = C.POINTER(C.c_void_p)
+    sigs = {
+        "hs2_bridge_kv": [P, I32, P, P, P, P, SP, P],
+        "hs2_full_attn_lse": [P, P, P, P, P, SP, P],
+        "hs2_select_topk": [P, P, P, P, P, SP, P, SZ, P],
+        "hs2_sparse_attn": [P, P, P, P, P, P, SP, P],
+        "hs2_block_prefill": [P, I32, P, P, P, P, P, P, P, P, I32, PP, PP, SP, P, SZ, P],
+        "hs2_block_decode": [I32, C.POINTER(C.c_int64), P, P, P, P, P, P, P, P, I32, PP, PP, SP,
+                             P, SZ, P],
+    }
+    for name, args in sigs.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = C.c_int
+    L.hs2_workspace_size.argtypes = [I32, SP, I32, I32]
+    L.hs2_workspace_size.restype = SZ
+    L.hs2_get_device_status.argtypes = [P]
+    L.hs2_get_device_status.restype = C.c_int
+    L.hs2_status_string.argtypes = [C.c_int]
+    L.hs2_status_string.restype = C.c_char_p
+    L.hs2_kernel_launches.restype = C.c_uint64
+    return L
+
+
+_lib = _load()
+
+EXPORTED = ["hs2_bridge_kv", "hs2_full_attn_lse", "hs2_select_topk", "hs2_sparse_attn",
+            "hs2_block_prefill", "hs2_block_decode", "hs2_workspace_size",
+            "hs2_get_device_status", "hs2_status_string", "hs2_kernel_launches"]
+
+
+def _ptr(t, dtype, what, nullable=False):
+    if t is None:
+        if nullable:
+            return None
+        raise ValueError(f"{what} is required")
+    if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
+        raise ValueError(f"{what} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{what} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{what} must be contiguous")
+    return C.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        return C.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return C.c_void_p(stream.cuda_stream)
+    return C.c_void_p(int(stream))
+
+
+def _check(status, what):
+    if status != OK:
+        raise HS2Error(status, what)
+
+
+BF16, F32, I32T, U8 = torch.bfloat16, torch.float32, torch.int32, torch.uint8
+
+
+def workspace_size(op: int, shape: Shape, batch: int = 1, d_model: int = 0) -> int:
+    n = _lib.hs2_workspace_size(op, C.byref(shape), batch, d_model)
+    if n == C.c_size_t(-1).value:
+        raise HS2Error(ERR_INVALID_ARG, "hs2_workspace_size")
+    return int(n)
+
+
+def hs2_bridge_kv(H, W_k, W_v, K, V, shape: Shape, stream=None):
+    _check(_lib.hs2_bridge_kv(_ptr(H, BF16, "H"), H.shape[-1], _ptr(W_k, BF16, "W_k"),
+                              _ptr(W_v, BF16, "W_v"), _ptr(K, BF16, "K"), _ptr(V, BF16, "V"),
+                              C.byref(shape), _stream(stream)), "hs2_bridge_kv")
+
+
+def hs2_full_attn_lse(Q, K, V, O, lse, shape: Shape, stream=None):
+    _check(_lib.hs2_full_attn_lse(_ptr(Q, BF16, "Q"), _ptr(K, BF16, "K"), _ptr(V, BF16, "V"),
+                                  _ptr(O, BF16, "O"), _ptr(lse, F32, "lse"), C.byref(shape),
+                                  _stream(stream)), "hs2_full_attn_lse")
+
+
+def hs2_select_topk(Q, K, lse, idx, kth, shape: Shape, workspace, stream=None):
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.hs2_select_topk(_ptr(Q, BF16, "Q"), _ptr(K, BF16, "K"), _ptr(lse, F32, "lse"),
+                                _ptr(idx, I32T, "idx"), _ptr(kth, F32, "kth", True),
+                                C.byref(shape), _ptr(workspace, U8, "workspace", True), nbytes,
+                                _stream(stream)), "hs2_select_topk")
+
+
+def hs2_sparse_attn(Q, K, V, idx, O, lse, shape: Shape, stream=None):
+    _check(_lib.hs2_sparse_attn(_ptr(Q, BF16, "Q"), _ptr(K, BF16, "K"), _ptr(V, BF16, "V"),
+                                _ptr(idx, I32T, "idx"), _ptr(O, BF16, "O"),
+                                _ptr(lse, F32, "lse", True), C.byref(shape), _stream(stream)),
+           "hs2_sparse_attn")
+
+
+def _ptr_array(ts, dtype, what):
+    arr = (C.c_void_p * max(1, len(ts)))()
+    for i, t in enumerate(ts):
+        arr[i] = _ptr(t, dtype, f"{what}[{i}]").value
+    return C.cast(arr, C.POINTER(C.c_void_p)), arr
+
+
+def hs2_block_prefill(H, W_k, W_v, K, V, Q_full, O_full, lse, idx, Q_sparse, O_sparse,
+                      shape: Shape, workspace, stream=None):
+    qs, _keep_q = _ptr_array(Q_sparse, BF16, "Q_sparse")
+    os_, _keep_o = _ptr_array(O_sparse, BF16, "O_sparse")
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.hs2_block_prefill(
+        _ptr(H, BF16, "H", True), 0 if H is None else H.shape[-1], _ptr(W_k, BF16, "W_k", True),
+        _ptr(W_v, BF16, "W_v", True), _ptr(K, BF16, "K"), _ptr(V, BF16, "V"),
+        _ptr(Q_full, BF16, "Q_full"), _ptr(O_full, BF16, "O_full"), _ptr(lse, F32, "lse"),
+        _ptr(idx, I32T, "idx"), len(Q_sparse), qs, os_, C.byref(shape),
+        _ptr(workspace, U8, "workspace", True), nbytes, _stream(stream)), "hs2_block_prefill")
+
+
+def hs2_block_decode(seq_len, q_full, Kc, Vc, k_scale, v_scale, o_full, lse, idx, q_sparse,
+                     o_sparse, shape: Shape, workspace, stream=None):
+    B = len(seq_len)
+    lens = (C.c_int64 * B)(*[int(x) for x in seq_len])
+    qs, _keep_q = _ptr_array(q_sparse, BF16, "q_sparse")
+    os_, _keep_o = _ptr_array(o_sparse, BF16, "o_sparse")
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.hs2_block_decode(
+        B, lens, _ptr(q_full, BF16, "q_full"), _ptr(Kc, U8, "Kc"), _ptr(Vc, U8, "Vc"),
+        _ptr(k_scale, F32, "k_scale"), _ptr(v_scale, F32, "v_scale"), _ptr(o_full, BF16, "o_full"),
+        _ptr(lse, F32, "lse"), _ptr(idx, I32T, "idx"), len(q_sparse), qs, os_, C.byref(shape),
+        _ptr(workspace, U8, "workspace", True), nbytes, _stream(stream)), "hs2_block_decode")
+
+
+def hs2_get_device_status(stream=None) -> int:
+    return int(_lib.hs2_get_device_status(_stream(stream)))
+
+
+def hs2_kernel_launches() -> int:
+    return int(_lib.hs2_kernel_launches())
+
+
+def hs2_status_string(status: int) -> str:
+    return _lib.hs2_status_string(status).decode()

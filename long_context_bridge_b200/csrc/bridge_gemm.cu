@@ -1,0 +1,163 @@
+// bridge_gemm.cu -- KV Bridging projection K = H W_k, V = H W_v on tcgen05.
+//
+// KV Bridging (javabetter.cn explainer "mimo-v3-hysparse2", KV Bridging
+// paragraph; siami.tw article section 一): the cross-decoder full-attention
+// layer computes its K/V from self-decoder hidden states with its own weights.
+//
+// One CTA computes a 128 x BN tile of [K | V] (N index n < Nkv -> K, else V):
+//   warp 0     TMA producer: H tile [128 x 64] (K-major) and W tile [64 x BN]
+//              (MN-major, W is row-major [d_model, Nkv]) into a STAGES ring
+//   warp 1     allocates TMEM, one lane issues tcgen05.mma 128xBNx16 and
+//              commits each stage back to the producer
+//   warps 2-5  epilogue: TMEM -> registers -> bf16 -> global
+#include "common.cuh"
+#include "kernels.h"
+
+namespace hs2 {
+
+HS2_STATUS_ACCESSOR(status_bridge)
+
+
+namespace {
+constexpr int BM = 128, BK = 64, STAGES = 3;
+constexpr int THREADS = 192;
+
+template <int BN>
+struct BridgeCfg {
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BK * BN * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr uint32_t IDESC = idesc_bf16(BM, BN, /*a_mn=*/0, /*b_mn=*/1);
+};
+
+template <int BN>
+__global__ void __launch_bounds__(THREADS, 1)
+    bridge_gemm_kernel(const __grid_constant__ CUtensorMap tmH,
+                       const __grid_constant__ CUtensorMap tmWk,
+                       const __grid_constant__ CUtensorMap tmWv, __nv_bfloat16* __restrict__ K,
+                       __nv_bfloat16* __restrict__ V, int T, int dm, int Nkv) {
+  using C = BridgeCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* accbar = empty + STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accbar + 1);
+
+  const int warp = warp_id(), lane = lane_id();
+  const int n0 = blockIdx.x * BN;  // column of [K | V]
+  const int m0 = blockIdx.y * BM;
+  const bool isV = n0 >= Nkv;
+  const int nloc = isV ? n0 - Nkv : n0;
+  const int num_kb = dm / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accbar, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, BN);
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer ----------------
+    prefetch_tmap(&tmH);
+    prefetch_tmap(isV ? &tmWv : &tmWk);
+    for (int kb = 0; kb < num_kb; ++kb) {
+      const int s = kb % STAGES;
+      if (kb >= STAGES && !mbar_wait(&empty[s], ((kb / STAGES) & 1) ^ 1)) break;
+      uint8_t* sA = smem + s * C::STAGE_BYTES;
+      uint8_t* sB = sA + C::A_BYTES;
+      mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+      tma_load_2d(sA, &tmH, &full[s], kb * BK, m0);
+#pragma unroll
+      for (int c = 0; c < BN / 64; ++c)
+        tma_load_2d(sB + c * (BK * 128), isV ? &tmWv : &tmWk, &full[s], nloc + c * 64, kb * BK);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer ----------------
+    bool ok = true;
+    for (int kb = 0; kb < num_kb && ok; ++kb) {
+      const int s = kb % STAGES;
+      if (!mbar_wait(&full[s], (kb / STAGES) & 1)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t a0 = smem_u32(smem + s * C::STAGE_BYTES);
+      const uint32_t b0 = a0 + C::A_BYTES;
+#pragma unroll
+      for (int ks = 0; ks < BK / 16; ++ks) {
+        // A: K-major, advance 16 elements = 32 B inside the 128 B swizzle row
+        const uint64_t ad = sdesc_sw128(a0 + ks * 32, 16, 1024);
+        // B: MN-major, advance 16 K-rows of 128 B; MN chunks of 64 are BK*128 B apart
+        const uint64_t bd = sdesc_sw128(b0 + ks * 16 * 128, BK * 128, 1024);
+        mma_ss(tmem, ad, bd, C::IDESC, (kb | ks) != 0);
+      }
+      mma_commit(&empty[s]);
+    }
+    mma_commit(accbar);
+  } else if (warp >= 2) {
+    // ---------------- epilogue ----------------
+    const int sub = warp & 3;  // TMEM lanes 32*sub .. 32*sub+31
+    const bool ok = mbar_wait(accbar, 0);
+    tc_fence_after();
+    const int row = m0 + sub * 32 + lane;
+    __nv_bfloat16* out = isV ? V : K;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      uint32_t r[32];
+      tmem_ld32(tmem + (uint32_t(sub * 32) << 16) + c * 32, r);
+      tmem_wait_ld();
+      if (ok && row < T) {
+        uint4* dst = reinterpret_cast<uint4*>(out + size_t(row) * Nkv + nloc + c * 32);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint4 v;
+          v.x = pack_bf16x2(__uint_as_float(r[8 * q + 0]), __uint_as_float(r[8 * q + 1]));
+          v.y = pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3]));
+          v.z = pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5]));
+          v.w = pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7]));
+          dst[q] = v;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, BN);
+  }
+}
+}  // namespace
+
+cudaError_t launch_bridge(const BridgeArgs& a, cudaStream_t stream) {
+  constexpr int BN = 128;
+  using C = BridgeCfg<BN>;
+  CUtensorMap tmH, tmWk, tmWv;
+  // H [T, dm]: x = feature (contiguous), y = token; box 64 x 128
+  if (!make_tmap_2d(&tmH, a.H, a.dm, a.T, size_t(a.dm) * 2, 64, BM)) return cudaErrorInvalidValue;
+  // W [dm, Nkv]: x = output column (contiguous), y = feature; box 64 x 64
+  if (!make_tmap_2d(&tmWk, a.Wk, a.Nkv, a.dm, size_t(a.Nkv) * 2, 64, BK))
+    return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tmWv, a.Wv, a.Nkv, a.dm, size_t(a.Nkv) * 2, 64, BK))
+    return cudaErrorInvalidValue;
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(bridge_gemm_kernel<BN>), C::SMEM);
+  if (e != cudaSuccess) return e;
+  dim3 grid(2 * a.Nkv / BN, (a.T + BM - 1) / BM);
+  bridge_gemm_kernel<BN><<<grid, THREADS, C::SMEM, stream>>>(
+      tmH, tmWk, tmWv, reinterpret_cast<__nv_bfloat16*>(a.K),
+      reinterpret_cast<__nv_bfloat16*>(a.V), int(a.T), a.dm, a.Nkv);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace hs2

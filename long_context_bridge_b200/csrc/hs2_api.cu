@@ -1,0 +1,295 @@
+// hs2_api.cu -- the C ABI declared in include/hs2.h: host-side argument
+// checks, workspace sizing and kernel launches.  Every step of the block runs
+// in the kernels of this library; nothing here computes results on the host.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "../../include/hs2.h"
+#include "common.cuh"
+#include "kernels.h"
+
+namespace hs2 {
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+// ---------------------------------------------------------------------------
+// tensor maps through the driver entry point (no link-time libcuda dependency)
+// ---------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+static bool encode(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                   const uint64_t* strides, const uint32_t* box) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  const uint32_t elem[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims,
+                  strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_2d(CUtensorMap* map, const void* base, uint64_t dim_x, uint64_t dim_y,
+                  uint64_t stride_y, uint32_t box_x, uint32_t box_y) {
+  const uint64_t dims[2] = {dim_x, dim_y};
+  const uint64_t strides[1] = {stride_y};
+  const uint32_t box[2] = {box_x, box_y};
+  return encode(map, base, 2, dims, strides, box);
+}
+
+bool make_tmap_3d(CUtensorMap* map, const void* base, uint64_t dim_x, uint64_t dim_y,
+                  uint64_t dim_z, uint64_t stride_y, uint64_t stride_z, uint32_t box_x,
+                  uint32_t box_y, uint32_t box_z) {
+  const uint64_t dims[3] = {dim_x, dim_y, dim_z};
+  const uint64_t strides[2] = {stride_y, stride_z};
+  const uint32_t box[3] = {box_x, box_y, box_z};
+  return encode(map, base, 3, dims, strides, box);
+}
+
+cudaError_t ensure_smem_attr(const void* func, int bytes) {
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done.count({func, dev})) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.insert({func, dev});
+  return e;
+}
+
+}  // namespace hs2
+
+using namespace hs2;
+
+// ---------------------------------------------------------------------------
+// argument checks
+// ---------------------------------------------------------------------------
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+hs2_status check_shape(const hs2_shape* s, bool need_select) {
+  if (s == nullptr) return HS2_ERR_INVALID_ARG;
+  if (s->T <= 0 || s->T > INT32_MAX || s->n_q_heads <= 0 || s->n_kv_heads <= 0)
+    return HS2_ERR_INVALID_ARG;
+  if (!(s->scale > 0.f) || s->scale != s->scale) return HS2_ERR_INVALID_ARG;
+  if (s->head_dim != 128) return HS2_ERR_UNSUPPORTED;
+  if (s->n_q_heads % s->n_kv_heads != 0) return HS2_ERR_UNSUPPORTED;
+  const int G = s->n_q_heads / s->n_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return HS2_ERR_UNSUPPORTED;
+  if (double(s->T) * s->n_q_heads * 128.0 >= double(1ull << 40)) return HS2_ERR_UNSUPPORTED;
+  if (need_select) {
+    if (s->k_global < 0 || s->window < 1) return HS2_ERR_INVALID_ARG;
+    if (s->k_global > 2048 || s->window > 2048) return HS2_ERR_UNSUPPORTED;
+  }
+  return HS2_OK;
+}
+
+hs2_status cuda_status(cudaError_t e) {
+  return e == cudaSuccess ? HS2_OK : HS2_ERR_CUDA;
+}
+
+#define HS2_TRY(expr)                   \
+  do {                                  \
+    hs2_status st_ = (expr);            \
+    if (st_ != HS2_OK) return st_;      \
+  } while (0)
+
+#define HS2_NEED(cond)                            \
+  do {                                            \
+    if (!(cond)) return HS2_ERR_INVALID_ARG;      \
+  } while (0)
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace
+
+extern "C" {
+
+const char* hs2_status_string(hs2_status s) {
+  switch (s) {
+    case HS2_OK: return "ok";
+    case HS2_ERR_INVALID_ARG: return "invalid argument";
+    case HS2_ERR_UNSUPPORTED: return "unsupported shape";
+    case HS2_ERR_WORKSPACE: return "workspace too small";
+    case HS2_ERR_CUDA: return "CUDA error";
+    case HS2_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+uint64_t hs2_kernel_launches(void) { return g_launches.load(); }
+
+hs2_status hs2_get_device_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return HS2_ERR_CUDA;
+  unsigned v = 0;
+  v |= status_bridge(true);
+  v |= status_full_attn(true);
+  v |= status_select(true);
+  v |= status_sparse(true);
+  v |= status_decode(true);
+  if (v == ~0u) return HS2_ERR_CUDA;
+  if (v != 0) return HS2_ERR_TIMEOUT;
+  return HS2_OK;
+}
+
+size_t hs2_workspace_size(int32_t op, const hs2_shape* s, int32_t batch, int32_t d_model) {
+  (void)d_model;
+  const bool sel = op == HS2_OP_SELECT || op == HS2_OP_BLOCK_PREFILL || op == HS2_OP_BLOCK_DECODE;
+  if (check_shape(s, sel) != HS2_OK) return size_t(-1);
+  switch (op) {
+    case HS2_OP_BRIDGE:
+    case HS2_OP_FULL_ATTN:
+    case HS2_OP_SPARSE: return 0;
+    case HS2_OP_SELECT:
+    case HS2_OP_BLOCK_PREFILL:
+      return select_workspace_bytes(s->T, s->n_q_heads, s->n_kv_heads, s->k_global, s->window);
+    case HS2_OP_BLOCK_DECODE:
+      if (batch <= 0) return size_t(-1);
+      return decode_workspace_bytes(batch, s->T, s->n_q_heads, s->n_kv_heads, s->k_global,
+                                    s->window);
+  }
+  return size_t(-1);
+}
+
+hs2_status hs2_bridge_kv(const hs2_bf16* H, int32_t d_model, const hs2_bf16* W_k,
+                         const hs2_bf16* W_v, hs2_bf16* K, hs2_bf16* V, const hs2_shape* s,
+                         void* stream) {
+  HS2_TRY(check_shape(s, false));
+  HS2_NEED(H && W_k && W_v && K && V);
+  HS2_NEED(aligned16(H) && aligned16(W_k) && aligned16(W_v) && aligned16(K) && aligned16(V));
+  HS2_NEED(d_model > 0 && d_model % 64 == 0);
+  BridgeArgs a{H, W_k, W_v, K, V, s->T, d_model, s->n_kv_heads * 128};
+  return cuda_status(launch_bridge(a, static_cast<cudaStream_t>(stream)));
+}
+
+hs2_status hs2_full_attn_lse(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V,
+                             hs2_bf16* O, float* lse, const hs2_shape* s, void* stream) {
+  HS2_TRY(check_shape(s, false));
+  HS2_NEED(Q && K && V && O && lse);
+  HS2_NEED(aligned16(Q) && aligned16(K) && aligned16(V) && aligned16(O) && aligned16(lse));
+  AttnArgs a{Q, K, V, O, lse, s->T, s->n_q_heads, s->n_kv_heads, s->scale};
+  return cuda_status(launch_full_attn(a, static_cast<cudaStream_t>(stream)));
+}
+
+hs2_status hs2_select_topk(const hs2_bf16* Q, const hs2_bf16* K, const float* lse, int32_t* idx,
+                           float* kth, const hs2_shape* s, void* ws, size_t ws_bytes,
+                           void* stream) {
+  HS2_TRY(check_shape(s, true));
+  HS2_NEED(Q && K && lse && idx);
+  HS2_NEED(aligned16(Q) && aligned16(K) && aligned16(lse) && aligned16(idx));
+  HS2_NEED(kth == nullptr || aligned16(kth));
+  const size_t need =
+      select_workspace_bytes(s->T, s->n_q_heads, s->n_kv_heads, s->k_global, s->window);
+  if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws))) return HS2_ERR_WORKSPACE;
+  SelectArgs a{Q, K, lse, idx, kth, s->T, s->n_q_heads, s->n_kv_heads, s->scale,
+               s->k_global, s->window, ws, ws_bytes};
+  return cuda_status(launch_select(a, static_cast<cudaStream_t>(stream)));
+}
+
+hs2_status hs2_sparse_attn(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V,
+                           const int32_t* idx, hs2_bf16* O, float* lse, const hs2_shape* s,
+                           void* stream) {
+  HS2_TRY(check_shape(s, true));
+  HS2_NEED(Q && K && V && idx && O);
+  HS2_NEED(aligned16(Q) && aligned16(K) && aligned16(V) && aligned16(idx) && aligned16(O));
+  SparseArgs a{};
+  a.Q = Q;
+  a.K = K;
+  a.V = V;
+  a.idx = idx;
+  a.O = O;
+  a.lse = lse;
+  a.T = s->T;
+  a.Hq = s->n_q_heads;
+  a.Hkv = s->n_kv_heads;
+  a.scale = s->scale;
+  a.kw = s->k_global + s->window;
+  return cuda_status(launch_sparse(a, static_cast<cudaStream_t>(stream)));
+}
+
+hs2_status hs2_block_prefill(const hs2_bf16* H, int32_t d_model, const hs2_bf16* W_k,
+                             const hs2_bf16* W_v, hs2_bf16* K, hs2_bf16* V,
+                             const hs2_bf16* Q_full, hs2_bf16* O_full, float* lse, int32_t* idx,
+                             int32_t n_sparse, const hs2_bf16* const* Q_sparse,
+                             hs2_bf16* const* O_sparse, const hs2_shape* s, void* ws,
+                             size_t ws_bytes, void* stream) {
+  HS2_TRY(check_shape(s, true));
+  HS2_NEED(n_sparse >= 0 && (n_sparse == 0 || (Q_sparse && O_sparse)));
+  for (int l = 0; l < n_sparse; ++l) HS2_NEED(Q_sparse[l] && O_sparse[l]);
+  const size_t need =
+      select_workspace_bytes(s->T, s->n_q_heads, s->n_kv_heads, s->k_global, s->window);
+  if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws))) return HS2_ERR_WORKSPACE;
+  if (H != nullptr) HS2_TRY(hs2_bridge_kv(H, d_model, W_k, W_v, K, V, s, stream));
+  HS2_TRY(hs2_full_attn_lse(Q_full, K, V, O_full, lse, s, stream));
+  HS2_TRY(hs2_select_topk(Q_full, K, lse, idx, nullptr, s, ws, ws_bytes, stream));
+  for (int l = 0; l < n_sparse; ++l)
+    HS2_TRY(hs2_sparse_attn(Q_sparse[l], K, V, idx, O_sparse[l], nullptr, s, stream));
+  return HS2_OK;
+}
+
+hs2_status hs2_block_decode(int32_t batch, const int64_t* seq_len, const hs2_bf16* q_full,
+                            const hs2_fp8e4m3* Kc, const hs2_fp8e4m3* Vc, const float* k_scale,
+                            const float* v_scale, hs2_bf16* o_full, float* lse, int32_t* idx,
+                            int32_t n_sparse, const hs2_bf16* const* q_sparse,
+                            hs2_bf16* const* o_sparse, const hs2_shape* s, void* ws,
+                            size_t ws_bytes, void* stream) {
+  HS2_TRY(check_shape(s, true));
+  HS2_NEED(batch > 0 && seq_len && q_full && Kc && Vc && k_scale && v_scale && o_full && lse &&
+           idx);
+  HS2_NEED(aligned16(q_full) && aligned16(Kc) && aligned16(Vc) && aligned16(o_full) &&
+           aligned16(lse) && aligned16(idx));
+  HS2_NEED((reinterpret_cast<uintptr_t>(k_scale) & 3) == 0 &&
+           (reinterpret_cast<uintptr_t>(v_scale) & 3) == 0);
+  for (int b = 0; b < batch; ++b) HS2_NEED(seq_len[b] >= 1 && seq_len[b] <= s->T);
+  HS2_NEED(n_sparse >= 0 && (n_sparse == 0 || (q_sparse && o_sparse)));
+  for (int l = 0; l < n_sparse; ++l)
+    HS2_NEED(q_sparse[l] && o_sparse[l] && aligned16(q_sparse[l]) && aligned16(o_sparse[l]));
+  const size_t need = decode_workspace_bytes(batch, s->T, s->n_q_heads, s->n_kv_heads,
+                                             s->k_global, s->window);
+  if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws))) return HS2_ERR_WORKSPACE;
+  DecodeArgs a{};
+  a.B = batch;
+  a.seq_len_host = seq_len;
+  a.q = q_full;
+  a.Kc = Kc;
+  a.Vc = Vc;
+  a.ks = k_scale;
+  a.vs = v_scale;
+  a.o = o_full;
+  a.lse = lse;
+  a.idx = idx;
+  a.n_sparse = n_sparse;
+  a.qs = reinterpret_cast<const void* const*>(q_sparse);
+  a.os = reinterpret_cast<void* const*>(o_sparse);
+  a.cap = s->T;
+  a.Hq = s->n_q_heads;
+  a.Hkv = s->n_kv_heads;
+  a.scale = s->scale;
+  a.k = s->k_global;
+  a.w = s->window;
+  a.ws = ws;
+  a.ws_bytes = ws_bytes;
+  return cuda_status(launch_decode(a, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,116 @@
+// kernels.h -- host-side launch interface between the C ABI (hs2_api.cu) and
+// the kernels.  Internal to the library.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace hs2 {
+
+// counts every kernel launch of the library (hs2_kernel_launches)
+void count_launch(unsigned n = 1);
+
+// sticky device status word of each kernel file: read (and clear)
+unsigned status_bridge(bool clear);
+unsigned status_full_attn(bool clear);
+unsigned status_select(bool clear);
+unsigned status_sparse(bool clear);
+unsigned status_decode(bool clear);
+
+// Tensor maps (bf16, 128-byte swizzle, zero fill out of bounds).
+// dims/strides: x fastest; strides in bytes for dims 1.. .
+bool make_tmap_2d(CUtensorMap* map, const void* base, uint64_t dim_x, uint64_t dim_y,
+                  uint64_t stride_y, uint32_t box_x, uint32_t box_y);
+bool make_tmap_3d(CUtensorMap* map, const void* base, uint64_t dim_x, uint64_t dim_y,
+                  uint64_t dim_z, uint64_t stride_y, uint64_t stride_z, uint32_t box_x,
+                  uint32_t box_y, uint32_t box_z);
+
+// set the dynamic shared memory limit of a kernel once per device
+cudaError_t ensure_smem_attr(const void* func, int bytes);
+
+struct BridgeArgs {
+  const void* H;
+  const void* Wk;
+  const void* Wv;
+  void* K;
+  void* V;
+  int64_t T;
+  int dm;
+  int Nkv;  // n_kv_heads * 128
+};
+cudaError_t launch_bridge(const BridgeArgs& a, cudaStream_t stream);
+
+struct AttnArgs {
+  const void* Q;
+  const void* K;
+  const void* V;
+  void* O;
+  float* lse;
+  int64_t T;
+  int Hq, Hkv;
+  float scale;
+};
+cudaError_t launch_full_attn(const AttnArgs& a, cudaStream_t stream);
+
+struct SelectArgs {
+  const void* Q;
+  const void* K;
+  const float* lse;
+  int32_t* idx;
+  float* kth;
+  int64_t T;
+  int Hq, Hkv;
+  float scale;
+  int k, w;
+  void* ws;
+  size_t ws_bytes;
+};
+size_t select_workspace_bytes(int64_t T, int Hq, int Hkv, int k, int w);
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);
+
+struct SparseArgs {
+  const void* Q;
+  const void* K;
+  const void* V;
+  const int32_t* idx;
+  void* O;
+  float* lse;
+  int64_t T;  // query rows
+  int Hq, Hkv;
+  float scale;
+  int kw;     // entries per list (k + w)
+  // FP8 source (decode): codes + per-(token, head) scales; K/V above unused
+  const uint8_t* Kc;
+  const uint8_t* Vc;
+  const float* ks;
+  const float* vs;
+  int64_t cache_T;  // decode: tokens per sequence in the cache
+};
+cudaError_t launch_sparse(const SparseArgs& a, cudaStream_t stream);
+
+struct DecodeArgs {
+  int B;
+  const int64_t* seq_len_host;
+  const void* q;
+  const uint8_t* Kc;
+  const uint8_t* Vc;
+  const float* ks;
+  const float* vs;
+  void* o;
+  float* lse;
+  int32_t* idx;
+  int n_sparse;
+  const void* const* qs;
+  void* const* os;
+  int64_t cap;  // tokens per sequence in the cache
+  int Hq, Hkv;
+  float scale;
+  int k, w;
+  void* ws;
+  size_t ws_bytes;
+};
+size_t decode_workspace_bytes(int B, int64_t cap, int Hq, int Hkv, int k, int w);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+
+}  // namespace hs2

@@ -1,0 +1,87 @@
+"""The C-ABI library loads, exports every entry point include/hs2.h declares,
+and rejects bad arguments on the host before touching the GPU (CPU only)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def hs2():
+    from long_context_bridge_b200 import build
+    build.build()
+    import long_context_bridge_b200 as m
+    return m
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "hs2.h")).read()
+    return set(re.findall(r"^\s*(?:hs2_status|size_t|const char\*|uint64_t)\s+(hs2_\w+)\s*\(",
+                          text, flags=re.M))
+
+
+def test_exports_match_header(hs2):
+    decl = declared_symbols()
+    assert {"hs2_bridge_kv", "hs2_full_attn_lse", "hs2_select_topk", "hs2_sparse_attn",
+            "hs2_block_prefill", "hs2_block_decode"} <= decl
+    lib = C.CDLL(hs2.LIB_PATH)
+    for name in decl:
+        assert hasattr(lib, name), name
+    assert decl == set(hs2.EXPORTED)
+
+
+def _raw(hs2):
+    return hs2._lib
+
+
+def test_host_side_errors(hs2):
+    L = _raw(hs2)
+    ok_ptr = C.c_void_p(0x10000)
+    bad_ptr = C.c_void_p(0x10001)
+    s = hs2.Shape.make(1024, 8, 2)
+    # head_dim other than 128 is unsupported
+    s64 = hs2.Shape.make(1024, 8, 2, head_dim=64)
+    assert L.hs2_full_attn_lse(ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr, C.byref(s64), None) == hs2.ERR_UNSUPPORTED
+    # Hq not a multiple of Hkv, G = 3, G = 32
+    for hq, hkv in ((7, 2), (6, 2), (64, 2)):
+        sh = hs2.Shape.make(1024, hq, hkv)
+        assert L.hs2_full_attn_lse(ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr, C.byref(sh), None) == hs2.ERR_UNSUPPORTED
+    # null, misaligned, T <= 0
+    assert L.hs2_full_attn_lse(None, ok_ptr, ok_ptr, ok_ptr, ok_ptr, C.byref(s), None) == hs2.ERR_INVALID_ARG
+    assert L.hs2_full_attn_lse(ok_ptr, bad_ptr, ok_ptr, ok_ptr, ok_ptr, C.byref(s), None) == hs2.ERR_INVALID_ARG
+    s0 = hs2.Shape.make(0, 8, 2)
+    assert L.hs2_full_attn_lse(ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr, C.byref(s0), None) == hs2.ERR_INVALID_ARG
+    # bad selection budget
+    sk = hs2.Shape.make(1024, 8, 2, k_global=-1)
+    assert L.hs2_sparse_attn(ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr, None, C.byref(sk), None) == hs2.ERR_INVALID_ARG
+    sw = hs2.Shape.make(1024, 8, 2, window=0)
+    assert L.hs2_sparse_attn(ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr, None, C.byref(sw), None) == hs2.ERR_INVALID_ARG
+    # bridge: d_model must be a positive multiple of 64
+    assert L.hs2_bridge_kv(ok_ptr, 100, ok_ptr, ok_ptr, ok_ptr, ok_ptr, C.byref(s), None) == hs2.ERR_INVALID_ARG
+    # workspace too small for selection
+    need = hs2.workspace_size(hs2.OP_SELECT, s)
+    if need > 0:
+        assert L.hs2_select_topk(ok_ptr, ok_ptr, ok_ptr, ok_ptr, None, C.byref(s), ok_ptr,
+                                 need - 16, None) == hs2.ERR_WORKSPACE
+        assert L.hs2_select_topk(ok_ptr, ok_ptr, ok_ptr, ok_ptr, None, C.byref(s), None,
+                                 need, None) == hs2.ERR_WORKSPACE
+    # decode: sequence longer than the cache
+    lens = (C.c_int64 * 2)(10, 5000)
+    sd = hs2.Shape.make(4096, 8, 2)
+    arr = (C.c_void_p * 1)()
+    assert L.hs2_block_decode(2, lens, ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr,
+                              ok_ptr, 0, C.cast(arr, C.POINTER(C.c_void_p)),
+                              C.cast(arr, C.POINTER(C.c_void_p)), C.byref(sd), ok_ptr, 1 << 40,
+                              None) == hs2.ERR_INVALID_ARG
+    assert hs2.hs2_status_string(hs2.ERR_TIMEOUT) == "device-side wait timed out"
+
+
+def test_workspace_size_queries(hs2):
+    s = hs2.Shape.make(32768, 16, 2)
+    assert hs2.workspace_size(hs2.OP_FULL_ATTN, s) == 0
+    assert hs2.workspace_size(hs2.OP_SPARSE, s) == 0
+    with pytest.raises(hs2.HS2Error):
+        hs2.workspace_size(hs2.OP_FULL_ATTN, hs2.Shape.make(32768, 16, 2, head_dim=96))
