@@ -1,0 +1,414 @@
+#!/usr/bin/env python
+"""Benchmark of the HySparse2 cross-decoder block on B200.
+
+One step = the whole block over one 131072-token prompt (32 query / 4 KV
+heads, head_dim 128): KV bridge from H[T, 2048], needle keys planted, causal
+full attention with lse, top-1024 + recent-128 selection, and 3 sparse layers
+reusing K/V and the index list.  Inputs are seeded synthetic tensors already
+resident in HBM (H alone is 512 MiB, larger than the 126 MB L2, so no flush is
+needed between steps).  Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Multi-GPU: one process per GPU, each running an independent block (the block
+has no cross-sequence exchange), weak scaling, max time over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+CFG = synth.CONFIGS["C3"]
+METRIC = "cross-decoder block prefill tokens/s @128K"
+UNIT = "tokens/s"
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 6650.0, 1400.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# inputs (seeded, on the device)
+# ---------------------------------------------------------------------------
+def make_inputs(cfg, device):
+    T, dm, Hq, Hkv = cfg.T, cfg.d_model, cfg.n_q_heads, cfg.n_kv_heads
+    N = Hkv * 128
+    g = lambda tid, n, sd=1.0: synth.normal_bf16_torch(cfg.seed, tid, 0, n, sd, device=device)
+    H = g(synth.TID_H, T * dm).view(T, dm)
+    Wk = g(synth.TID_WK, dm * N, dm ** -0.5).view(dm, N)
+    Wv = g(synth.TID_WV, dm * N, dm ** -0.5).view(dm, N)
+    u = torch.from_numpy(synth.needle_dirs(cfg)).to(device)            # [Hkv, d] fp64
+
+    def qmix(tid):
+        out = torch.empty(T, Hq, 128, dtype=torch.bfloat16, device=device)
+        ug = u.repeat_interleave(cfg.G, 0)[None]
+        rows = 4096
+        for r0 in range(0, T, rows):
+            n = min(rows, T - r0)
+            z = synth.normals_torch(cfg.seed, tid, r0 * Hq * 128, n * Hq * 128, device).view(n, Hq, 128)
+            out[r0:r0 + n] = (0.5 * z + 0.5 * math.sqrt(128) * ug).float().bfloat16()
+        return out
+
+    Q = qmix(synth.TID_Q)
+    Qs = [qmix(synth.TID_QS0 + l) for l in range(cfg.n_sparse)]
+    pos = synth.prefill_needles(cfg)
+    nk = torch.from_numpy(synth.needle_key_bits(cfg).view(np.int16)).to(device).view(torch.bfloat16)
+    needle_rows = torch.cat([torch.from_numpy(p) for p in pos]).to(device)
+    needle_heads = torch.cat([torch.full((len(p),), g_, dtype=torch.int64) for g_, p in enumerate(pos)]).to(device)
+    return dict(H=H, Wk=Wk, Wv=Wv, Q=Q, Qs=Qs, needle_rows=needle_rows, needle_heads=needle_heads,
+                needle_vals=nk[needle_heads])
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    def __init__(self, dev_index):
+        self.dev = dev_index
+        self.samples = []
+        self.proc = None
+
+    def __enter__(self):
+        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.dev)],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 7:
+                self.samples.append(parts)
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
+        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in self.samples for i in range(4) if s[3 + i].lower() == "active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons}
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work per launch (roofline numerators)
+# ---------------------------------------------------------------------------
+def algorithmic(cfg):
+    T, Hq, Hkv, dm, k, w = cfg.T, cfg.n_q_heads, cfg.n_kv_heads, cfg.d_model, cfg.k_global, cfg.window
+    pairs = T * (T + 1) / 2
+    n_sel = np.minimum(np.arange(T) + 1, k + w).sum()
+    return {
+        "bridge_kv": ("tensor", 2.0 * T * dm * 2 * Hkv * 128),
+        "full_attn_lse": ("tensor", 4.0 * 128 * Hq * pairs),
+        "select_topk": ("tensor", 2.0 * 128 * Hq * pairs),
+        "sparse_attn": ("hbm", float(n_sel) * Hkv * 2 * 128 * 2 + T * Hq * 128 * 2 * 2),
+    }
+
+
+def traffic_from_profiles(kernel):
+    """Per-launch DRAM bytes of `kernel` from profiles/dram_traffic.txt, if the
+    capture was taken on the current source of that kernel's file."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    for line in open(path):
+        parts = line.split()
+        if len(parts) >= 4 and parts[0] == kernel and not line.startswith("#"):
+            src = os.path.join(ROOT, "long_context_bridge_b200", "csrc", parts[1])
+            h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:12] if os.path.exists(src) else ""
+            if h == parts[2]:
+                return float(parts[3])
+    return None
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the oracle on a bounded sample of the same workload
+# ---------------------------------------------------------------------------
+class OracleSample:
+    """The oracle on a bounded sample of the workload: query rows drawn
+    uniformly from [k + w, T), each taken through the whole block."""
+
+    def __init__(self, cfg):
+        import oracle
+        oracle.build()
+        self.oracle, self.cfg = oracle, cfg
+        T, Hkv = cfg.T, cfg.n_kv_heads
+        # K/V of every row a sample can attend to: the generator's N(0,1) rows
+        # (the bridge output's distribution) plus needles.  The bridge itself
+        # is timed on the sampled rows' hidden states.
+        self.K = synth.normal_bf16_np(cfg.seed, synth.TID_K, 0, T * Hkv * 128).reshape(T, Hkv, 128)
+        self.V = synth.normal_bf16_np(cfg.seed, synth.TID_V, 0, T * Hkv * 128).reshape(T, Hkv, 128)
+        synth.plant_needles_np(cfg, self.K, synth.prefill_needles(cfg))
+        self.kv = oracle.KV(self.K, self.V)
+        N = Hkv * 128
+        self.Wk = synth.normal_bf16_np(cfg.seed, synth.TID_WK, 0, cfg.d_model * N,
+                                       cfg.d_model ** -0.5).reshape(cfg.d_model, N)
+        self.Wv = synth.normal_bf16_np(cfg.seed, synth.TID_WV, 0, cfg.d_model * N,
+                                       cfg.d_model ** -0.5).reshape(cfg.d_model, N)
+
+    def run(self, n_rows, seed):
+        cfg, orc = self.cfg, self.oracle
+        rng = np.random.default_rng(seed)
+        rows = np.sort(rng.choice(np.arange(cfg.k_global + cfg.window, cfg.T), n_rows, replace=False))
+        H = np.concatenate([synth.normal_bf16_np(cfg.seed, synth.TID_H, int(r) * cfg.d_model,
+                                                 cfg.d_model)[None] for r in rows])
+        Q = synth.q_rows_np(cfg, synth.TID_Q, rows)
+        Qs = [synth.q_rows_np(cfg, synth.TID_QS0 + l, rows) for l in range(cfg.n_sparse)]
+        t0 = time.perf_counter()
+        orc.bridge(H, self.Wk)
+        orc.bridge(H, self.Wv)
+        orc.block_rows(self.kv, Q, Qs, rows, cfg.scale)
+        dt = time.perf_counter() - t0
+        # one sampled row = one token through the block; rows are uniform over
+        # [k + w, T), so their mean cost matches the prompt's mean row cost
+        return {"value": n_rows / dt, "unit": UNIT, "cores": orc.threads(), "kind": "oracle",
+                "sample": f"{n_rows} query rows drawn uniformly from [1152, 131072), each through "
+                          f"bridge + full attention + selection + 3 sparse layers; {dt:.1f} s"}
+
+
+# ---------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    cfg = CFG
+    config = {"workload": cfg.name, "T": cfg.T, "n_q_heads": cfg.n_q_heads,
+              "n_kv_heads": cfg.n_kv_heads, "head_dim": 128, "d_model": cfg.d_model,
+              "k_global": cfg.k_global, "window": cfg.window, "n_sparse": cfg.n_sparse,
+              "needles_per_kv_head": cfg.n_needles, "l2": "inputs larger than L2 (H is 512 MiB)",
+              "parallelism": f"replicas{args.gpus}"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        sampler = OracleSample(cfg)
+        vals = []
+        for s in range(args.warmup + args.steps):
+            cb = sampler.run(4, seed=100 + s)
+            if s >= args.warmup:
+                vals.append(cb["value"])
+        v = float(np.mean(vals))
+        cb["value"] = v
+        print(json.dumps({"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT,
+                          "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                          "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                          "dtype": "f64", "data": "synthetic", "config": config,
+                          "cpu_baseline": cb,
+                          "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0,
+                                  "d2h_bytes_per_step": 0}}), flush=True)
+        return
+
+    import long_context_bridge_b200 as hs2
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        pg = True
+
+    T, Hq, Hkv = cfg.T, cfg.n_q_heads, cfg.n_kv_heads
+    inp = make_inputs(cfg, dev)
+    shape = hs2.Shape.make(T, Hq, Hkv)
+    K = torch.empty(T, Hkv, 128, dtype=torch.bfloat16, device=dev)
+    V = torch.empty_like(K)
+    O = torch.empty_like(inp["Q"])
+    Os = [torch.empty_like(inp["Q"]) for _ in range(cfg.n_sparse)]
+    lse = torch.empty(T, Hq, dtype=torch.float32, device=dev)
+    idx = torch.empty(T, Hkv, cfg.k_global + cfg.window, dtype=torch.int32, device=dev)
+    ws = torch.empty(hs2.workspace_size(hs2.OP_BLOCK_PREFILL, shape), dtype=torch.uint8, device=dev)
+    nr, nh, nv = inp["needle_rows"], inp["needle_heads"], inp["needle_vals"]
+
+    names = ["bridge_kv", "full_attn_lse", "select_topk", "sparse_attn"]
+    ev = {n: [] for n in names}
+
+    def step(record=False):
+        def mark():
+            e = torch.cuda.Event(enable_timing=True)
+            e.record()
+            return e
+        e0 = mark() if record else None
+        hs2.hs2_bridge_kv(inp["H"], inp["Wk"], inp["Wv"], K, V, shape)
+        e1 = mark() if record else None
+        K[nr, nh] = nv  # planted needle keys (input recipe of the workload)
+        e2 = mark() if record else None
+        hs2.hs2_full_attn_lse(inp["Q"], K, V, O, lse, shape)
+        e3 = mark() if record else None
+        hs2.hs2_select_topk(inp["Q"], K, lse, idx, None, shape, ws)
+        e4 = mark() if record else None
+        spans = []
+        for l in range(cfg.n_sparse):
+            a = mark() if record else None
+            hs2.hs2_sparse_attn(inp["Qs"][l], K, V, idx, Os[l], None, shape)
+            b = mark() if record else None
+            spans.append((a, b))
+        if record:
+            ev["bridge_kv"].append((e0, e1))
+            ev["full_attn_lse"].append((e2, e3))
+            ev["select_topk"].append((e3, e4))
+            ev["sparse_attn"].extend(spans)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = hs2.hs2_get_device_status()
+    assert st == hs2.OK, f"device status {st}"
+
+    def barrier():
+        if pg:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+    with ClockSampler(local) as clk:
+        barrier()
+        n0 = hs2.hs2_kernel_launches()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record()
+        for _ in range(args.steps):
+            step(record=True)
+        end.record()
+        barrier()
+        n_launch = hs2.hs2_kernel_launches() - n0
+    ms = start.elapsed_time(end) / args.steps
+    if pg:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    kern_ms = {n: float(np.mean([a.elapsed_time(b) for a, b in ev[n]])) for n in names}
+    st = hs2.hs2_get_device_status()
+    assert st == hs2.OK, f"device status {st}"
+
+    # end-to-end through the public block call with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        hH = inp["H"].cpu().pin_memory()
+        hQ = inp["Q"].cpu().pin_memory()
+        hQs = [q.cpu().pin_memory() for q in inp["Qs"]]
+        hO = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+        hOs = [torch.empty(O.shape, dtype=O.dtype).pin_memory() for _ in range(cfg.n_sparse)]
+        hidx = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
+        hlse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        dH, dQ = torch.empty_like(inp["H"]), torch.empty_like(inp["Q"])
+        dQs = [torch.empty_like(inp["Q"]) for _ in range(cfg.n_sparse)]
+
+        def e2e_step():
+            dH.copy_(hH, non_blocking=True)
+            dQ.copy_(hQ, non_blocking=True)
+            for a, b in zip(dQs, hQs):
+                a.copy_(b, non_blocking=True)
+            hs2.hs2_block_prefill(dH, inp["Wk"], inp["Wv"], K, V, dQ, O, lse, idx, dQs, Os, shape, ws)
+            hO.copy_(O, non_blocking=True)
+            for a, b in zip(hOs, Os):
+                a.copy_(b, non_blocking=True)
+            hidx.copy_(idx, non_blocking=True)
+            hlse.copy_(lse, non_blocking=True)
+
+        e2e_step()
+        barrier()
+        s2, t2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record()
+        n_e2e = max(1, min(args.steps, 3))
+        for _ in range(n_e2e):
+            e2e_step()
+        t2.record()
+        barrier()
+        ms_e2e = s2.elapsed_time(t2) / n_e2e
+        if pg:
+            t = torch.tensor([ms_e2e], device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        h2d = sum(x.numel() * x.element_size() for x in [hH, hQ, *hQs])
+        d2h = sum(x.numel() * x.element_size() for x in [hO, *hOs, hidx, hlse])
+        e2e = {"value": T * world / (ms_e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
+               "note": "hs2_block_prefill (bridge inside) with pinned-host inputs and outputs; "
+                       "needles not planted on this path"}
+
+    if rank != 0:
+        if pg:
+            torch.distributed.destroy_process_group()
+        return
+
+    hbm, tfl, src = peaks()
+    work = algorithmic(cfg)
+    dom = max(names, key=lambda n: kern_ms[n])
+    bound, amount = work[dom]
+    secs = kern_ms[dom] / 1e3
+    if bound == "tensor":
+        achieved, peak, unit = amount / secs / 1e12, tfl, "TFLOP/s"
+    else:
+        achieved, peak, unit = amount / secs / 1e9, hbm, "GB/s"
+    roof = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+            "frac": achieved / peak, "traffic": traffic_from_profiles(dom),
+            "peak_source": f"{src} ({'bf16 sustained' if bound == 'tensor' else 'hbm copy'})"}
+    per_kernel = {}
+    for n in names:
+        b, a = work[n]
+        s = kern_ms[n] / 1e3
+        per_kernel[n] = {"ms": kern_ms[n],
+                         ("TFLOP/s" if b == "tensor" else "GB/s"):
+                             (a / s / 1e12) if b == "tensor" else (a / s / 1e9),
+                         "frac": ((a / s / 1e12) / tfl) if b == "tensor" else ((a / s / 1e9) / hbm)}
+    cpu = None
+    if not args.no_cpu and world == 1:
+        cpu = OracleSample(cfg).run(320, seed=5)
+    line = {"metric": METRIC, "value": T * world / (ms / 1e3), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": config, "clocks": clk.summary(), "e2e": e2e,
+            "gpu_launches": int(n_launch), "roofline": roof, "kernels": per_kernel,
+            "cpu_baseline": cpu}
+    print(json.dumps(line), flush=True)
+    if pg:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -40,10 +40,10 @@ class Shape(C.Structure):
                    int(k_global), int(window))
 
 
-def _load():
-    if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libhs2.so not built at {LIB_PATH}: run long_context_bridge_b200/build.py")
-    L = C.CDLL(LIB_PATH)
+def _load(path: str = LIB_PATH):
+    if not os.path.exists(path):
+        raise ImportError(f"libhs2.so not built at {path}: run long_context_bridge_b200/build.py")
+    L = C.CDLL(path)
     P, I32, I64, SZ = C.c_void_p, C.c_int32, C.c_int64, C.c_size_t
     SP = C.POINTER(Shape)
     PP = C.POINTER(C.c_void_p)

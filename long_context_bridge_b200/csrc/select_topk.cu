@@ -14,12 +14,16 @@
 //   warps 2-5  scorers: thread = key (TMEM lane); it reads the 128 columns of
 //              its key and sums exp2(s*scale*log2e - lse2) over each query's
 //              G heads in registers, so a query's score needs no shuffles.
-//              Passing candidates (score above the query's running threshold)
-//              are appended to a per-query buffer in ascending position order
-//              (ballot + per-warp counts).  When a buffer may overflow, one
-//              warp runs a radix select over the 64-bit key
-//              (score bits << 32 | ~j), keeps exactly the k best in place
-//              (stable, so positions stay ascending) and raises the threshold.
+//              A candidate passes when its score bucket (float bits >> 20:
+//              eighths of a binade) is at or above the query's floor; passing
+//              candidates are appended to a per-query buffer in ascending
+//              position order (ballot + per-warp counts), and a reduction
+//              barrier lets a tile with no passing candidate skip the append.
+//              A buffer about to overflow is trimmed, by one warp, to the
+//              buckets that still hold its k best (one histogram pass, one
+//              stable compaction) and the floor is raised.  At the end of the
+//              item an exact radix select over the 64-bit key
+//              (score bits << 32 | ~j) keeps the k best, still in position order.
 // Items whose every query has at most k candidates skip the scoring: all
 // candidates are selected.
 #include "common.cuh"
@@ -49,9 +53,9 @@ struct Misc {
   uint32_t tmem_slot;
   float lse2[128];          // base-2 lse of the item's 128 (query, head) rows
   uint32_t tot[2][128];     // entries in each query's buffer (by tile parity)
-  uint32_t thr[128];        // filter: keep scores with bits > thr
-  uint32_t has_thr[128];
-  uint32_t wcnt[4][128];    // per-warp pass counts of the current chunk
+  uint32_t bmin[128];       // filter: keep candidates whose score bucket >= bmin
+  uint32_t bseen[128];      // smallest bucket ever appended to each buffer
+  uint32_t wcnt[4][128];    // per-warp pass counts of the current tile
   uint32_t hist[4][256];    // per-warp radix histograms
 };
 constexpr int SMEM = OFF_MISC + int(sizeof(Misc)) + 1024;
@@ -60,70 +64,84 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int ks) {
   return sdesc_sw128(tile + (ks >> 2) * CHUNK + (ks & 3) * 32, 16, 1024);
 }
 
+// Named barrier of the 128 scorer threads; returns the OR of `pred` over them.
+__device__ __forceinline__ bool scorer_sync_or(bool pred) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+      "barrier.cta.red.or.pred q, 1, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(out)
+      : "r"(uint32_t(pred))
+      : "memory");
+  return out != 0;
+}
 __device__ __forceinline__ void scorer_sync() {
   asm volatile("bar.sync 1, 128;" ::: "memory");
 }
 
+// Score bucket: sign, exponent and 3 mantissa bits of the fp32 score (a
+// non-negative float), i.e. eighths of a binade; monotone in the score.
+__device__ __forceinline__ uint32_t bucket_of(uint32_t score_bits) { return score_bits >> 20; }
+
+// Ranking key: larger is better; equal scores rank the smaller position first.
 __device__ __forceinline__ uint64_t sel_key(uint2 v) {
   return (uint64_t(v.x) << 32) | uint64_t(~v.y);
 }
 
-// Keep the k best of buf[0..n) (n >= k) in place, in their original order.
-// Returns the score bits of the selection threshold: every kept entry has
-// score bits >= the returned value, and an entry appended later (larger j)
-// can only enter the top k if its score bits are greater.
-__device__ uint32_t warp_keep_topk(uint2* buf, uint32_t n, uint32_t k, uint32_t* hist,
-                                   int lane) {
-  uint64_t prefix = 0, mask = 0;
-  uint32_t remaining = k;
-  for (int shift = 56; shift >= 0; shift -= 8) {
-    for (int b = lane; b < 256; b += 32) hist[b] = 0;
-    __syncwarp();
-    for (uint32_t e = lane; e < n; e += 32) {
-      const uint64_t key = sel_key(buf[e]);
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
-    }
-    __syncwarp();
-    // lane l owns bins 255-8l .. 248-8l, highest first
-    uint32_t c8[8], local = 0;
+// Warp-aggregated histogram increment (one atomic per distinct bin).
+__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool active, int lane) {
+  const uint32_t act = __ballot_sync(0xffffffffu, active);
+  if (!active) return;
+  const uint32_t peers = __match_any_sync(act, bin);
+  if (lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+}
+
+// Find, scanning bins from 255 down, the bin where the running count reaches
+// `need`.  Returns the bin; `above` = entries in higher bins, `inbin` = its count.
+__device__ __forceinline__ uint32_t hist_cross(const uint32_t* hist, uint32_t need, int lane,
+                                               uint32_t& above, uint32_t& inbin) {
+  uint32_t c8[8], local = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    c8[i] = hist[255 - 8 * lane - i];
+    local += c8[i];
+  }
+  uint32_t incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  const uint32_t excl = incl - local;
+  const uint32_t bal = __ballot_sync(0xffffffffu, excl < need && need <= incl);
+  const int src = bal ? __ffs(bal) - 1 : 31;
+  uint32_t bin = 0, ab = 0, ib = 0;
+  if (lane == src) {
+    uint32_t cum = excl;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      c8[i] = hist[255 - 8 * lane - i];
-      local += c8[i];
-    }
-    uint32_t incl = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += t;
-    }
-    const uint32_t excl = incl - local;
-    const uint32_t bal = __ballot_sync(0xffffffffu, excl < remaining && remaining <= incl);
-    const int src = __ffs(bal) - 1;
-    uint32_t bin = 0, above = 0, inbin = 0;
-    if (lane == src) {
-      uint32_t cum = excl;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        if (cum + c8[i] >= remaining) {
-          bin = 255 - 8 * lane - i;
-          above = cum;
-          inbin = c8[i];
-          break;
-        }
-        cum += c8[i];
+      if (cum + c8[i] >= need) {
+        bin = 255 - 8 * lane - i;
+        ab = cum;
+        ib = c8[i];
+        break;
       }
+      cum += c8[i];
     }
-    bin = __shfl_sync(0xffffffffu, bin, src);
-    above = __shfl_sync(0xffffffffu, above, src);
-    inbin = __shfl_sync(0xffffffffu, inbin, src);
-    remaining -= above;
-    prefix |= uint64_t(bin) << shift;
-    mask |= uint64_t(0xFF) << shift;
-    __syncwarp();
-    if (inbin == remaining) break;  // the whole bucket is selected
   }
-  // stable in-place compaction of the selected entries
+  above = __shfl_sync(0xffffffffu, ab, src);
+  inbin = __shfl_sync(0xffffffffu, ib, src);
+  return __shfl_sync(0xffffffffu, bin, src);
+}
+
+__device__ __forceinline__ void hist_clear(uint32_t* hist, int lane) {
+  for (int b = lane; b < 256; b += 32) hist[b] = 0;
+  __syncwarp();
+}
+
+// Stable in-place compaction of buf[0..n): keep entries with keep(v).
+template <class Keep>
+__device__ __forceinline__ uint32_t warp_compact(uint2* buf, uint32_t n, int lane, Keep keep) {
   uint32_t out = 0;
   for (uint32_t base = 0; base < n; base += 32) {
     const uint32_t e = base + lane;
@@ -131,14 +149,93 @@ __device__ uint32_t warp_keep_topk(uint2* buf, uint32_t n, uint32_t k, uint32_t*
     bool sel = false;
     if (e < n) {
       v = buf[e];
-      sel = (sel_key(v) & mask) >= prefix;
+      sel = keep(v);
     }
     const uint32_t b = __ballot_sync(0xffffffffu, sel);
     if (sel) buf[out + __popc(b & ((1u << lane) - 1u))] = v;
     out += __popc(b);
   }
   __syncwarp();
-  return uint32_t(prefix >> 32);
+  return out;
+}
+
+// Coarse trim of a full buffer: keep the entries whose bucket is at or above
+// the highest bucket that still leaves >= k entries.  All entries have bucket
+// >= bmin.  Returns the new bucket floor; n is updated.
+__device__ uint32_t warp_trim_buckets(uint2* buf, uint32_t& n, uint32_t k, uint32_t bmin,
+                                      uint32_t* hist, int lane) {
+  hist_clear(hist, lane);
+  for (uint32_t base = 0; base < n; base += 32) {
+    const uint32_t e = base + lane;
+    uint32_t bin = 0;
+    if (e < n) bin = min(bucket_of(buf[e].x) - bmin, 255u);
+    hist_add(hist, bin, e < n, lane);
+  }
+  __syncwarp();
+  uint32_t above, inbin;
+  const uint32_t b = hist_cross(hist, k, lane, above, inbin);
+  const uint32_t floor_b = bmin + b;
+  n = warp_compact(buf, n, lane, [&](uint2 v) { return bucket_of(v.x) >= floor_b; });
+  return floor_b;
+}
+
+// Exact: keep the k best of buf[0..n) (n >= k) in place, in buffer order.
+// The first digit is the score bucket relative to bmin (entries all have
+// bucket >= bmin), then 8-bit digits of the remaining score and position bits.
+__device__ void warp_keep_topk(uint2* buf, uint32_t n, uint32_t k, uint32_t bmin, uint32_t* hist,
+                               int lane) {
+  uint64_t prefix = 0, mask = 0;
+  uint32_t remaining = k;
+  int shift;
+  // digit 1: bucket (key bits 63..52) relative to bmin
+  hist_clear(hist, lane);
+  for (uint32_t base = 0; base < n; base += 32) {
+    const uint32_t e = base + lane;
+    uint32_t bin = 0;
+    if (e < n) bin = min(bucket_of(buf[e].x) - bmin, 255u);
+    hist_add(hist, bin, e < n, lane);
+  }
+  __syncwarp();
+  {
+    uint32_t above, inbin;
+    const uint32_t b = hist_cross(hist, remaining, lane, above, inbin);
+    __syncwarp();
+    if (b < 255) {
+      prefix = uint64_t(bmin + b) << 52;
+      mask = uint64_t(0xFFF) << 52;
+      remaining -= above;
+      if (inbin == remaining) goto select;
+      shift = 44;
+    } else {
+      shift = 56;  // the crossing lies 32 binades above bmin: resolve from the top
+    }
+  }
+  for (; shift >= -4; shift -= 8) {
+    const int sh = shift < 0 ? 0 : shift;
+    const uint64_t dmask = shift < 0 ? 0xFull : 0xFFull;
+    hist_clear(hist, lane);
+    for (uint32_t base = 0; base < n; base += 32) {
+      const uint32_t e = base + lane;
+      uint32_t bin = 0;
+      bool act = false;
+      if (e < n) {
+        const uint64_t key = sel_key(buf[e]);
+        act = (key & mask) == prefix;
+        bin = uint32_t((key >> sh) & dmask);
+      }
+      hist_add(hist, bin, act, lane);
+    }
+    __syncwarp();
+    uint32_t above, inbin;
+    const uint32_t b = hist_cross(hist, remaining, lane, above, inbin);
+    __syncwarp();
+    remaining -= above;
+    prefix |= uint64_t(b) << sh;
+    mask |= dmask << sh;
+    if (inbin == remaining) break;
+  }
+select:
+  warp_compact(buf, n, lane, [&](uint2 v) { return (sel_key(v) & mask) >= prefix; });
 }
 
 template <int G>
@@ -148,7 +245,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                   float* __restrict__ kth, uint2* __restrict__ ws, int T, int Hkv, int k, int w,
                   int cap, float scale_log2) {
   constexpr int QT = TILE / G;   // queries per item
-  constexpr int QPC = 32 / G;    // queries per 32-column chunk
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -248,9 +344,15 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else {
     // -------------------------------- scorers -------------------------------
+    // queries scored per group: at least one 32-column chunk, at most 8
+    // queries (register budget) unless one chunk holds more
+    constexpr int QG = (32 / G > 8) ? 32 / G : (QT < 8 ? QT : 8);
+    constexpr int NG = QT / QG;            // groups per tile
+    constexpr int CPG = QG * G / 32;       // 32-column chunks per group
     const int sub = warp & 3;
     const int tid = threadIdx.x - 64;  // 0..127
     const uint32_t lane_addr = uint32_t(sub * 32) << 16;
+    const uint32_t lt_mask = (1u << lane) - 1u;
     uint32_t st = 0;
     bool ok = true;
     for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
@@ -263,8 +365,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (tid < QT) {
           ms->tot[0][tid] = 0;
           ms->tot[1][tid] = 0;
-          ms->thr[tid] = 0;
-          ms->has_thr[tid] = 0;
+          ms->bmin[tid] = 0;
+          ms->bseen[tid] = 0xFFFFFFFFu;
         }
       }
       scorer_sync();
@@ -274,60 +376,92 @@ __global__ void __launch_bounds__(THREADS, 1)
         ok = ok && mbar_wait(&ms->s_full[b], (st >> 1) & 1);
         tc_fence_after();
         const int j = t * TILE + sub * 32 + lane;  // this thread's key
+        // every key of the tile is a candidate of every query unless the tile
+        // reaches the window of the item's first query
+        const bool all_cand = (t + 1) * TILE - 1 + w <= q0;
+        bool need = false;  // a buffer this thread counted may overflow next tile
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_addr + b * 128 + c * 32, r);
-          tmem_wait_ld();
-          if (c == 3) {
-            tc_fence_before();
-            mbar_arrive(&ms->s_empty[b]);
+        for (int gi = 0; gi < NG; ++gi) {
+          uint32_t bal[QG];
+          float sc[QG];
+          bool any_pass = false;
+#pragma unroll
+          for (int cc = 0; cc < CPG; ++cc) {
+            const int c = gi * CPG + cc;  // chunk: columns 32c .. 32c+31
+            uint32_t r[32];
+            tmem_ld32(tmem + lane_addr + b * 128 + c * 32, r);
+            tmem_wait_ld();
+            if (gi == NG - 1 && cc == CPG - 1) {
+              tc_fence_before();
+              mbar_arrive(&ms->s_empty[b]);
+            }
+#pragma unroll
+            for (int qq = 0; qq < 32 / G; ++qq) {
+              float acc = 0.f;
+#pragma unroll
+              for (int h = 0; h < G; ++h)
+                acc += fast_exp2(fmaf(__uint_as_float(r[qq * G + h]), scale_log2,
+                                      -ms->lse2[c * 32 + qq * G + h]));
+              sc[cc * (32 / G) + qq] = acc;
+            }
           }
-          uint32_t bal[QPC];
-          float sc[QPC];
 #pragma unroll
-          for (int qq = 0; qq < QPC; ++qq) {
-            float acc = 0.f;
-#pragma unroll
-            for (int h = 0; h < G; ++h)
-              acc += fast_exp2(fmaf(__uint_as_float(r[qq * G + h]), scale_log2,
-                                    -ms->lse2[c * 32 + qq * G + h]));
-            sc[qq] = acc;
-            const int q = c * QPC + qq;
+          for (int ql = 0; ql < QG; ++ql) {
+            const int q = gi * QG + ql;
             const int qpos = q0 + q;
-            const bool cand = (j + w <= qpos) && qpos < T;
-            const uint32_t bits = __float_as_uint(acc);
-            const bool pass = cand && (!ms->has_thr[q] || bits > ms->thr[q]);
-            bal[qq] = __ballot_sync(0xffffffffu, pass);
-            if (lane == 0) ms->wcnt[sub][q] = __popc(bal[qq]);
+            const bool cand = (all_cand || j + w <= qpos) && qpos < T;
+            const bool pass = cand && bucket_of(__float_as_uint(sc[ql])) >= ms->bmin[q];
+            bal[ql] = __ballot_sync(0xffffffffu, pass);
+            if (lane == 0) ms->wcnt[sub][q] = __popc(bal[ql]);
+            any_pass |= bal[ql] != 0;
+          }
+          // append the passing candidates of this group in ascending position
+          if (scorer_sync_or(any_pass)) {
+#pragma unroll
+            for (int ql = 0; ql < QG; ++ql) {
+              const int q = gi * QG + ql;
+              if (bal[ql] == 0) continue;
+              uint32_t base = ms->tot[par][q];
+              for (int v = 0; v < sub; ++v) base += ms->wcnt[v][q];
+              if ((bal[ql] >> lane) & 1u) {
+                const uint32_t bits = __float_as_uint(sc[ql]);
+                qbuf0[size_t(q) * cap + base + __popc(bal[ql] & lt_mask)] =
+                    make_uint2(bits, uint32_t(j));
+                const uint32_t mb = __reduce_min_sync(bal[ql], bucket_of(bits));
+                if (lane == __ffs(bal[ql]) - 1) atomicMin(&ms->bseen[q], mb);
+              }
+            }
+            if (tid < QG) {
+              const int q = gi * QG + tid;
+              const uint32_t nt =
+                  ms->tot[par][q] + ms->wcnt[0][q] + ms->wcnt[1][q] + ms->wcnt[2][q] + ms->wcnt[3][q];
+              ms->tot[par ^ 1][q] = nt;
+              need |= nt > uint32_t(cap - TILE);
+            }
+          } else if (tid < QG) {
+            ms->tot[par ^ 1][gi * QG + tid] = ms->tot[par][gi * QG + tid];
+          }
+        }
+        // make room: a buffer that could overflow on the next tile is trimmed
+        // to the score buckets that still hold its k best
+        if (scorer_sync_or(need)) {
+          for (int q = sub; q < QT; q += 4) {
+            uint32_t n = ms->tot[par ^ 1][q];
+            if (n <= uint32_t(cap - TILE)) continue;
+            uint2* qb = qbuf0 + size_t(q) * cap;
+            const uint32_t base = max(ms->bmin[q], ms->bseen[q]);
+            uint32_t bm = warp_trim_buckets(qb, n, k, base, ms->hist[sub], lane);
+            if (n > uint32_t(cap + k) / 2) {  // coarse buckets: keep exactly k
+              warp_keep_topk(qb, n, k, bm, ms->hist[sub], lane);
+              n = k;
+            }
+            if (lane == 0) {
+              ms->tot[par ^ 1][q] = n;
+              ms->bmin[q] = bm;
+            }
           }
           scorer_sync();
-#pragma unroll
-          for (int qq = 0; qq < QPC; ++qq) {
-            const int q = c * QPC + qq;
-            uint32_t base = ms->tot[par][q];
-            for (int v = 0; v < sub; ++v) base += ms->wcnt[v][q];
-            if ((bal[qq] >> lane) & 1u) {
-              const uint32_t pos = base + __popc(bal[qq] & ((1u << lane) - 1u));
-              qbuf0[size_t(q) * cap + pos] = make_uint2(__float_as_uint(sc[qq]), uint32_t(j));
-            }
-            if (sub == 3 && lane == 0) ms->tot[par ^ 1][q] = base + __popc(bal[qq]);
-          }
         }
-        scorer_sync();
-        // make room: buffers that could overflow on the next tile keep their k best
-        for (int q = sub; q < QT; q += 4) {
-          const uint32_t n = ms->tot[par ^ 1][q];
-          if (n > uint32_t(cap - TILE)) {
-            const uint32_t thr = warp_keep_topk(qbuf0 + size_t(q) * cap, n, k, ms->hist[sub], lane);
-            if (lane == 0) {
-              ms->tot[par ^ 1][q] = k;
-              ms->thr[q] = thr;
-              ms->has_thr[q] = 1;
-            }
-          }
-        }
-        scorer_sync();
       }
       // ---- outputs of the item ----
       for (int q = sub; q < QT; q += 4) {
@@ -341,7 +475,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         } else {
           uint2* qb = qbuf0 + size_t(q) * cap;
           const uint32_t n = ms->tot[n_tiles & 1][q];
-          if (ok && n > uint32_t(k)) warp_keep_topk(qb, n, k, ms->hist[sub], lane);
+          if (ok && n > uint32_t(k))
+            warp_keep_topk(qb, n, k, max(ms->bmin[q], ms->bseen[q]), ms->hist[sub], lane);
           uint32_t mn = 0xFFFFFFFFu;
           for (int e = lane; e < k; e += 32) {
             const uint2 v = qb[e];
@@ -376,7 +511,7 @@ int sm_count() {
   return n > 0 ? n : 148;
 }
 
-int buffer_cap(int k) { return 2 * k + 256; }
+int buffer_cap(int k) { return 4 * k + 256; }
 
 template <int G>
 cudaError_t launch_g(const SelectArgs& a, cudaStream_t stream) {
