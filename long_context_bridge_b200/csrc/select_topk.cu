@@ -8,22 +8,32 @@
 // (equal scores: smaller j first) are kept, then the w most recent positions.
 //
 // Persistent kernel, one CTA per SM, work item = (128/G queries, KV head):
-//   warp 0     TMA: the item's Q tile once, K tiles into a 4-stage ring
+//   warp 0     TMA: the item's Q tile once, K tiles into a ring
 //   warp 1     TMEM owner; one lane issues S^T = K Q^T (M = 128 keys,
 //              N = 128 (query, head) rows) into TMEM buffer t%2
-//   warps 2-5  scorers: thread = key (TMEM lane); it reads the 128 columns of
-//              its key and sums exp2(s*scale*log2e - lse2) over each query's
-//              G heads in registers, so a query's score needs no shuffles.
-//              A candidate passes when its score bucket (float bits >> 20:
-//              eighths of a binade) is at or above the query's floor; passing
-//              candidates are appended to a per-query buffer in ascending
-//              position order (ballot + per-warp counts), and a reduction
-//              barrier lets a tile with no passing candidate skip the append.
-//              A buffer about to overflow is trimmed, by one warp, to the
-//              buckets that still hold its k best (one histogram pass, one
-//              stable compaction) and the floor is raised.  At the end of the
-//              item an exact radix select over the 64-bit key
-//              (score bits << 32 | ~j) keeps the k best, still in position order.
+//   warps 2-9  scorers, two per TMEM lane quarter: thread = key (TMEM lane);
+//              warps 2-5 take the first half of the item's queries (columns
+//              0-63), warps 6-9 the second half; a thread sums
+//              exp2(s*scale*log2e - lse2) over each query's G heads in
+//              registers, so a query's score needs no shuffles.
+// Streaming exact top-k without CTA barriers in the tile loop:
+//   * every scorer warp appends the candidates of its 32 keys to its own
+//     per-query sub-buffer (ballot order = ascending position); the four
+//     warps of a query's half hold disjoint key sets;
+//   * every append is also counted in a per-query histogram of score bins
+//     (eighths of a binade below the largest possible score G) in shared
+//     memory; whatever snapshot of it a warp reads, the highest bin with at
+//     least k appended entries at or above it bounds the k-th best score from
+//     below, so candidates in lower bins are dropped.  The bin floor is shared
+//     by the warps (atomicMax) and only rises;
+//   * a full sub-buffer drops its entries below the floor (stable), or, if
+//     that is not enough, keeps its own exact k best;
+//   * at the end of the item one warp per query selects the k best of the
+//     union of the four sub-buffers on the 64-bit key
+//     (score bits << 32 | ~position), larger score first and equal scores to
+//     the smaller position: a bin histogram fixes the k-th best's bin, radix
+//     digits resolve inside that bin only, and the chosen positions are
+//     sorted ascending by a register bitonic sort.
 // Items whose every query has at most k candidates skip the scoring: all
 // candidates are selected.
 #include "common.cuh"
@@ -35,76 +45,78 @@ HS2_STATUS_ACCESSOR(status_select)
 
 namespace {
 
-constexpr int THREADS = 192;
+constexpr int THREADS = 320;   // producer warp, MMA warp, 8 scorer warps
+constexpr int SCORERS = 256;
 constexpr int TILE = 128;
 constexpr int CHUNK = TILE * 128;
 constexpr int TILE_BYTES = 2 * CHUNK;
-constexpr int KSTAGES = 4;
 constexpr int OFF_Q = 0;
 constexpr int OFF_K = OFF_Q + TILE_BYTES;
-constexpr int OFF_MISC = OFF_K + KSTAGES * TILE_BYTES;
+constexpr int MAX_STAGES = 4;
 constexpr uint32_t IDESC = idesc_bf16(128, 128, 0, 0);
 constexpr float kLog2e = 1.4426950408889634f;
 
-struct Misc {
+template <int G>
+struct SelCfg {
+  static constexpr int QT = TILE / G;                 // queries per item
+  static constexpr int QH = QT / 2;                   // queries per scorer half
+  static constexpr int NB = QT <= 32 ? 256 : 64;      // histogram bins per query
+  static constexpr int BSHIFT = QT <= 32 ? 20 : 22;   // bin width: 2^-3 or 2^-1 binade
+  // queries scored per group: at least one 32-column chunk, at most 8
+  static constexpr int QG = (32 / G > 8) ? 32 / G : (QH < 8 ? QH : 8);
+  static constexpr int NG = QH / QG;                  // groups per tile
+  static constexpr int CPG = QG * G / 32;             // 32-column chunks per group
+};
+
+struct Bars {
   uint64_t q_full, q_empty;
-  uint64_t k_full[KSTAGES], k_empty[KSTAGES];
+  uint64_t k_full[MAX_STAGES], k_empty[MAX_STAGES];
   uint64_t s_full[2], s_empty[2];
   uint32_t tmem_slot;
-  float lse2[128];          // base-2 lse of the item's 128 (query, head) rows
-  uint32_t tot[2][128];     // entries in each query's buffer (by tile parity)
-  uint32_t bmin[128];       // filter: keep candidates whose score bucket >= bmin
-  uint32_t bseen[128];      // smallest bucket ever appended to each buffer
-  uint32_t wcnt[4][128];    // per-warp pass counts of the current tile
-  uint32_t hist[4][256];    // per-warp radix histograms
 };
-constexpr int SMEM = OFF_MISC + int(sizeof(Misc)) + 1024;
+
+template <int G>
+struct Misc {
+  static constexpr int QT = SelCfg<G>::QT, NB = SelCfg<G>::NB;
+  Bars bars;
+  float lse2[128];            // base-2 lse of the item's 128 (query, head) rows
+  uint32_t floor_bin[QT];     // candidates need bin >= floor_bin
+  uint32_t cnt[4][QT];        // entries in each sub-buffer
+  uint32_t hist[QT][NB];      // appended entries per score bin
+  uint32_t dig[8][256];       // per-warp radix histograms of the final select
+};
 
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int ks) {
   return sdesc_sw128(tile + (ks >> 2) * CHUNK + (ks & 3) * 32, 16, 1024);
 }
 
-// Named barrier of the 128 scorer threads; returns the OR of `pred` over them.
-__device__ __forceinline__ bool scorer_sync_or(bool pred) {
-  uint32_t out;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-      "barrier.cta.red.or.pred q, 1, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(out)
-      : "r"(uint32_t(pred))
-      : "memory");
-  return out != 0;
-}
 __device__ __forceinline__ void scorer_sync() {
-  asm volatile("bar.sync 1, 128;" ::: "memory");
+  asm volatile("bar.sync 1, 256;" ::: "memory");
 }
-
-// Score bucket: sign, exponent and 3 mantissa bits of the fp32 score (a
-// non-negative float), i.e. eighths of a binade; monotone in the score.
-__device__ __forceinline__ uint32_t bucket_of(uint32_t score_bits) { return score_bits >> 20; }
 
 // Ranking key: larger is better; equal scores rank the smaller position first.
 __device__ __forceinline__ uint64_t sel_key(uint2 v) {
   return (uint64_t(v.x) << 32) | uint64_t(~v.y);
 }
 
-// Warp-aggregated histogram increment (one atomic per distinct bin).
-__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool active, int lane) {
-  const uint32_t act = __ballot_sync(0xffffffffu, active);
-  if (!active) return;
-  const uint32_t peers = __match_any_sync(act, bin);
-  if (lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+template <int NB, int BSHIFT>
+__device__ __forceinline__ uint32_t bin_of(uint32_t score_bits, uint32_t lo) {
+  const uint32_t bk = score_bits >> BSHIFT;
+  return bk >= lo ? min(bk - lo, uint32_t(NB - 1)) : 0u;
 }
 
-// Find, scanning bins from 255 down, the bin where the running count reaches
-// `need`.  Returns the bin; `above` = entries in higher bins, `inbin` = its count.
-__device__ __forceinline__ uint32_t hist_cross(const uint32_t* hist, uint32_t need, int lane,
-                                               uint32_t& above, uint32_t& inbin) {
-  uint32_t c8[8], local = 0;
+// Scan bins from the top: the bin where the running count reaches `need`;
+// `above` = count in higher bins, `inbin` = its own count.  -1 when the total
+// is below `need`.
+template <int NB>
+__device__ __forceinline__ int hist_cross(const uint32_t* hist, uint32_t need, int lane,
+                                          uint32_t& above, uint32_t& inbin) {
+  constexpr int PER = NB / 32;
+  uint32_t c[PER], local = 0;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    c8[i] = hist[255 - 8 * lane - i];
-    local += c8[i];
+  for (int i = 0; i < PER; ++i) {
+    c[i] = hist[NB - 1 - PER * lane - i];
+    local += c[i];
   }
   uint32_t incl = local;
 #pragma unroll
@@ -114,19 +126,25 @@ __device__ __forceinline__ uint32_t hist_cross(const uint32_t* hist, uint32_t ne
   }
   const uint32_t excl = incl - local;
   const uint32_t bal = __ballot_sync(0xffffffffu, excl < need && need <= incl);
-  const int src = bal ? __ffs(bal) - 1 : 31;
-  uint32_t bin = 0, ab = 0, ib = 0;
+  if (bal == 0) {
+    above = __shfl_sync(0xffffffffu, incl, 31);
+    inbin = 0;
+    return -1;
+  }
+  const int src = __ffs(bal) - 1;
+  int bin = 0;
+  uint32_t ab = 0, ib = 0;
   if (lane == src) {
     uint32_t cum = excl;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (cum + c8[i] >= need) {
-        bin = 255 - 8 * lane - i;
+    for (int i = 0; i < PER; ++i) {
+      if (cum + c[i] >= need) {
+        bin = NB - 1 - PER * lane - i;
         ab = cum;
-        ib = c8[i];
+        ib = c[i];
         break;
       }
-      cum += c8[i];
+      cum += c[i];
     }
   }
   above = __shfl_sync(0xffffffffu, ab, src);
@@ -134,9 +152,25 @@ __device__ __forceinline__ uint32_t hist_cross(const uint32_t* hist, uint32_t ne
   return __shfl_sync(0xffffffffu, bin, src);
 }
 
-__device__ __forceinline__ void hist_clear(uint32_t* hist, int lane) {
-  for (int b = lane; b < 256; b += 32) hist[b] = 0;
-  __syncwarp();
+// Apply fn(entry, valid) to every entry of up to four lists, eight loads in
+// flight per lane.  The lane-to-entry map is the same on every call.
+template <class Fn>
+__device__ __forceinline__ void for_each_entry(uint2* const* sub, const uint32_t* n, int lane,
+                                               Fn fn) {
+  for (int w = 0; w < 4; ++w) {
+    const uint2* b = sub[w];
+    const uint32_t nw = n[w];
+    for (uint32_t base = 0; base < nw; base += 256) {
+      uint2 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const uint32_t e = base + u * 32 + lane;
+        v[u] = e < nw ? b[e] : make_uint2(0u, 0xFFFFFFFFu);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) fn(v[u], base + u * 32 + lane < nw, w);
+    }
+  }
 }
 
 // Stable in-place compaction of buf[0..n): keep entries with keep(v).
@@ -159,100 +193,113 @@ __device__ __forceinline__ uint32_t warp_compact(uint2* buf, uint32_t n, int lan
   return out;
 }
 
-// Coarse trim of a full buffer: keep the entries whose bucket is at or above
-// the highest bucket that still leaves >= k entries.  All entries have bucket
-// >= bmin.  Returns the new bucket floor; n is updated.
-__device__ uint32_t warp_trim_buckets(uint2* buf, uint32_t& n, uint32_t k, uint32_t bmin,
-                                      uint32_t* hist, int lane) {
-  hist_clear(hist, lane);
-  for (uint32_t base = 0; base < n; base += 32) {
-    const uint32_t e = base + lane;
-    uint32_t bin = 0;
-    if (e < n) bin = min(bucket_of(buf[e].x) - bmin, 255u);
-    hist_add(hist, bin, e < n, lane);
-  }
-  __syncwarp();
-  uint32_t above, inbin;
-  const uint32_t b = hist_cross(hist, k, lane, above, inbin);
-  const uint32_t floor_b = bmin + b;
-  n = warp_compact(buf, n, lane, [&](uint2 v) { return bucket_of(v.x) >= floor_b; });
-  return floor_b;
-}
-
-// Exact: keep the k best of buf[0..n) (n >= k) in place, in buffer order.
-// The first digit is the score bucket relative to bmin (entries all have
-// bucket >= bmin), then 8-bit digits of the remaining score and position bits.
-__device__ void warp_keep_topk(uint2* buf, uint32_t n, uint32_t k, uint32_t bmin, uint32_t* hist,
-                               int lane) {
+// Exact selection over up to four lists (total >= k): (prefix, mask) such
+// that exactly the k entries with (key & mask) >= prefix are the k best.
+// Digit 1 is the score bin; when that bin is exact, later digits only look at
+// the entries inside it.
+template <int NB, int BSHIFT>
+__device__ void radix_select(uint2* const* sub, const uint32_t* n, uint32_t k, uint32_t lo,
+                             uint32_t* hist, int lane, uint64_t& prefix_out,
+                             uint64_t& mask_out) {
   uint64_t prefix = 0, mask = 0;
   uint32_t remaining = k;
-  int shift;
-  // digit 1: bucket (key bits 63..52) relative to bmin
-  hist_clear(hist, lane);
-  for (uint32_t base = 0; base < n; base += 32) {
-    const uint32_t e = base + lane;
-    uint32_t bin = 0;
-    if (e < n) bin = min(bucket_of(buf[e].x) - bmin, 255u);
-    hist_add(hist, bin, e < n, lane);
-  }
+  int shift = 56;
+  for (int b = lane; b < NB; b += 32) hist[b] = 0;
+  __syncwarp();
+  for_each_entry(sub, n, lane, [&](uint2 v, bool act, int) {
+    if (act) atomicAdd(&hist[bin_of<NB, BSHIFT>(v.x, lo)], 1u);
+  });
   __syncwarp();
   {
     uint32_t above, inbin;
-    const uint32_t b = hist_cross(hist, remaining, lane, above, inbin);
+    const int b = hist_cross<NB>(hist, remaining, lane, above, inbin);
     __syncwarp();
-    if (b < 255) {
-      prefix = uint64_t(bmin + b) << 52;
-      mask = uint64_t(0xFFF) << 52;
+    if (b > 0 && b < NB - 1) {  // an exact bucket: key bits 63 .. 32+BSHIFT
+      prefix = uint64_t(lo + b) << (32 + BSHIFT);
+      mask = ~uint64_t(0) << (32 + BSHIFT);
       remaining -= above;
-      if (inbin == remaining) goto select;
-      shift = 44;
-    } else {
-      shift = 56;  // the crossing lies 32 binades above bmin: resolve from the top
+      shift = (inbin == remaining) ? -100 : 32 + BSHIFT - 8;
     }
   }
-  for (; shift >= -4; shift -= 8) {
+  for (; shift > -8; shift -= 8) {
     const int sh = shift < 0 ? 0 : shift;
-    const uint64_t dmask = shift < 0 ? 0xFull : 0xFFull;
-    hist_clear(hist, lane);
-    for (uint32_t base = 0; base < n; base += 32) {
-      const uint32_t e = base + lane;
-      uint32_t bin = 0;
-      bool act = false;
-      if (e < n) {
-        const uint64_t key = sel_key(buf[e]);
-        act = (key & mask) == prefix;
-        bin = uint32_t((key >> sh) & dmask);
-      }
-      hist_add(hist, bin, act, lane);
-    }
+    const uint32_t width = shift < 0 ? 8 + shift : 8;
+    const uint64_t dmask = (uint64_t(1) << width) - 1;
+    for (int b = lane; b < 256; b += 32) hist[b] = 0;
+    __syncwarp();
+    for_each_entry(sub, n, lane, [&](uint2 v, bool act, int) {
+      const uint64_t key = sel_key(v);
+      if (act && (key & mask) == prefix) atomicAdd(&hist[uint32_t((key >> sh) & dmask)], 1u);
+    });
     __syncwarp();
     uint32_t above, inbin;
-    const uint32_t b = hist_cross(hist, remaining, lane, above, inbin);
+    const int b = hist_cross<256>(hist, remaining, lane, above, inbin);
     __syncwarp();
     remaining -= above;
     prefix |= uint64_t(b) << sh;
     mask |= dmask << sh;
     if (inbin == remaining) break;
   }
-select:
-  warp_compact(buf, n, lane, [&](uint2 v) { return (sel_key(v) & mask) >= prefix; });
+  prefix_out = prefix;
+  mask_out = mask;
+}
+
+// Ascending bitonic sort of 1024 values held as v[r] of lane l = element
+// r * 32 + l.  Strides below 32 cross lanes (shuffles), larger ones cross
+// registers of one lane.
+__device__ __forceinline__ void warp_sort1024(uint32_t (&v)[32], int lane) {
+#pragma unroll
+  for (int size = 2; size <= 1024; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      if (stride < 32) {
+#pragma unroll
+        for (int r = 0; r < 32; ++r) {
+          const uint32_t o = __shfl_xor_sync(0xffffffffu, v[r], stride);
+          const int i = r * 32 + lane;
+          const bool up = (i & size) == 0;
+          const bool lower = (lane & stride) == 0;
+          v[r] = (lower == up) ? min(v[r], o) : max(v[r], o);
+        }
+      } else {
+        const int rs = stride >> 5;
+#pragma unroll
+        for (int r = 0; r < 32; ++r) {
+          if (r & rs) continue;
+          const int i = r * 32 + lane;
+          const bool up = (i & size) == 0;
+          const uint32_t a = v[r], b = v[r + rs];
+          const bool sw = (a > b) == up;
+          v[r] = sw ? b : a;
+          v[r + rs] = sw ? a : b;
+        }
+      }
+    }
+  }
 }
 
 template <int G>
 __global__ void __launch_bounds__(THREADS, 1)
     select_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const float* __restrict__ lse, int32_t* __restrict__ idx,
-                  float* __restrict__ kth, uint2* __restrict__ ws, int T, int Hkv, int k, int w,
-                  int cap, float scale_log2) {
-  constexpr int QT = TILE / G;   // queries per item
+                  float* __restrict__ kth, uint2* __restrict__ ws, uint32_t* __restrict__ wsort,
+                  int T, int Hkv, int k, int w, int capw, int kst, float scale_log2) {
+  using Cfg = SelCfg<G>;
+  constexpr int QT = Cfg::QT, QH = Cfg::QH, NB = Cfg::NB, BSHIFT = Cfg::BSHIFT;
+  constexpr int QG = Cfg::QG, NG = Cfg::NG, CPG = Cfg::CPG;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  Misc* ms = reinterpret_cast<Misc*>(smem + OFF_MISC);
+  Misc<G>* ms = reinterpret_cast<Misc<G>*>(smem + OFF_K + kst * TILE_BYTES);
+  Bars* br = &ms->bars;
   const int warp = warp_id(), lane = lane_id();
   const int Hq = Hkv * G;
   const int nqb = (T + QT - 1) / QT;
   const int n_items = nqb * Hkv;
+  // score bins: bucket (bits >> BSHIFT) relative to lo; the top bin holds the
+  // largest possible score G, bin 0 everything NB-1 bins and more below it
+  const uint32_t top = __float_as_uint(float(G)) >> BSHIFT;
+  const uint32_t lo = top - (NB - 1);
 
   auto item = [&](int it, int& q0, int& g, int& n_tiles, bool& score) {
     const int qb = nqb - 1 - it / Hkv;  // heaviest items first
@@ -264,25 +311,25 @@ __global__ void __launch_bounds__(THREADS, 1)
   };
 
   if (threadIdx.x == 0) {
-    mbar_init(&ms->q_full, 1);
-    mbar_init(&ms->q_empty, 1);
-    for (int s = 0; s < KSTAGES; ++s) {
-      mbar_init(&ms->k_full[s], 1);
-      mbar_init(&ms->k_empty[s], 1);
+    mbar_init(&br->q_full, 1);
+    mbar_init(&br->q_empty, 1);
+    for (int s = 0; s < kst; ++s) {
+      mbar_init(&br->k_full[s], 1);
+      mbar_init(&br->k_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&ms->s_full[b], 1);
-      mbar_init(&ms->s_empty[b], 128);
+      mbar_init(&br->s_full[b], 1);
+      mbar_init(&br->s_empty[b], SCORERS);
     }
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(&ms->tmem_slot, 256);
+    tmem_alloc(&br->tmem_slot, 256);
     tc_fence_before();
   }
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = ms->tmem_slot;
+  const uint32_t tmem = br->tmem_slot;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -296,19 +343,19 @@ __global__ void __launch_bounds__(THREADS, 1)
         bool score;
         item(it, q0, g, n_tiles, score);
         if (!score) continue;
-        if (qn > 0 && !mbar_wait(&ms->q_empty, (qn - 1) & 1)) { ok = false; break; }
-        mbar_arrive_expect_tx(&ms->q_full, TILE_BYTES);
+        if (qn > 0 && !mbar_wait(&br->q_empty, (qn - 1) & 1)) { ok = false; break; }
+        mbar_arrive_expect_tx(&br->q_full, TILE_BYTES);
         for (int c = 0; c < 2; ++c)
-          tma_load_3d(smem + OFF_Q + c * CHUNK, &tmQ, &ms->q_full, c * 64, g * G, q0);
+          tma_load_3d(smem + OFF_Q + c * CHUNK, &tmQ, &br->q_full, c * 64, g * G, q0);
         for (int t = 0; t < n_tiles; ++t, ++kt) {
-          const int s = kt % KSTAGES;
-          if (kt >= KSTAGES && !mbar_wait(&ms->k_empty[s], ((kt / KSTAGES) & 1) ^ 1)) {
+          const int s = kt % kst;
+          if (kt >= uint32_t(kst) && !mbar_wait(&br->k_empty[s], ((kt / kst) & 1) ^ 1)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&ms->k_full[s], TILE_BYTES);
+          mbar_arrive_expect_tx(&br->k_full[s], TILE_BYTES);
           for (int c = 0; c < 2; ++c)
-            tma_load_3d(smem + OFF_K + s * TILE_BYTES + c * CHUNK, &tmK, &ms->k_full[s], c * 64,
+            tma_load_3d(smem + OFF_K + s * TILE_BYTES + c * CHUNK, &tmK, &br->k_full[s], c * 64,
                         g, t * TILE);
         }
         ++qn;
@@ -325,75 +372,67 @@ __global__ void __launch_bounds__(THREADS, 1)
         bool score;
         item(it, q0, g, n_tiles, score);
         if (!score) continue;
-        if (!mbar_wait(&ms->q_full, qn & 1)) { ok = false; break; }
+        if (!mbar_wait(&br->q_full, qn & 1)) { ok = false; break; }
         for (int t = 0; t < n_tiles; ++t, ++kt, ++st) {
-          const int s = kt % KSTAGES, b = st & 1;
-          if (!mbar_wait(&ms->k_full[s], (kt / KSTAGES) & 1)) { ok = false; break; }
-          if (st >= 2 && !mbar_wait(&ms->s_empty[b], ((st >> 1) & 1) ^ 1)) { ok = false; break; }
+          const int s = kt % kst, b = st & 1;
+          if (!mbar_wait(&br->k_full[s], (kt / kst) & 1)) { ok = false; break; }
+          if (st >= 2 && !mbar_wait(&br->s_empty[b], ((st >> 1) & 1) ^ 1)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sK = smem_u32(smem + OFF_K + s * TILE_BYTES);
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks)
             mma_ss(tmem + b * 128, kmajor_desc(sK, ks), kmajor_desc(sQ, ks), IDESC, ks > 0);
-          mma_commit(&ms->s_full[b]);
-          mma_commit(&ms->k_empty[s]);
+          mma_commit(&br->s_full[b]);
+          mma_commit(&br->k_empty[s]);
         }
-        mma_commit(&ms->q_empty);
+        mma_commit(&br->q_empty);
         ++qn;
       }
     }
   } else {
     // -------------------------------- scorers -------------------------------
-    // queries scored per group: at least one 32-column chunk, at most 8
-    // queries (register budget) unless one chunk holds more
-    constexpr int QG = (32 / G > 8) ? 32 / G : (QT < 8 ? QT : 8);
-    constexpr int NG = QT / QG;            // groups per tile
-    constexpr int CPG = QG * G / 32;       // 32-column chunks per group
-    const int sub = warp & 3;
-    const int tid = threadIdx.x - 64;  // 0..127
+    const int sw = warp - 2;          // scorer warp 0..7
+    const int half = sw >> 2;         // which half of the item's queries
+    const int sub = warp & 3;         // TMEM lane quarter = key quarter of a tile
+    const int tid = threadIdx.x - 64; // 0..255
     const uint32_t lane_addr = uint32_t(sub * 32) << 16;
     const uint32_t lt_mask = (1u << lane) - 1u;
+    uint2* my_bufs = ws + (size_t(blockIdx.x) * 4 + sub) * QT * capw;  // [QT][capw]
     uint32_t st = 0;
     bool ok = true;
     for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
       int q0, g, n_tiles;
       bool score;
       item(it, q0, g, n_tiles, score);
-      {
+      if (tid < 128) {
         const int qrow = q0 + tid / G;
         ms->lse2[tid] = qrow < T ? lse[size_t(qrow) * Hq + g * G + tid % G] * kLog2e : INFINITY;
-        if (tid < QT) {
-          ms->tot[0][tid] = 0;
-          ms->tot[1][tid] = 0;
-          ms->bmin[tid] = 0;
-          ms->bseen[tid] = 0xFFFFFFFFu;
-        }
       }
+      for (int i = tid; i < QT; i += SCORERS) {
+        ms->floor_bin[i] = 0;
+        ms->cnt[0][i] = ms->cnt[1][i] = ms->cnt[2][i] = ms->cnt[3][i] = 0;
+      }
+      for (int i = tid; i < QT * NB; i += SCORERS) (&ms->hist[0][0])[i] = 0;
       scorer_sync();
-      uint2* qbuf0 = ws + size_t(blockIdx.x) * QT * cap;
       for (int t = 0; t < n_tiles; ++t, ++st) {
-        const int b = st & 1, par = t & 1;
-        ok = ok && mbar_wait(&ms->s_full[b], (st >> 1) & 1);
+        const int b = st & 1;
+        ok = ok && mbar_wait(&br->s_full[b], (st >> 1) & 1);
         tc_fence_after();
         const int j = t * TILE + sub * 32 + lane;  // this thread's key
-        // every key of the tile is a candidate of every query unless the tile
-        // reaches the window of the item's first query
         const bool all_cand = (t + 1) * TILE - 1 + w <= q0;
-        bool need = false;  // a buffer this thread counted may overflow next tile
 #pragma unroll 1
         for (int gi = 0; gi < NG; ++gi) {
-          uint32_t bal[QG];
+          const int qb0 = half * QH + gi * QG;  // first query of the group
           float sc[QG];
-          bool any_pass = false;
 #pragma unroll
           for (int cc = 0; cc < CPG; ++cc) {
-            const int c = gi * CPG + cc;  // chunk: columns 32c .. 32c+31
+            const int c = qb0 * G / 32 + cc;  // chunk: columns 32c .. 32c+31
             uint32_t r[32];
             tmem_ld32(tmem + lane_addr + b * 128 + c * 32, r);
             tmem_wait_ld();
             if (gi == NG - 1 && cc == CPG - 1) {
               tc_fence_before();
-              mbar_arrive(&ms->s_empty[b]);
+              mbar_arrive(&br->s_empty[b]);
             }
 #pragma unroll
             for (int qq = 0; qq < 32 / G; ++qq) {
@@ -405,66 +444,72 @@ __global__ void __launch_bounds__(THREADS, 1)
               sc[cc * (32 / G) + qq] = acc;
             }
           }
+          uint32_t bal[QG], binv[QG], anymask = 0;
 #pragma unroll
           for (int ql = 0; ql < QG; ++ql) {
-            const int q = gi * QG + ql;
+            const int q = qb0 + ql;
             const int qpos = q0 + q;
-            const bool cand = (all_cand || j + w <= qpos) && qpos < T;
-            const bool pass = cand && bucket_of(__float_as_uint(sc[ql])) >= ms->bmin[q];
+            binv[ql] = bin_of<NB, BSHIFT>(__float_as_uint(sc[ql]), lo);
+            const bool pass =
+                (all_cand || j + w <= qpos) && qpos < T && binv[ql] >= ms->floor_bin[q];
             bal[ql] = __ballot_sync(0xffffffffu, pass);
-            if (lane == 0) ms->wcnt[sub][q] = __popc(bal[ql]);
-            any_pass |= bal[ql] != 0;
+            anymask |= uint32_t(bal[ql] != 0) << ql;
           }
-          // append the passing candidates of this group in ascending position
-          if (scorer_sync_or(any_pass)) {
+          if (anymask == 0) continue;
+          uint32_t n[QG];
 #pragma unroll
-            for (int ql = 0; ql < QG; ++ql) {
-              const int q = gi * QG + ql;
-              if (bal[ql] == 0) continue;
-              uint32_t base = ms->tot[par][q];
-              for (int v = 0; v < sub; ++v) base += ms->wcnt[v][q];
-              if ((bal[ql] >> lane) & 1u) {
-                const uint32_t bits = __float_as_uint(sc[ql]);
-                qbuf0[size_t(q) * cap + base + __popc(bal[ql] & lt_mask)] =
-                    make_uint2(bits, uint32_t(j));
-                const uint32_t mb = __reduce_min_sync(bal[ql], bucket_of(bits));
-                if (lane == __ffs(bal[ql]) - 1) atomicMin(&ms->bseen[q], mb);
-              }
+          for (int ql = 0; ql < QG; ++ql) n[ql] = ms->cnt[sub][qb0 + ql];
+#pragma unroll
+          for (int ql = 0; ql < QG; ++ql) {
+            if (!((anymask >> ql) & 1u) || n[ql] + 32 <= uint32_t(capw)) continue;
+            // make room: drop entries below the current floor, else keep the
+            // sub-buffer's own k best (they contain its part of the top k)
+            const int q = qb0 + ql;
+            uint2* buf = my_bufs + size_t(q) * capw;
+            const uint32_t fl = ms->floor_bin[q];
+            n[ql] = warp_compact(buf, n[ql], lane,
+                                 [&](uint2 v) { return bin_of<NB, BSHIFT>(v.x, lo) >= fl; });
+            if (n[ql] + 32 > uint32_t(capw) / 2 + k / 2 && n[ql] > uint32_t(k)) {
+              uint2* one[4] = {buf, buf, buf, buf};
+              const uint32_t nn[4] = {n[ql], 0, 0, 0};
+              uint64_t pf, mk;
+              radix_select<NB, BSHIFT>(one, nn, k, lo, ms->dig[sw], lane, pf, mk);
+              n[ql] = warp_compact(buf, n[ql], lane,
+                                   [&](uint2 v) { return (sel_key(v) & mk) >= pf; });
             }
-            if (tid < QG) {
-              const int q = gi * QG + tid;
-              const uint32_t nt =
-                  ms->tot[par][q] + ms->wcnt[0][q] + ms->wcnt[1][q] + ms->wcnt[2][q] + ms->wcnt[3][q];
-              ms->tot[par ^ 1][q] = nt;
-              need |= nt > uint32_t(cap - TILE);
-            }
-          } else if (tid < QG) {
-            ms->tot[par ^ 1][gi * QG + tid] = ms->tot[par][gi * QG + tid];
           }
+          // append in position order; count the appends per score bin
+#pragma unroll
+          for (int ql = 0; ql < QG; ++ql) {
+            if ((bal[ql] >> lane) & 1u) {
+              const int q = qb0 + ql;
+              my_bufs[size_t(q) * capw + n[ql] + __popc(bal[ql] & lt_mask)] =
+                  make_uint2(__float_as_uint(sc[ql]), uint32_t(j));
+              atomicAdd(&ms->hist[q][binv[ql]], 1u);
+            }
+          }
+          __syncwarp();
+          if (lane == 0) {
+#pragma unroll
+            for (int ql = 0; ql < QG; ++ql) ms->cnt[sub][qb0 + ql] = n[ql] + __popc(bal[ql]);
+          }
+          __syncwarp();
         }
-        // make room: a buffer that could overflow on the next tile is trimmed
-        // to the score buckets that still hold its k best
-        if (scorer_sync_or(need)) {
-          for (int q = sub; q < QT; q += 4) {
-            uint32_t n = ms->tot[par ^ 1][q];
-            if (n <= uint32_t(cap - TILE)) continue;
-            uint2* qb = qbuf0 + size_t(q) * cap;
-            const uint32_t base = max(ms->bmin[q], ms->bseen[q]);
-            uint32_t bm = warp_trim_buckets(qb, n, k, base, ms->hist[sub], lane);
-            if (n > uint32_t(cap + k) / 2) {  // coarse buckets: keep exactly k
-              warp_keep_topk(qb, n, k, bm, ms->hist[sub], lane);
-              n = k;
-            }
-            if (lane == 0) {
-              ms->tot[par ^ 1][q] = n;
-              ms->bmin[q] = bm;
-            }
+        // raise the floors of this warp's queries to the highest bin with at
+        // least k appended entries at or above it (any snapshot of the counts
+        // gives a valid floor)
+        if ((t & 1) || t == n_tiles - 1) {
+          for (int q = half * QH + sub; q < (half + 1) * QH; q += 4) {
+            uint32_t above, inbin;
+            const int fb = hist_cross<NB>(ms->hist[q], uint32_t(k), lane, above, inbin);
+            if (fb > 0 && lane == 0) atomicMax(&ms->floor_bin[q], uint32_t(fb));
           }
-          scorer_sync();
         }
       }
-      // ---- outputs of the item ----
-      for (int q = sub; q < QT; q += 4) {
+      scorer_sync();
+      // ---- outputs of the item: one warp per query ----
+      uint32_t* sp = wsort + (size_t(blockIdx.x) * 8 + sw) * 2048;  // staging of positions
+      for (int q = sw; q < QT; q += 8) {
         const int qpos = q0 + q;
         if (qpos >= T) continue;
         const int ncand = max(0, qpos - w + 1);
@@ -473,19 +518,72 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!score || ncand <= k) {
           for (int e = lane; e < k; e += 32) out[e] = e < ncand ? e : -1;
         } else {
-          uint2* qb = qbuf0 + size_t(q) * cap;
-          const uint32_t n = ms->tot[n_tiles & 1][q];
-          if (ok && n > uint32_t(k))
-            warp_keep_topk(qb, n, k, max(ms->bmin[q], ms->bseen[q]), ms->hist[sub], lane);
-          uint32_t mn = 0xFFFFFFFFu;
-          for (int e = lane; e < k; e += 32) {
-            const uint2 v = qb[e];
-            out[e] = int32_t(v.y);
-            mn = min(mn, v.x);
+          uint2* sb[4];
+          uint32_t nb[4];
+          for (int v = 0; v < 4; ++v) {
+            sb[v] = ws + ((size_t(blockIdx.x) * 4 + v) * QT + q) * capw;
+            nb[v] = ms->cnt[v][q];
+          }
+          uint64_t pf = 0, mk = 0;
+          if (ok) radix_select<NB, BSHIFT>(sb, nb, k, lo, ms->dig[sw], lane, pf, mk);
+          // gather the chosen positions (each list is in position order)
+          uint32_t got = 0, mn = 0xFFFFFFFFu;
+          for (int v = 0; v < 4; ++v) {
+            for (uint32_t base = 0; base < nb[v]; base += 32) {
+              const uint32_t e = base + lane;
+              uint2 x = make_uint2(0u, 0u);
+              bool sel = false;
+              if (e < nb[v]) {
+                x = sb[v][e];
+                sel = (sel_key(x) & mk) >= pf;
+              }
+              const uint32_t bb = __ballot_sync(0xffffffffu, sel);
+              const uint32_t pos = got + __popc(bb & lt_mask);
+              if (sel && pos < uint32_t(k)) {
+                sp[pos] = x.y;
+                mn = min(mn, x.x);
+              }
+              got += __popc(bb);
+            }
+          }
+          got = min(got, uint32_t(k));
+          __syncwarp();
+          if (k <= 1024) {
+            uint32_t v[32];
+#pragma unroll
+            for (int r = 0; r < 32; ++r) {
+              const int e = r * 32 + lane;
+              v[r] = e < int(got) ? sp[e] : 0xFFFFFFFFu;
+            }
+            warp_sort1024(v, lane);
+#pragma unroll
+            for (int r = 0; r < 32; ++r) {
+              const int e = r * 32 + lane;
+              if (e < k) out[e] = e < int(got) ? int32_t(v[r]) : -1;
+            }
+          } else {
+            // k in (1024, 2048]: bitonic sort of the staging buffer
+            for (int e = got + lane; e < 2048; e += 32) sp[e] = 0xFFFFFFFFu;
+            __syncwarp();
+            for (int size = 2; size <= 2048; size <<= 1)
+              for (int stride = size >> 1; stride > 0; stride >>= 1) {
+                for (int i = lane; i < 1024; i += 32) {
+                  const int a0 = 2 * stride * (i / stride) + (i % stride), a1 = a0 + stride;
+                  const bool up = (a0 & size) == 0;
+                  const uint32_t x0 = sp[a0], x1 = sp[a1];
+                  if ((x0 > x1) == up) {
+                    sp[a0] = x1;
+                    sp[a1] = x0;
+                  }
+                }
+                __syncwarp();
+              }
+            for (int e = lane; e < k; e += 32) out[e] = e < int(got) ? int32_t(sp[e]) : -1;
           }
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
           kv = __uint_as_float(mn);
+          __syncwarp();
         }
         for (int t2 = lane; t2 < w; t2 += 32) {
           const int p = qpos - w + 1 + t2;
@@ -511,7 +609,14 @@ int sm_count() {
   return n > 0 ? n : 148;
 }
 
-int buffer_cap(int k) { return 4 * k + 256; }
+int buffer_cap(int k) { return max(2 * k, 256); }
+
+template <int G>
+int stages_for() {
+  // as many K stages as fit next to Q, the bookkeeping and 1 KB of alignment
+  const int fixed = OFF_K + int(sizeof(Misc<G>)) + 1024;
+  return min(MAX_STAGES, (227 * 1024 - fixed) / TILE_BYTES);
+}
 
 template <int G>
 cudaError_t launch_g(const SelectArgs& a, cudaStream_t stream) {
@@ -521,13 +626,17 @@ cudaError_t launch_g(const SelectArgs& a, cudaStream_t stream) {
     return cudaErrorInvalidValue;
   if (!make_tmap_3d(&tmK, a.K, 128, a.Hkv, a.T, 256, uint64_t(a.Hkv) * 256, 64, 1, TILE))
     return cudaErrorInvalidValue;
-  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(select_kernel<G>), SMEM);
+  const int kst = stages_for<G>();
+  const int smem = OFF_K + kst * TILE_BYTES + int(sizeof(Misc<G>)) + 1024;
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(select_kernel<G>), smem);
   if (e != cudaSuccess) return e;
   const int n_items = int((a.T + QT - 1) / QT) * a.Hkv;
   const int grid = min(sm_count(), n_items);
-  select_kernel<G><<<grid, THREADS, SMEM, stream>>>(
-      tmQ, tmK, a.lse, a.idx, a.kth, reinterpret_cast<uint2*>(a.ws), int(a.T), a.Hkv, a.k, a.w,
-      buffer_cap(a.k), a.scale * kLog2e);
+  uint2* ws = reinterpret_cast<uint2*>(a.ws);
+  uint32_t* wsort = reinterpret_cast<uint32_t*>(ws + size_t(sm_count()) * 4 * QT * buffer_cap(a.k));
+  select_kernel<G><<<grid, THREADS, smem, stream>>>(tmQ, tmK, a.lse, a.idx, a.kth, ws, wsort,
+                                                    int(a.T), a.Hkv, a.k, a.w, buffer_cap(a.k),
+                                                    kst, a.scale * kLog2e);
   count_launch();
   return cudaGetLastError();
 }
@@ -538,7 +647,8 @@ size_t select_workspace_bytes(int64_t T, int Hq, int Hkv, int k, int w) {
   (void)T;
   (void)w;
   const int QT = TILE / (Hq / Hkv);
-  return size_t(sm_count()) * QT * buffer_cap(k) * sizeof(uint2);
+  return size_t(sm_count()) * (size_t(4) * QT * buffer_cap(k) * sizeof(uint2) +
+                               size_t(8) * 2048 * sizeof(uint32_t));
 }
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream) {
