@@ -1,10 +1,664 @@
-// decode.cu -- placeholder until the decode kernels land
+// decode.cu -- one decode step of the cross-decoder block over an FP8 KV cache.
+//
+// The FP8 KV cache of the zgeo.com.cn comparison table and of the
+// javabetter.cn explainer's 1M-token figures; the cross-decoder runs while
+// generating (zgeo.com.cn, section 核心技术原理解析).  For each sequence b the
+// new token is the last cache entry i = N_b - 1; the block runs full
+// attention, token selection and the sparse layers on
+//   K^[t,g,:] = e4m3(Kc[b,t,g,:]) * k_scale[b,t,g]  (likewise V).
+//
+// Kernels (all on `stream`):
+//   decode_partial  split-KV attention of the G query heads of (b, g) over a
+//                   4096-key chunk with mma.sync m16n8k16 (e4m3 codes -> f16
+//                   exactly, fp32 accumulation).  The dot-product dimension
+//                   and the output dims are permuted so every lane reads 16
+//                   contiguous bytes of a K or V row (fully coalesced rows).
+//                   Writes base-2 logits (fp32) for the scoring pass and the
+//                   chunk's (max, sum, unnormalised output).
+//   decode_merge    merges the chunks: o (bf16), lse (natural log).
+//   decode_score    score_j = sum_h exp2(logit_hj - lse2_h) for candidates
+//                   j <= i - w, stored; histogram of score buckets (fp32
+//                   bits >> 20: eighths of a binade) per (b, g).
+//   decode_collect  every candidate in the bucket holding the k-th best score
+//                   or above goes to a per-(b, g) list (about k + a few
+//                   hundred entries).
+//   decode_final    per (b, g): exact top k of the list on the 64-bit key
+//                   (score bits << 32 | ~j), positions sorted ascending, then
+//                   the window; an exact radix select over all candidates
+//                   when the list overflows.
+// The sparse layers then gather the FP8 rows at idx (sparse_attn.cu).
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
 #include "common.cuh"
 #include "kernels.h"
+
 namespace hs2 {
 
 HS2_STATUS_ACCESSOR(status_decode)
 
-size_t decode_workspace_bytes(int, int64_t, int, int, int, int) { return 0; }
-cudaError_t launch_decode(const DecodeArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+namespace {
+
+constexpr int CH = 4096;            // keys per decode_partial CTA
+constexpr int DP_WARPS = 4;         // each warp: CH / 4 keys, 16 per step
+constexpr int NBUCKET = 2048;       // score buckets (bits >> 20 of fp32 < 2^8)
+constexpr int CAPC = 8192;          // candidate list capacity per (b, g)
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+constexpr int MAX_B = 64;
+constexpr float kPScale = 1024.f;   // P' = p * v_scale * 2^10 keeps f16 products normal
+
+struct Partial {  // per (b, h, chunk)
+  float m, l;
+};
+
+struct SeqLens {  // sequence lengths, passed by value
+  int n[MAX_B];
+};
+
+__device__ __forceinline__ uint32_t cvt_e4m3x2_f16x2(uint32_t two_bytes) {
+  __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_bytes & 0xFFFFu),
+                                             __NV_E4M3);
+  return uint32_t(h.x) | (uint32_t(h.y) << 16);
+}
+
+__device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                        uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// byte x (0..15) of a uint4
+__device__ __forceinline__ uint32_t byte_of(const uint4& v, int x) {
+  const uint32_t w = x < 4 ? v.x : x < 8 ? v.y : x < 12 ? v.z : v.w;
+  return (w >> (8 * (x & 3))) & 0xFFu;
+}
+
+// ---------------------------------------------------------------------------
+// decode_partial: grid (chunks, Hkv, B), DP_WARPS warps
+// ---------------------------------------------------------------------------
+template <int G>
+__global__ void __launch_bounds__(DP_WARPS * 32)
+    decode_partial(const __nv_bfloat16* __restrict__ q, const uint8_t* __restrict__ Kc,
+                   const uint8_t* __restrict__ Vc, const float* __restrict__ ks,
+                   const float* __restrict__ vs, SeqLens seq_len, int64_t cap,
+                   int Hkv, int nch, float scale_log2, float* __restrict__ logits,
+                   Partial* __restrict__ part, float* __restrict__ part_o) {
+  constexpr int NT = G > 8 ? G / 8 : 1;   // 8-head n-tiles
+  constexpr int GH = G < 8 ? G : 8;       // real heads per n-tile
+  __shared__ uint16_t sP[DP_WARPS][NT][8 * 16];      // P' [head][key] f16 per warp
+  __shared__ float sM[DP_WARPS][NT * 8], sL[DP_WARPS][NT * 8];
+  __shared__ float sO[DP_WARPS][NT * 8][128];
+
+  const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int warp = warp_id(), lane = lane_id();
+  const int gid = lane >> 2, t = lane & 3;
+  const int N = seq_len.n[b];
+  const int Hq = Hkv * G;
+  const int64_t key_lo = int64_t(c) * CH + warp * (CH / DP_WARPS);
+  const int64_t key_hi = min(int64_t(c) * CH + (warp + 1) * (CH / DP_WARPS), int64_t(N));
+  const size_t rowbase = size_t(b) * cap;  // first cache row of sequence b
+
+  // query fragments (B operand of S^T = K q^T): dims permuted so that lane t
+  // uses dims 32t .. 32t+31: MMA step s, k-slot {2t,2t+1,2t+8,2t+9} ->
+  // dim 32t + 4s + {0,1,2,3}
+  uint32_t qf[NT][8][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int hh = nt * 8 + gid;
+    const bool real = hh < G;
+    const __nv_bfloat16* qr = q + (size_t(b) * Hq + g * G + (real ? hh : 0)) * 128 + 32 * t;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint4 w = real ? *reinterpret_cast<const uint4*>(qr + 8 * u) : make_uint4(0, 0, 0, 0);
+      const uint32_t ws4[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {  // two steps per 16 bytes
+        const int s = 2 * u + h2;
+        qf[nt][s][0] = pack_f16x2(bf16lo(ws4[2 * h2]), bf16hi(ws4[2 * h2]));
+        qf[nt][s][1] = pack_f16x2(bf16lo(ws4[2 * h2 + 1]), bf16hi(ws4[2 * h2 + 1]));
+      }
+    }
+  }
+
+  float m_run[NT][2], l_run[NT][2], o[NT][8][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    m_run[nt][0] = m_run[nt][1] = -INFINITY;
+    l_run[nt][0] = l_run[nt][1] = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[nt][i][0] = o[nt][i][1] = o[nt][i][2] = o[nt][i][3] = 0.f;
+  }
+  float* lg = logits + (size_t(b) * Hkv + g) * cap * G;
+
+  for (int64_t key0 = key_lo; key0 < key_hi; key0 += 16) {
+    // ---- S^T = K q^T : rows key0+gid and key0+gid+8, lane bytes 32t..32t+31
+    const int64_t r0 = key0 + gid, r1 = key0 + gid + 8;
+    const bool v0 = r0 < key_hi, v1 = r1 < key_hi;
+    const uint8_t* k0 = Kc + ((rowbase + (v0 ? r0 : key_lo)) * Hkv + g) * 128 + 32 * t;
+    const uint8_t* k1 = Kc + ((rowbase + (v1 ? r1 : key_lo)) * Hkv + g) * 128 + 32 * t;
+    const uint4 ka = __ldg(reinterpret_cast<const uint4*>(k0));
+    const uint4 kb = __ldg(reinterpret_cast<const uint4*>(k0 + 16));
+    const uint4 kc = __ldg(reinterpret_cast<const uint4*>(k1));
+    const uint4 kd = __ldg(reinterpret_cast<const uint4*>(k1 + 16));
+    // ---- V rows key0 + 4t + u, bytes 16*gid .. 16*gid+15
+    uint4 vr[4];
+    float vsc[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t rv = key0 + 4 * t + u;
+      const bool ok = rv < key_hi;
+      vr[u] = __ldg(reinterpret_cast<const uint4*>(
+          Vc + ((rowbase + (ok ? rv : key_lo)) * Hkv + g) * 128 + 16 * gid));
+      vsc[u] = ok ? __ldg(vs + (rowbase + rv) * Hkv + g) * kPScale : 0.f;
+    }
+    const float ks0 = v0 ? __ldg(ks + (rowbase + r0) * Hkv + g) : 0.f;
+    const float ks1 = v1 ? __ldg(ks + (rowbase + r1) * Hkv + g) : 0.f;
+
+    const uint32_t kw0[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
+    const uint32_t kw1[8] = {kc.x, kc.y, kc.z, kc.w, kd.x, kd.y, kd.z, kd.w};
+    float sacc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      const uint32_t a0 = cvt_e4m3x2_f16x2(kw0[s]);        // row gid,   slots 2t,2t+1
+      const uint32_t a1 = cvt_e4m3x2_f16x2(kw1[s]);        // row gid+8, slots 2t,2t+1
+      const uint32_t a2 = cvt_e4m3x2_f16x2(kw0[s] >> 16);  // row gid,   slots 2t+8,2t+9
+      const uint32_t a3 = cvt_e4m3x2_f16x2(kw1[s] >> 16);  // row gid+8, slots 2t+8,2t+9
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) mma_f16(sacc[nt], a0, a1, a2, a3, qf[nt][s][0], qf[nt][s][1]);
+    }
+    // base-2 logits; lane holds keys r0 (c0,c1) and r1 (c2,c3), heads 2t, 2t+1
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int h0 = nt * 8 + 2 * t;
+      float s00 = v0 ? sacc[nt][0] * ks0 * scale_log2 : -INFINITY;
+      float s01 = v0 ? sacc[nt][1] * ks0 * scale_log2 : -INFINITY;
+      float s10 = v1 ? sacc[nt][2] * ks1 * scale_log2 : -INFINITY;
+      float s11 = v1 ? sacc[nt][3] * ks1 * scale_log2 : -INFINITY;
+      if (h0 >= GH + nt * 8) s00 = s10 = -INFINITY;      // padded heads
+      if (h0 + 1 >= GH + nt * 8) s01 = s11 = -INFINITY;
+      if (h0 + 1 < G) {
+        if (v0) *reinterpret_cast<float2*>(lg + r0 * G + h0) = make_float2(s00, s01);
+        if (v1) *reinterpret_cast<float2*>(lg + r1 * G + h0) = make_float2(s10, s11);
+      } else if (h0 < G) {
+        if (v0) lg[r0 * G + h0] = s00;
+        if (v1) lg[r1 * G + h0] = s10;
+      }
+      // online softmax over this step's 16 keys for heads h0, h0+1
+      float mx0 = fmaxf(s00, s10), mx1 = fmaxf(s01, s11);
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+      }
+      const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
+      const float al0 = mn0 == -INFINITY ? 1.f : fast_exp2(m_run[nt][0] - mn0);
+      const float al1 = mn1 == -INFINITY ? 1.f : fast_exp2(m_run[nt][1] - mn1);
+      const float p00 = mn0 == -INFINITY ? 0.f : fast_exp2(s00 - mn0);
+      const float p10 = mn0 == -INFINITY ? 0.f : fast_exp2(s10 - mn0);
+      const float p01 = mn1 == -INFINITY ? 0.f : fast_exp2(s01 - mn1);
+      const float p11 = mn1 == -INFINITY ? 0.f : fast_exp2(s11 - mn1);
+      m_run[nt][0] = mn0;
+      m_run[nt][1] = mn1;
+      l_run[nt][0] = l_run[nt][0] * al0 + p00 + p10;
+      l_run[nt][1] = l_run[nt][1] * al1 + p01 + p11;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        o[nt][i][0] *= al0;
+        o[nt][i][2] *= al0;
+        o[nt][i][1] *= al1;
+        o[nt][i][3] *= al1;
+      }
+      // P (unscaled by V's scale yet) to shared memory, [head][key] f16;
+      // local keys gid (r0) and gid+8 (r1)
+      uint16_t* sp = sP[warp][nt];
+      const __half hp00 = __float2half_rn(p00), hp01 = __float2half_rn(p01);
+      const __half hp10 = __float2half_rn(p10), hp11 = __float2half_rn(p11);
+      sp[(2 * t) * 16 + gid] = *reinterpret_cast<const uint16_t*>(&hp00);
+      sp[(2 * t + 1) * 16 + gid] = *reinterpret_cast<const uint16_t*>(&hp01);
+      sp[(2 * t) * 16 + gid + 8] = *reinterpret_cast<const uint16_t*>(&hp10);
+      sp[(2 * t + 1) * 16 + gid + 8] = *reinterpret_cast<const uint16_t*>(&hp11);
+    }
+    __syncwarp();
+    // ---- O^T += V^T P'^T: M = 16 dims (permuted), K = 16 keys (4t+u), N = heads
+    // B fragment: P'[head gid][keys 4t, 4t+1] and [4t+2, 4t+3], times V scale
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const uint16_t* sp = sP[warp][nt] + gid * 16 + 4 * t;
+      const float f0 = __half2float(*reinterpret_cast<const __half*>(sp + 0)) * vsc[0];
+      const float f1 = __half2float(*reinterpret_cast<const __half*>(sp + 1)) * vsc[1];
+      const float f2 = __half2float(*reinterpret_cast<const __half*>(sp + 2)) * vsc[2];
+      const float f3 = __half2float(*reinterpret_cast<const __half*>(sp + 3)) * vsc[3];
+      // vsc already carries the 2^10 factor (see below)
+      const uint32_t b0 = pack_f16x2(f0, f1), b1 = pack_f16x2(f2, f3);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        // dims 16*gid + 2i (MMA row gid) and 16*gid + 2i + 1 (row gid+8)
+        const uint32_t a0 = cvt_e4m3x2_f16x2(byte_of(vr[0], 2 * i) | (byte_of(vr[1], 2 * i) << 8));
+        const uint32_t a1 =
+            cvt_e4m3x2_f16x2(byte_of(vr[0], 2 * i + 1) | (byte_of(vr[1], 2 * i + 1) << 8));
+        const uint32_t a2 = cvt_e4m3x2_f16x2(byte_of(vr[2], 2 * i) | (byte_of(vr[3], 2 * i) << 8));
+        const uint32_t a3 =
+            cvt_e4m3x2_f16x2(byte_of(vr[2], 2 * i + 1) | (byte_of(vr[3], 2 * i + 1) << 8));
+        mma_f16(o[nt][i], a0, a1, a2, a3, b0, b1);
+      }
+    }
+    __syncwarp();
+  }
+
+  // ---- combine the warps of the CTA, then one partial per (b, h, chunk)
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      float l = l_run[nt][e];
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+      l_run[nt][e] = l;
+    }
+    if (gid == 0) {
+      sM[warp][nt * 8 + 2 * t] = m_run[nt][0];
+      sM[warp][nt * 8 + 2 * t + 1] = m_run[nt][1];
+      sL[warp][nt * 8 + 2 * t] = l_run[nt][0];
+      sL[warp][nt * 8 + 2 * t + 1] = l_run[nt][1];
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      sO[warp][nt * 8 + 2 * t][16 * gid + 2 * i] = o[nt][i][0];
+      sO[warp][nt * 8 + 2 * t + 1][16 * gid + 2 * i] = o[nt][i][1];
+      sO[warp][nt * 8 + 2 * t][16 * gid + 2 * i + 1] = o[nt][i][2];
+      sO[warp][nt * 8 + 2 * t + 1][16 * gid + 2 * i + 1] = o[nt][i][3];
+    }
+  }
+  __syncthreads();
+  for (int hh = warp; hh < G; hh += DP_WARPS) {
+    float M = -INFINITY;
+    for (int w2 = 0; w2 < DP_WARPS; ++w2) M = fmaxf(M, sM[w2][hh]);
+    float L = 0.f, f[DP_WARPS];
+    for (int w2 = 0; w2 < DP_WARPS; ++w2) {
+      f[w2] = M == -INFINITY ? 0.f : fast_exp2(sM[w2][hh] - M);
+      L += sL[w2][hh] * f[w2];
+    }
+    const size_t pi = (size_t(b) * Hq + g * G + hh) * nch + c;
+    for (int d = lane; d < 128; d += 32) {
+      float acc = 0.f;
+      for (int w2 = 0; w2 < DP_WARPS; ++w2) acc += sO[w2][hh][d] * f[w2];
+      part_o[pi * 128 + d] = acc * (1.f / kPScale);
+    }
+    if (lane == 0) part[pi] = Partial{M, L};
+  }
+}
+
+// ---------------------------------------------------------------------------
+// decode_merge: grid (Hq, B), 128 threads
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128)
+    decode_merge(const Partial* __restrict__ part, const float* __restrict__ part_o,
+                 SeqLens seq_len, int Hq, int nch, __nv_bfloat16* __restrict__ o,
+                 float* __restrict__ lse, float* __restrict__ lse2_out) {
+  const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
+  const int nc = (seq_len.n[b] + CH - 1) / CH;
+  const size_t base = (size_t(b) * Hq + h) * nch;
+  float M = -INFINITY;
+  for (int c = 0; c < nc; ++c) M = fmaxf(M, part[base + c].m);
+  float L = 0.f, acc = 0.f;
+  for (int c = 0; c < nc; ++c) {
+    const Partial p = part[base + c];
+    const float f = p.m == -INFINITY ? 0.f : fast_exp2(p.m - M);
+    L += p.l * f;
+    acc += part_o[(base + c) * 128 + d] * f;
+  }
+  o[(size_t(b) * Hq + h) * 128 + d] = __float2bfloat16_rn(acc / L);
+  if (d == 0) {
+    const float l2 = M + __log2f(L);
+    lse[size_t(b) * Hq + h] = l2 * kLn2;
+    lse2_out[size_t(b) * Hq + h] = l2;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// decode_score: grid (chunks, Hkv, B), 256 threads
+// ---------------------------------------------------------------------------
+template <int G>
+__global__ void __launch_bounds__(256)
+    decode_score(const float* __restrict__ logits, const float* __restrict__ lse2,
+                 SeqLens seq_len, int64_t cap, int Hkv, int w,
+                 float* __restrict__ score, uint32_t* __restrict__ hist) {
+  __shared__ uint32_t sh[NBUCKET];
+  __shared__ float sl[G];
+  const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int N = seq_len.n[b];
+  const int64_t ncand = int64_t(N) - w;  // candidates j < ncand (j <= i - w)
+  for (int i = threadIdx.x; i < NBUCKET; i += 256) sh[i] = 0;
+  if (threadIdx.x < G) sl[threadIdx.x] = lse2[size_t(b) * Hkv * G + g * G + threadIdx.x];
+  __syncthreads();
+  const float* lg = logits + (size_t(b) * Hkv + g) * cap * G;
+  float* sc = score + (size_t(b) * Hkv + g) * cap;
+  const int64_t j_hi = min(int64_t(c + 1) * CH, ncand);
+  for (int64_t j = int64_t(c) * CH + threadIdx.x; j < j_hi; j += 256) {
+    float acc = 0.f;
+#pragma unroll
+    for (int h = 0; h < G; ++h) acc += fast_exp2(lg[j * G + h] - sl[h]);
+    sc[j] = acc;
+    atomicAdd(&sh[__float_as_uint(acc) >> 20], 1u);
+  }
+  __syncthreads();
+  uint32_t* gh = hist + (size_t(b) * Hkv + g) * NBUCKET;
+  for (int i = threadIdx.x; i < NBUCKET; i += 256)
+    if (sh[i]) atomicAdd(&gh[i], sh[i]);
+}
+
+// bucket holding the k-th largest count from the top (NBUCKET bins, 256
+// threads); returns -1 if the total is below k
+__device__ int block_kth_bucket(const uint32_t* __restrict__ gh, uint32_t k, uint32_t* s_scan) {
+  // each thread sums 8 bins (highest first)
+  const int tid = threadIdx.x;
+  uint32_t c8[8], local = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    c8[i] = gh[NBUCKET - 1 - 8 * tid - i];
+    local += c8[i];
+  }
+  s_scan[tid] = local;
+  __syncthreads();
+  // inclusive scan over 256 threads (simple Hillis-Steele)
+  for (int off = 1; off < 256; off <<= 1) {
+    const uint32_t v = tid >= off ? s_scan[tid - off] : 0u;
+    __syncthreads();
+    s_scan[tid] += v;
+    __syncthreads();
+  }
+  __shared__ int found;
+  if (tid == 0) found = -1;
+  __syncthreads();
+  const uint32_t incl = s_scan[tid], excl = incl - local;
+  if (excl < k && k <= incl) {
+    uint32_t cum = excl;
+    for (int i = 0; i < 8; ++i) {
+      if (cum + c8[i] >= k) {
+        found = NBUCKET - 1 - 8 * tid - i;
+        break;
+      }
+      cum += c8[i];
+    }
+  }
+  __syncthreads();
+  return found;
+}
+
+// ---------------------------------------------------------------------------
+// decode_collect: grid (chunks, Hkv, B), 256 threads
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+    decode_collect(const float* __restrict__ score, const uint32_t* __restrict__ hist,
+                   SeqLens seq_len, int64_t cap, int Hkv, int k, int w,
+                   uint2* __restrict__ cand, uint32_t* __restrict__ ccount) {
+  __shared__ uint32_t s_scan[256];
+  const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int N = seq_len.n[b];
+  const int64_t ncand = int64_t(N) - w;
+  if (ncand <= k) return;  // everything is selected; decode_final writes it
+  const int64_t j_lo = int64_t(c) * CH;
+  if (j_lo >= ncand) return;
+  const size_t bg = size_t(b) * Hkv + g;
+  const int kb = block_kth_bucket(hist + bg * NBUCKET, uint32_t(k), s_scan);
+  const uint32_t thr = kb < 0 ? 0u : uint32_t(kb);
+  const float* sc = score + bg * cap;
+  const int64_t j_hi = min(j_lo + CH, ncand);
+  const int lane = lane_id();
+  for (int64_t base = j_lo; base < j_hi; base += 256) {
+    const int64_t j = base + threadIdx.x;
+    float v = 0.f;
+    bool take = false;
+    if (j < j_hi) {
+      v = sc[j];
+      take = (__float_as_uint(v) >> 20) >= thr;
+    }
+    const uint32_t bal = __ballot_sync(0xffffffffu, take);
+    if (bal) {
+      uint32_t pos = 0;
+      if (lane == __ffs(bal) - 1) pos = atomicAdd(&ccount[bg], __popc(bal));
+      pos = __shfl_sync(0xffffffffu, pos, __ffs(bal) - 1);
+      const uint32_t p = pos + __popc(bal & ((1u << lane) - 1u));
+      if (take && p < uint32_t(CAPC)) cand[bg * CAPC + p] = make_uint2(__float_as_uint(v), uint32_t(j));
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// decode_final: grid (Hkv, B), 512 threads
+// ---------------------------------------------------------------------------
+__device__ void block_bitonic_u64(uint64_t* s, int np, bool descending) {
+  for (int size = 2; size <= np; size <<= 1)
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = threadIdx.x; i < np / 2; i += blockDim.x) {
+        const int lo = 2 * stride * (i / stride) + (i % stride), hi = lo + stride;
+        const bool up = ((lo & size) == 0) != descending;
+        const uint64_t a = s[lo], bb = s[hi];
+        if ((a > bb) == up) {
+          s[lo] = bb;
+          s[hi] = a;
+        }
+      }
+      __syncthreads();
+    }
+}
+
+__global__ void __launch_bounds__(512)
+    decode_final(const uint2* __restrict__ cand, const uint32_t* __restrict__ ccount,
+                 const float* __restrict__ score, SeqLens seq_len, int64_t cap,
+                 int Hkv, int k, int w, int32_t* __restrict__ idx) {
+  extern __shared__ uint64_t sk[];  // CAPC keys
+  __shared__ uint32_t s_hist[256];
+  __shared__ uint32_t s_misc[4];
+  const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int N = seq_len.n[b];
+  const int64_t i = N - 1;
+  const int64_t ncand = max(int64_t(0), i - w + 1);
+  const size_t bg = size_t(b) * Hkv + g;
+  int32_t* out = idx + bg * (k + w);
+  for (int t2 = tid; t2 < w; t2 += blockDim.x) {
+    const int64_t p = i - w + 1 + t2;
+    out[k + t2] = p >= 0 ? int32_t(p) : -1;
+  }
+  if (ncand <= k) {
+    for (int e = tid; e < k; e += blockDim.x) out[e] = e < ncand ? e : -1;
+    return;
+  }
+  const uint32_t n = ccount[bg];
+  if (n <= uint32_t(CAPC)) {
+    int np = 1;
+    while (np < int(n)) np <<= 1;
+    for (int e = tid; e < np; e += blockDim.x) {
+      if (e < int(n)) {
+        const uint2 v = cand[bg * CAPC + e];
+        sk[e] = (uint64_t(v.x) << 32) | uint64_t(~v.y);
+      } else {
+        sk[e] = 0;  // below every real key
+      }
+    }
+    __syncthreads();
+    block_bitonic_u64(sk, np, true);  // best first
+    // the k best positions, ascending
+    int kp = 1;
+    while (kp < k) kp <<= 1;
+    __syncthreads();
+    for (int e = tid; e < kp; e += blockDim.x)
+      sk[e] = e < k ? uint64_t(~uint32_t(sk[e])) : ~uint64_t(0);
+    __syncthreads();
+    block_bitonic_u64(sk, kp, false);
+    for (int e = tid; e < k; e += blockDim.x) out[e] = int32_t(sk[e]);
+    return;
+  }
+  // overflow: exact radix select over every candidate's score, then the
+  // selected positions in ascending order by a block-wide ordered scan
+  const float* sc = score + bg * cap;
+  uint64_t prefix = 0, mask = 0;
+  uint32_t remaining = k;
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    for (int e = tid; e < 256; e += blockDim.x) s_hist[e] = 0;
+    __syncthreads();
+    for (int64_t j = tid; j < ncand; j += blockDim.x) {
+      const uint64_t key = (uint64_t(__float_as_uint(sc[j])) << 32) | uint64_t(~uint32_t(j));
+      if ((key & mask) == prefix) atomicAdd(&s_hist[(key >> shift) & 255], 1u);
+    }
+    __syncthreads();
+    if (tid == 0) {
+      uint32_t cum = 0;
+      int bin = 255;
+      for (; bin >= 0; --bin) {
+        if (cum + s_hist[bin] >= remaining) break;
+        cum += s_hist[bin];
+      }
+      s_misc[0] = uint32_t(bin);
+      s_misc[1] = cum;
+      s_misc[2] = s_hist[bin];
+    }
+    __syncthreads();
+    const uint32_t bin = s_misc[0], above = s_misc[1], inbin = s_misc[2];
+    __syncthreads();
+    remaining -= above;
+    prefix |= uint64_t(bin) << shift;
+    mask |= uint64_t(0xFF) << shift;
+    if (inbin == remaining) break;
+  }
+  __shared__ uint32_t s_warp[16];
+  uint32_t written = 0;
+  for (int64_t base = 0; base < ncand; base += blockDim.x) {
+    const int64_t j = base + tid;
+    bool sel = false;
+    if (j < ncand) {
+      const uint64_t key = (uint64_t(__float_as_uint(sc[j])) << 32) | uint64_t(~uint32_t(j));
+      sel = (key & mask) >= prefix;
+    }
+    const uint32_t bal = __ballot_sync(0xffffffffu, sel);
+    if (lane_id() == 0) s_warp[warp_id()] = __popc(bal);
+    __syncthreads();
+    uint32_t before = written;
+    for (int w2 = 0; w2 < warp_id(); ++w2) before += s_warp[w2];
+    uint32_t tot = 0;
+    for (int w2 = 0; w2 < int(blockDim.x / 32); ++w2) tot += s_warp[w2];
+    if (sel) {
+      const uint32_t p = before + __popc(bal & ((1u << lane_id()) - 1u));
+      if (p < uint32_t(k)) out[p] = int32_t(j);
+    }
+    written += tot;
+    __syncthreads();
+  }
+}
+
+template <int G>
+cudaError_t launch_dec_g(const DecodeArgs& a, const SeqLens& d_seq, int max_len, cudaStream_t st,
+                         uint8_t* w8) {
+  const int Hq = a.Hq, Hkv = a.Hkv, B = a.B;
+  const int nch = int((a.cap + CH - 1) / CH);
+  const int nch_used = (max_len + CH - 1) / CH;
+  // workspace layout (see decode_workspace_bytes)
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    uint8_t* p = w8 + off;
+    off += (bytes + 255) / 256 * 256;
+    return p;
+  };
+  float* logits = reinterpret_cast<float*>(take(size_t(B) * Hkv * a.cap * G * 4));
+  float* score = reinterpret_cast<float*>(take(size_t(B) * Hkv * a.cap * 4));
+  Partial* part = reinterpret_cast<Partial*>(take(size_t(B) * Hq * nch * sizeof(Partial)));
+  float* part_o = reinterpret_cast<float*>(take(size_t(B) * Hq * nch * 128 * 4));
+  float* lse2 = reinterpret_cast<float*>(take(size_t(B) * Hq * 4));
+  uint32_t* hist = reinterpret_cast<uint32_t*>(take(size_t(B) * Hkv * NBUCKET * 4));
+  uint32_t* ccount = reinterpret_cast<uint32_t*>(take(size_t(B) * Hkv * 4));
+  uint2* cand = reinterpret_cast<uint2*>(take(size_t(B) * Hkv * CAPC * 8));
+
+  cudaError_t e = cudaMemsetAsync(hist, 0, size_t(B) * Hkv * NBUCKET * 4, st);
+  if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(ccount, 0, size_t(B) * Hkv * 4, st);
+  if (e != cudaSuccess) return e;
+  const float sl2 = a.scale * kLog2e;
+  decode_partial<G><<<dim3(nch_used, Hkv, B), DP_WARPS * 32, 0, st>>>(
+      reinterpret_cast<const __nv_bfloat16*>(a.q), a.Kc, a.Vc, a.ks, a.vs, d_seq, a.cap, Hkv, nch,
+      sl2, logits, part, part_o);
+  decode_merge<<<dim3(Hq, B), 128, 0, st>>>(part, part_o, d_seq, Hq, nch,
+                                            reinterpret_cast<__nv_bfloat16*>(a.o), a.lse, lse2);
+  decode_score<G><<<dim3(nch_used, Hkv, B), 256, 0, st>>>(logits, lse2, d_seq, a.cap, Hkv, a.w,
+                                                          score, hist);
+  decode_collect<<<dim3(nch_used, Hkv, B), 256, 0, st>>>(score, hist, d_seq, a.cap, Hkv, a.k, a.w,
+                                                         cand, ccount);
+  const int fsmem = CAPC * 8;
+  e = ensure_smem_attr(reinterpret_cast<const void*>(decode_final), fsmem);
+  if (e != cudaSuccess) return e;
+  decode_final<<<dim3(Hkv, B), 512, fsmem, st>>>(cand, ccount, score, d_seq, a.cap, Hkv, a.k, a.w,
+                                                 a.idx);
+  count_launch(5);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  for (int l = 0; l < a.n_sparse; ++l) {
+    SparseArgs s{};
+    s.Q = a.qs[l];
+    s.idx = a.idx;
+    s.O = a.os[l];
+    s.lse = nullptr;
+    s.T = B;
+    s.Hq = Hq;
+    s.Hkv = Hkv;
+    s.scale = a.scale;
+    s.kw = a.k + a.w;
+    s.Kc = a.Kc;
+    s.Vc = a.Vc;
+    s.ks = a.ks;
+    s.vs = a.vs;
+    s.cache_T = a.cap;
+    e = launch_sparse(s, st);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+size_t dec_ws_bytes(int B, int64_t cap, int Hq, int Hkv) {
+  const int G = Hq / Hkv;
+  const int nch = int((cap + CH - 1) / CH);
+  auto r = [](size_t x) { return (x + 255) / 256 * 256; };
+  return r(size_t(B) * Hkv * cap * G * 4) + r(size_t(B) * Hkv * cap * 4) +
+         r(size_t(B) * Hq * nch * sizeof(Partial)) + r(size_t(B) * Hq * nch * 128 * 4) +
+         r(size_t(B) * Hq * 4) + r(size_t(B) * Hkv * NBUCKET * 4) + r(size_t(B) * Hkv * 4) +
+         r(size_t(B) * Hkv * CAPC * 8);
+}
+
+}  // namespace
+
+size_t decode_workspace_bytes(int B, int64_t cap, int Hq, int Hkv, int k, int w) {
+  (void)k;
+  (void)w;
+  return dec_ws_bytes(B, cap, Hq, Hkv);
+}
+
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
+  if (a.B > MAX_B || a.k > CAPC / 2 || a.cap > INT32_MAX) return cudaErrorNotSupported;
+  SeqLens d_seq{};
+  int max_len = 0;
+  for (int b = 0; b < a.B; ++b) {
+    d_seq.n[b] = int(a.seq_len_host[b]);
+    max_len = d_seq.n[b] > max_len ? d_seq.n[b] : max_len;
+  }
+  uint8_t* w8 = reinterpret_cast<uint8_t*>(a.ws);
+  switch (a.Hq / a.Hkv) {
+    case 1: return launch_dec_g<1>(a, d_seq, max_len, st, w8);
+    case 2: return launch_dec_g<2>(a, d_seq, max_len, st, w8);
+    case 4: return launch_dec_g<4>(a, d_seq, max_len, st, w8);
+    case 8: return launch_dec_g<8>(a, d_seq, max_len, st, w8);
+    case 16: return launch_dec_g<16>(a, d_seq, max_len, st, w8);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 }  // namespace hs2
