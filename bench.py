@@ -205,6 +205,104 @@ class OracleSample:
 
 
 # ---------------------------------------------------------------------------
+# decode step at 1M context (8 sequences, FP8 cache)
+# ---------------------------------------------------------------------------
+def bench_decode(hs2, dev, steps, warmup):
+    cfg = synth.CONFIGS["C5"]
+    B, N, Hq, Hkv = cfg.batch, cfg.T, cfg.n_q_heads, cfg.n_kv_heads
+    k, w = cfg.k_global, cfg.window
+    Kc, Vc, S = synth.decode_cache_torch(cfg, N, device=dev)
+    u = torch.from_numpy(synth.needle_dirs(cfg)).to(dev).repeat_interleave(cfg.G, 0)
+
+    def qrow(tid):
+        z = synth.normals_torch(cfg.seed, tid, 0, B * Hq * 128, dev).view(B, Hq, 128)
+        return (0.5 * z + 0.5 * math.sqrt(128) * u[None]).float().bfloat16()
+
+    q = qrow(synth.TID_Q)
+    qs = [qrow(synth.TID_QS0 + l) for l in range(cfg.n_sparse)]
+    shape = hs2.Shape.make(N, Hq, Hkv, k_global=k, window=w)
+    o = torch.empty(B, Hq, 128, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+    idx = torch.empty(B, Hkv, k + w, dtype=torch.int32, device=dev)
+    os_ = [torch.empty_like(o) for _ in range(cfg.n_sparse)]
+    ws = torch.empty(hs2.workspace_size(hs2.OP_BLOCK_DECODE, shape, B), dtype=torch.uint8, device=dev)
+    lens = [N] * B
+
+    def step():
+        hs2.hs2_block_decode(lens, q, Kc, Vc, S, S, o, lse, idx, qs, os_, shape, ws)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    assert hs2.hs2_get_device_status() == hs2.OK
+    n0 = hs2.hs2_kernel_launches()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    us = a.elapsed_time(b) / steps * 1e3
+    # algorithmic bytes: every K and V code once, one scale per (token, KV head),
+    # the sparse layers' gathered rows, queries and outputs
+    algo = (B * N * Hkv * 128 * 2 + B * N * Hkv * 4 +
+            cfg.n_sparse * B * Hkv * (k + w) * (128 * 2 + 4) + (1 + cfg.n_sparse) * B * Hq * 128 * 4)
+    hbm, _, src = peaks()
+    gbs = algo / (us * 1e-6) / 1e9
+    return {"metric": "decode us/step @1M", "value": us, "unit": "us/step",
+            "higher_is_better": False, "steps": steps, "warmup": warmup,
+            "config": {"workload": cfg.name, "batch": B, "context": N, "n_q_heads": Hq,
+                       "n_kv_heads": Hkv, "cache": "e4m3 + fp32 scale per (token, KV head)",
+                       "k_global": k, "window": w, "n_sparse": cfg.n_sparse,
+                       "needles_per_kv_head": cfg.n_needles,
+                       "l2": "inputs larger than L2 (8.6 GB cache)"},
+            "gpu_launches_per_step": (hs2.hs2_kernel_launches() - n0) / steps,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                         "frac": gbs / hbm, "algorithmic_bytes": algo,
+                         "peak_source": f"{src} (hbm copy)"}}
+
+
+# ---------------------------------------------------------------------------
+# one launch of each hot kernel at a moderate size (for profiler captures)
+# ---------------------------------------------------------------------------
+def kernels_once(dev):
+    import long_context_bridge_b200 as hs2
+    T, Hq, Hkv, dm = 32768, 32, 4, 2048
+    cfg = synth.CONFIGS["C3"]
+    g = lambda tid, n, sd=1.0: synth.normal_bf16_torch(cfg.seed, tid, 0, n, sd, device=dev)
+    H = g(synth.TID_H, T * dm).view(T, dm)
+    Wk = g(synth.TID_WK, dm * Hkv * 128, dm ** -0.5).view(dm, Hkv * 128)
+    Wv = g(synth.TID_WV, dm * Hkv * 128, dm ** -0.5).view(dm, Hkv * 128)
+    K = torch.empty(T, Hkv, 128, dtype=torch.bfloat16, device=dev)
+    V = torch.empty_like(K)
+    sh = hs2.Shape.make(T, Hq, Hkv)
+    hs2.hs2_bridge_kv(H, Wk, Wv, K, V, sh)
+    Q = g(synth.TID_Q, T * Hq * 128).view(T, Hq, 128)
+    O = torch.empty_like(Q)
+    lse = torch.empty(T, Hq, dtype=torch.float32, device=dev)
+    hs2.hs2_full_attn_lse(Q, K, V, O, lse, sh)
+    ws = torch.empty(hs2.workspace_size(hs2.OP_SELECT, sh), dtype=torch.uint8, device=dev)
+    idx = torch.empty(T, Hkv, 1152, dtype=torch.int32, device=dev)
+    hs2.hs2_select_topk(Q, K, lse, idx, None, sh, ws)
+    hs2.hs2_sparse_attn(g(synth.TID_QS0, T * Hq * 128).view(T, Hq, 128), K, V, idx, O, None, sh)
+    dcfg = synth.CONFIGS["C5"]
+    N, B = 262144, dcfg.batch
+    Kc, Vc, S = synth.decode_cache_torch(dcfg, N, device=dev)
+    q = [g(synth.TID_Q + 100 * i, B * Hq * 128).view(B, Hq, 128) for i in range(4)]
+    shd = hs2.Shape.make(N, Hq, Hkv)
+    o = torch.empty(B, Hq, 128, dtype=torch.bfloat16, device=dev)
+    os_ = [torch.empty_like(o) for _ in range(3)]
+    wsd = torch.empty(hs2.workspace_size(hs2.OP_BLOCK_DECODE, shd, B), dtype=torch.uint8, device=dev)
+    hs2.hs2_block_decode([N] * B, q[0], Kc, Vc, S, S, o,
+                         torch.empty(B, Hq, dtype=torch.float32, device=dev),
+                         torch.empty(B, Hkv, 1152, dtype=torch.int32, device=dev), q[1:], os_, shd, wsd)
+    torch.cuda.synchronize()
+    assert hs2.hs2_get_device_status() == hs2.OK
+    print("kernels-once: 32K block (bridge, full attention, selection, one sparse layer) and "
+          "one decode step of 8 x 262144 tokens", flush=True)
+
+
+# ---------------------------------------------------------------------------
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -213,7 +311,14 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--kernels-once", action="store_true",
+                    help="run each hot kernel once at a moderate size (profiler driver) and exit")
     args = ap.parse_args()
+    if args.kernels_once:
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        kernels_once(torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0"))))
+        return
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -396,6 +501,11 @@ def main():
                          ("TFLOP/s" if b == "tensor" else "GB/s"):
                              (a / s / 1e12) if b == "tensor" else (a / s / 1e9),
                          "frac": ((a / s / 1e12) / tfl) if b == "tensor" else ((a / s / 1e9) / hbm)}
+    dec = None
+    if not args.no_decode:
+        del inp, K, V, O, Os, lse, idx, ws
+        torch.cuda.empty_cache()
+        dec = bench_decode(hs2, dev, args.steps, args.warmup)
     cpu = None
     if not args.no_cpu and world == 1:
         cpu = OracleSample(cfg).run(320, seed=5)
@@ -404,7 +514,7 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": config, "clocks": clk.summary(), "e2e": e2e,
             "gpu_launches": int(n_launch), "roofline": roof, "kernels": per_kernel,
-            "cpu_baseline": cpu}
+            "decode": dec, "cpu_baseline": cpu}
     print(json.dumps(line), flush=True)
     if pg:
         torch.distributed.destroy_process_group()

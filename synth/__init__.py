@@ -344,6 +344,33 @@ def decode_cache_np(cfg: BlockConfig, N: int, batch: int | None = None) -> Decod
     return DecodeCache(Kc, Vc, S, needles)
 
 
+def decode_cache_torch(cfg: BlockConfig, N: int, batch: int | None = None, device="cuda"):
+    """decode_cache_np's recipe on the device (torch); the e4m3 rounding is
+    torch's float8_e4m3fn cast of values clamped to [-448, 448], pinned to the
+    numpy quantiser by the tests.  Returns (Kc, Vc, scale) as uint8/uint8/fp32
+    tensors [B, N, Hkv, d], [B, N, Hkv]."""
+    import torch
+    B = cfg.batch if batch is None else batch
+    Hkv, d = cfg.n_kv_heads, cfg.head_dim
+    Kc = torch.empty(B, N, Hkv, d, dtype=torch.uint8, device=device)
+    Vc = torch.empty_like(Kc)
+    S = torch.empty(B, N, Hkv, dtype=torch.float32, device=device)
+    nrows = torch.from_numpy(bf16_bits_to_f32(needle_key_bits(cfg))).to(device)
+    for b in range(B):
+        K = normal_bf16_torch(cfg.seed, TID_DEC_K0 + b, 0, N * Hkv * d, device=device).float().view(N, Hkv, d)
+        V = normal_bf16_torch(cfg.seed, TID_DEC_V0 + b, 0, N * Hkv * d, device=device).float().view(N, Hkv, d)
+        for g in range(Hkv):
+            pos = needle_positions(cfg.seed, TID_DEC_POS0 + b, g, min(cfg.n_needles, N), N)
+            K[torch.from_numpy(pos).to(device), g, :] = nrows[g]
+        amax = torch.maximum(K.abs().amax(dim=2), V.abs().amax(dim=2))
+        s = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+        S[b] = s
+        Kc[b] = (K / s[:, :, None]).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
+        Vc[b] = (V / s[:, :, None]).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
+        del K, V
+    return Kc, Vc, S
+
+
 def decode_queries_np(cfg: BlockConfig, tid: int, batch: int | None = None) -> np.ndarray:
     """One query per sequence [B, Hq, d] as bf16 bits (row b of stream tid)."""
     B = cfg.batch if batch is None else batch

@@ -286,3 +286,14 @@ def test_decode_equals_prefill_last_row(orc):
     for key in ("O", "lse", "idx"):
         assert np.array_equal(full[key], dec[key])
     assert np.array_equal(full["O_sparse"][0], dec["O_sparse"][0])
+
+
+def test_synth_decode_cache_torch_matches_numpy():
+    cfg = synth.BlockConfig("t", 5, 3000, 8, 2, n_needles=16, q_mix=True, batch=2, fp8_cache=True)
+    a = synth.decode_cache_np(cfg, 3000)
+    Kc, Vc, S = synth.decode_cache_torch(cfg, 3000, device="cpu")
+    assert np.array_equal(S.numpy(), a.scale)
+    # +-0 codes may differ in sign between the two quantisers
+    for got, want in ((Kc.numpy(), a.Kc), (Vc.numpy(), a.Vc)):
+        nz = (want & 0x7F) != 0
+        assert np.array_equal(got[nz], want[nz]) and np.all((got[~nz] & 0x7F) == 0)
