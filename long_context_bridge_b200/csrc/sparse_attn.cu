@@ -5,15 +5,22 @@
 // full-attention layer's K/V cache at the positions on that layer's token list
 // and keeps no K/V of its own.
 //
-// One warp handles one (query row, KV head) pair and its G query heads:
-//   * the warp walks the list 32 entries at a time; lane t gathers K row
-//     idx[t] with 16-byte loads and forms the G logits against the queries
-//     held in shared memory (pre-scaled by scale * log2 e);
-//   * online softmax per head across the warp (base-2 exponent);
-//   * V rows of the batch are read coalesced (lane l owns dims 4l..4l+3) and
-//     accumulated with the batch's probabilities, staged in shared memory.
-// The FP8 variant reads e4m3 codes and folds the per-(token, head) scales into
-// the logit (K) and into the probability weight (V).
+// Tensor-core gather attention with mma.sync m16n8k16, one (query row, KV
+// head) pair per warp (or per group of WPR warps that split its list):
+//   S^T[16 keys x 8 heads] = K_sel Q^T   and   O^T[16 dims x 8 heads] += V_sel^T P^T
+// The dot-product dimension and the output dims are permuted (a sum does not
+// care about the order of its terms, and the output permutation is undone at
+// the store) so that every lane's fragment words are contiguous in memory:
+//   * QK^T: lane (gid, t) reads dims 32t..32t+31 of gathered key rows gid and
+//     gid+8 -- for bf16 these words are the A registers as they are;
+//   * PV: lane (gid, t) reads dims 16*gid..16*gid+15 of gathered value rows
+//     4t..4t+3, paired into A registers with one byte permute each.
+// Each gathered row is read by four (K) or eight (V) lanes with 16-byte loads
+// that cover it exactly.  Softmax is online and base 2; P goes through 256
+// bytes of shared memory per warp to become the B operand.  The FP8 variant
+// converts e4m3 codes to f16 exactly, multiplies the logits by the key's
+// scale and folds the value's scale into P.
+#include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
 #include "common.cuh"
@@ -25,209 +32,368 @@ HS2_STATUS_ACCESSOR(status_sparse)
 
 namespace {
 
-constexpr int WARPS = 4;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kPScale = 1024.f;  // FP8: P * v_scale * 2^10 stays in f16's normal range
 
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
+template <bool F16>
+__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  if constexpr (F16) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  } else {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  }
 }
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
+
+__device__ __forceinline__ uint32_t e4m3x2_f16x2(uint32_t two) {
+  __half2_raw h =
+      __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two & 0xFFFFu), __NV_E4M3);
+  return uint32_t(h.x) | (uint32_t(h.y) << 16);
 }
 
-// two e4m3 codes (low byte first) -> two floats, exact
-__device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t two) {
-  __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two), __NV_E4M3);
-  __half2 hh = *reinterpret_cast<__half2*>(&h);
-  return __half22float2(hh);
+template <bool F16>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  if constexpr (F16) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  } else {
+    return pack_bf16x2(lo, hi);
+  }
 }
 
-template <int G, bool FP8>
-__global__ void __launch_bounds__(WARPS * 32)
-    sparse_attn_kernel(const __nv_bfloat16* __restrict__ Q, const void* __restrict__ Kp,
-                       const void* __restrict__ Vp, const float* __restrict__ ks,
-                       const float* __restrict__ vs, const int32_t* __restrict__ idx,
-                       __nv_bfloat16* __restrict__ O, float* __restrict__ lse, int64_t rows,
-                       int Hkv, int kw, float scale_log2, int64_t cache_T) {
-  __shared__ __align__(16) float sq[WARPS][G][128];
-  __shared__ float sp[WARPS][G][32];
-  __shared__ int sj[WARPS][32];
-  __shared__ float svs[WARPS][32];
+template <bool F16>
+__device__ __forceinline__ uint16_t one16(float x) {
+  if constexpr (F16) {
+    __half h = __float2half_rn(x);
+    return *reinterpret_cast<uint16_t*>(&h);
+  } else {
+    __nv_bfloat16 h = __float2bfloat16_rn(x);
+    return *reinterpret_cast<uint16_t*>(&h);
+  }
+}
 
-  const int w = warp_id(), lane = lane_id();
-  const int64_t pair = int64_t(blockIdx.x) * WARPS + w;
-  if (pair >= rows * Hkv) return;
-  const int64_t r = pair / Hkv;
-  const int g = int(pair % Hkv);
+template <bool F16>
+__device__ __forceinline__ float from16(uint16_t v) {
+  if constexpr (F16) {
+    return __half2float(*reinterpret_cast<__half*>(&v));
+  } else {
+    return __uint_as_float(uint32_t(v) << 16);
+  }
+}
+
+// G query heads of one KV head; FP8: e4m3 cache with per-(token, head) scales;
+// WPR warps share one (row, KV head) pair, splitting its list.
+template <int G, bool FP8, int WPR>
+__global__ void __launch_bounds__(128)
+    sparse_mma_kernel(const __nv_bfloat16* __restrict__ Q, const void* __restrict__ Kp,
+                      const void* __restrict__ Vp, const float* __restrict__ ks,
+                      const float* __restrict__ vs, const int32_t* __restrict__ idx,
+                      __nv_bfloat16* __restrict__ O, float* __restrict__ lse, int64_t rows,
+                      int Hkv, int kw, float scale_log2, int64_t cache_T) {
+  constexpr int NT = G > 8 ? G / 8 : 1;  // 8-head n-tiles
+  constexpr int NW = 4;                  // warps per CTA
+  constexpr int PAIRS = NW / WPR;        // (row, KV head) pairs per CTA
+  constexpr bool F16 = FP8;              // FP8 path: f16 MMA; bf16 path: bf16 MMA
+  __shared__ uint16_t sP[NW][NT][8 * 16];
+  __shared__ float sM[NW][NT * 8], sL[NW][NT * 8];
+  __shared__ float sO[WPR > 1 ? NW : 1][WPR > 1 ? NT * 8 : 1][WPR > 1 ? 128 : 1];
+
+  const int warp = warp_id(), lane = lane_id();
+  const int gid = lane >> 2, t = lane & 3;
+  const int64_t pair = int64_t(blockIdx.x) * PAIRS + warp / WPR;
+  const int part = warp % WPR;
+  const bool active = pair < rows * Hkv;
+  const int64_t r = active ? pair / Hkv : 0;
+  const int g = active ? int(pair % Hkv) : 0;
   const int Hq = Hkv * G;
-  const int64_t tok0 = FP8 ? r * cache_T : 0;  // decode: sequence r's cache
+  const int64_t tok0 = FP8 ? r * cache_T : 0;  // decode: sequence r's cache rows
+  const int32_t* list = idx + (active ? pair : 0) * kw;
+  const int per = (kw + WPR - 1) / WPR;
+  const int e_lo = part * per, e_hi = min(kw, e_lo + per);
 
-  // queries of the group, pre-scaled to the base-2 logit domain
+  // query fragments: head nt*8+gid, dims 32t..32t+31 (words 2s, 2s+1 of step s)
+  uint32_t qf[NT][8][2];
 #pragma unroll
-  for (int h = 0; h < G; ++h) {
-    const uint2 v = *reinterpret_cast<const uint2*>(Q + (r * Hq + g * G + h) * 128 + lane * 4);
-    sq[w][h][lane * 4 + 0] = bf16lo(v.x) * scale_log2;
-    sq[w][h][lane * 4 + 1] = bf16hi(v.x) * scale_log2;
-    sq[w][h][lane * 4 + 2] = bf16lo(v.y) * scale_log2;
-    sq[w][h][lane * 4 + 3] = bf16hi(v.y) * scale_log2;
+  for (int nt = 0; nt < NT; ++nt) {
+    const int hh = nt * 8 + gid;
+    const bool real = hh < G && active;
+    const uint4* qr = reinterpret_cast<const uint4*>(Q + (r * Hq + g * G + (real ? hh : 0)) * 128 +
+                                                     32 * t);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint4 w = real ? __ldg(qr + u) : make_uint4(0, 0, 0, 0);
+      const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int s = 2 * u + h2;
+        if constexpr (F16) {
+          qf[nt][s][0] = pack2<true>(bf16lo(w4[2 * h2]), bf16hi(w4[2 * h2]));
+          qf[nt][s][1] = pack2<true>(bf16lo(w4[2 * h2 + 1]), bf16hi(w4[2 * h2 + 1]));
+        } else {
+          qf[nt][s][0] = w4[2 * h2];
+          qf[nt][s][1] = w4[2 * h2 + 1];
+        }
+      }
+    }
   }
-  __syncwarp();
 
-  const int32_t* list = idx + pair * kw;
-  float m[G], l[G], acc[G][4];
+  float m_run[NT][2], l_run[NT][2], o[NT][8][4];
 #pragma unroll
-  for (int h = 0; h < G; ++h) {
-    m[h] = -INFINITY;
-    l[h] = 0.f;
-    acc[h][0] = acc[h][1] = acc[h][2] = acc[h][3] = 0.f;
+  for (int nt = 0; nt < NT; ++nt) {
+    m_run[nt][0] = m_run[nt][1] = -INFINITY;
+    l_run[nt][0] = l_run[nt][1] = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[nt][i][0] = o[nt][i][1] = o[nt][i][2] = o[nt][i][3] = 0.f;
   }
 
-  for (int base = 0; base < kw; base += 32) {
-    const int t = base + lane;
-    const int j = t < kw ? list[t] : -1;
-    float s[G];
+  for (int e0 = e_lo; e0 < e_hi && active; e0 += 16) {
+    // positions of this step's 16 list entries (lanes 16-31 repeat 0-15)
+    const int ee = e0 + (lane & 15);
+    const int jl = ee < e_hi ? __ldg(list + ee) : -1;
+    const int jA = __shfl_sync(0xffffffffu, jl, gid), jB = __shfl_sync(0xffffffffu, jl, gid + 8);
+    int jP[4];
 #pragma unroll
-    for (int h = 0; h < G; ++h) s[h] = -INFINITY;
-    float vscale = 0.f;
-    if (j >= 0) {
+    for (int u = 0; u < 4; ++u) jP[u] = __shfl_sync(0xffffffffu, jl, 4 * t + u);
+    const bool vA = jA >= 0, vB = jB >= 0;
+    const int64_t rowA = (tok0 + (vA ? jA : 0)) * Hkv + g;
+    const int64_t rowB = (tok0 + (vB ? jB : 0)) * Hkv + g;
+
+    // ---- gathers: K rows (this lane's 32 dims), V rows 4t+u (16 dims)
+    uint32_t ka[16], kb[16];  // bf16: words; FP8: first 8 hold 32 codes
+    uint32_t vw[4][8];
+    float vsc[4] = {0.f, 0.f, 0.f, 0.f};
+    float ksA = 1.f, ksB = 1.f;
+    if constexpr (!FP8) {
+      const uint4* pa = reinterpret_cast<const uint4*>(
+          reinterpret_cast<const __nv_bfloat16*>(Kp) + rowA * 128 + 32 * t);
+      const uint4* pb = reinterpret_cast<const uint4*>(
+          reinterpret_cast<const __nv_bfloat16*>(Kp) + rowB * 128 + 32 * t);
 #pragma unroll
-      for (int h = 0; h < G; ++h) s[h] = 0.f;
-      const int64_t row = (tok0 + j) * Hkv + g;
+      for (int u = 0; u < 4; ++u) {
+        const uint4 x = __ldg(pa + u), y = __ldg(pb + u);
+        ka[4 * u] = x.x; ka[4 * u + 1] = x.y; ka[4 * u + 2] = x.z; ka[4 * u + 3] = x.w;
+        kb[4 * u] = y.x; kb[4 * u + 1] = y.y; kb[4 * u + 2] = y.z; kb[4 * u + 3] = y.w;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t rv = (tok0 + (jP[u] >= 0 ? jP[u] : 0)) * Hkv + g;
+        const uint4* pv = reinterpret_cast<const uint4*>(
+            reinterpret_cast<const __nv_bfloat16*>(Vp) + rv * 128 + 16 * gid);
+        const uint4 x = __ldg(pv), y = __ldg(pv + 1);
+        vw[u][0] = x.x; vw[u][1] = x.y; vw[u][2] = x.z; vw[u][3] = x.w;
+        vw[u][4] = y.x; vw[u][5] = y.y; vw[u][6] = y.z; vw[u][7] = y.w;
+        vsc[u] = jP[u] >= 0 ? 1.f : 0.f;
+      }
+    } else {
+      const uint4* pa = reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(Kp) +
+                                                       rowA * 128 + 32 * t);
+      const uint4* pb = reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(Kp) +
+                                                       rowB * 128 + 32 * t);
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const uint4 x = __ldg(pa + u), y = __ldg(pb + u);
+        ka[4 * u] = x.x; ka[4 * u + 1] = x.y; ka[4 * u + 2] = x.z; ka[4 * u + 3] = x.w;
+        kb[4 * u] = y.x; kb[4 * u + 1] = y.y; kb[4 * u + 2] = y.z; kb[4 * u + 3] = y.w;
+      }
+      ksA = vA ? __ldg(ks + rowA) : 0.f;
+      ksB = vB ? __ldg(ks + rowB) : 0.f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t rv = (tok0 + (jP[u] >= 0 ? jP[u] : 0)) * Hkv + g;
+        const uint4 x = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(Vp) +
+                                                             rv * 128 + 16 * gid));
+        vw[u][0] = x.x; vw[u][1] = x.y; vw[u][2] = x.z; vw[u][3] = x.w;
+        vsc[u] = jP[u] >= 0 ? __ldg(vs + rv) * kPScale : 0.f;
+      }
+    }
+
+    // ---- S^T = K Q^T
+    float sacc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      uint32_t a0, a1, a2, a3;
       if constexpr (!FP8) {
-        const uint4* kr = reinterpret_cast<const uint4*>(
-            reinterpret_cast<const __nv_bfloat16*>(Kp) + row * 128);
-#pragma unroll 4
-        for (int c = 0; c < 16; ++c) {
-          const uint4 u = __ldg(kr + c);
-          const float k8[8] = {bf16lo(u.x), bf16hi(u.x), bf16lo(u.y), bf16hi(u.y),
-                               bf16lo(u.z), bf16hi(u.z), bf16lo(u.w), bf16hi(u.w)};
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const float4 q0 = *reinterpret_cast<const float4*>(&sq[w][h][c * 8]);
-            const float4 q1 = *reinterpret_cast<const float4*>(&sq[w][h][c * 8 + 4]);
-            s[h] += q0.x * k8[0] + q0.y * k8[1] + q0.z * k8[2] + q0.w * k8[3] + q1.x * k8[4] +
-                    q1.y * k8[5] + q1.z * k8[6] + q1.w * k8[7];
-          }
-        }
+        a0 = ka[2 * s];      // row gid, dims 32t+4s+{0,1}
+        a1 = kb[2 * s];      // row gid+8
+        a2 = ka[2 * s + 1];  // row gid, dims 32t+4s+{2,3}
+        a3 = kb[2 * s + 1];
       } else {
-        const uint4* kr =
-            reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(Kp) + row * 128);
-#pragma unroll 2
-        for (int c = 0; c < 8; ++c) {
-          const uint4 u = __ldg(kr + c);
-          const uint32_t wds[4] = {u.x, u.y, u.z, u.w};
-          float k16[16];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float2 a = e4m3x2_to_float2(uint16_t(wds[q] & 0xFFFF));
-            const float2 b = e4m3x2_to_float2(uint16_t(wds[q] >> 16));
-            k16[4 * q + 0] = a.x;
-            k16[4 * q + 1] = a.y;
-            k16[4 * q + 2] = b.x;
-            k16[4 * q + 3] = b.y;
-          }
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            float acc_h = 0.f;
-#pragma unroll
-            for (int e = 0; e < 16; e += 4) {
-              const float4 qv = *reinterpret_cast<const float4*>(&sq[w][h][c * 16 + e]);
-              acc_h += qv.x * k16[e] + qv.y * k16[e + 1] + qv.z * k16[e + 2] + qv.w * k16[e + 3];
-            }
-            s[h] += acc_h;
-          }
-        }
-        const float kscale = __ldg(ks + row);
-#pragma unroll
-        for (int h = 0; h < G; ++h) s[h] *= kscale;
-        vscale = __ldg(vs + row);
+        a0 = e4m3x2_f16x2(ka[s]);
+        a1 = e4m3x2_f16x2(kb[s]);
+        a2 = e4m3x2_f16x2(ka[s] >> 16);
+        a3 = e4m3x2_f16x2(kb[s] >> 16);
       }
-    }
-    // online softmax, base 2
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const float bm = warp_max(s[h]);
-      const float mn = fmaxf(m[h], bm);
-      float p = 0.f, alpha = 1.f;
-      if (mn != -INFINITY) {
-        alpha = fast_exp2(m[h] - mn);  // m = -inf -> 0
-        p = j >= 0 ? fast_exp2(s[h] - mn) : 0.f;
-      }
-      l[h] = l[h] * alpha + warp_sum(p);
-      acc[h][0] *= alpha;
-      acc[h][1] *= alpha;
-      acc[h][2] *= alpha;
-      acc[h][3] *= alpha;
-      m[h] = mn;
-      sp[w][h][lane] = p;
+      for (int nt = 0; nt < NT; ++nt) mma16816<F16>(sacc[nt], a0, a1, a2, a3, qf[nt][s][0], qf[nt][s][1]);
     }
-    sj[w][lane] = j;
-    svs[w][lane] = vscale;
+
+    // ---- online softmax (base 2), lane: keys gid / gid+8, heads 2t, 2t+1
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int h0 = nt * 8 + 2 * t;
+      const float cA = scale_log2 * ksA, cB = scale_log2 * ksB;
+      float s00 = vA ? sacc[nt][0] * cA : -INFINITY, s01 = vA ? sacc[nt][1] * cA : -INFINITY;
+      float s10 = vB ? sacc[nt][2] * cB : -INFINITY, s11 = vB ? sacc[nt][3] * cB : -INFINITY;
+      if (h0 >= G) s00 = s10 = -INFINITY;
+      if (h0 + 1 >= G) s01 = s11 = -INFINITY;
+      float mx0 = fmaxf(s00, s10), mx1 = fmaxf(s01, s11);
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+      }
+      const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
+      const float al0 = mn0 == -INFINITY ? 1.f : fast_exp2(m_run[nt][0] - mn0);
+      const float al1 = mn1 == -INFINITY ? 1.f : fast_exp2(m_run[nt][1] - mn1);
+      const float p00 = mn0 == -INFINITY ? 0.f : fast_exp2(s00 - mn0);
+      const float p10 = mn0 == -INFINITY ? 0.f : fast_exp2(s10 - mn0);
+      const float p01 = mn1 == -INFINITY ? 0.f : fast_exp2(s01 - mn1);
+      const float p11 = mn1 == -INFINITY ? 0.f : fast_exp2(s11 - mn1);
+      m_run[nt][0] = mn0;
+      m_run[nt][1] = mn1;
+      l_run[nt][0] = l_run[nt][0] * al0 + p00 + p10;
+      l_run[nt][1] = l_run[nt][1] * al1 + p01 + p11;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        o[nt][i][0] *= al0;
+        o[nt][i][2] *= al0;
+        o[nt][i][1] *= al1;
+        o[nt][i][3] *= al1;
+      }
+      uint16_t* sp = sP[warp][nt];  // [head][key]
+      sp[(2 * t) * 16 + gid] = one16<F16>(p00);
+      sp[(2 * t + 1) * 16 + gid] = one16<F16>(p01);
+      sp[(2 * t) * 16 + gid + 8] = one16<F16>(p10);
+      sp[(2 * t + 1) * 16 + gid + 8] = one16<F16>(p11);
+    }
     __syncwarp();
-    const int nb = min(32, kw - base);
-    for (int tt = 0; tt < nb; ++tt) {
-      const int jj = sj[w][tt];
-      if (jj < 0) continue;
-      const int64_t row = (tok0 + jj) * Hkv + g;
-      float v4[4];
-      if constexpr (!FP8) {
-        const uint2 u = __ldg(reinterpret_cast<const uint2*>(
-            reinterpret_cast<const __nv_bfloat16*>(Vp) + row * 128 + lane * 4));
-        v4[0] = bf16lo(u.x);
-        v4[1] = bf16hi(u.x);
-        v4[2] = bf16lo(u.y);
-        v4[3] = bf16hi(u.y);
-      } else {
-        const uint32_t u = __ldg(reinterpret_cast<const uint32_t*>(
-            reinterpret_cast<const uint8_t*>(Vp) + row * 128 + lane * 4));
-        const float2 a = e4m3x2_to_float2(uint16_t(u & 0xFFFF));
-        const float2 b = e4m3x2_to_float2(uint16_t(u >> 16));
-        const float sv = svs[w][tt];
-        v4[0] = a.x * sv;
-        v4[1] = a.y * sv;
-        v4[2] = b.x * sv;
-        v4[3] = b.y * sv;
+    // ---- O^T += V^T P^T: K slots {2t,2t+1,2t+8,2t+9} = keys 4t+{0,1,2,3};
+    // MMA i, row gid -> dim 16*gid+2i, row gid+8 -> dim 16*gid+2i+1
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const uint16_t* sp = sP[warp][nt] + gid * 16 + 4 * t;
+      const uint32_t b0 = pack2<F16>(from16<F16>(sp[0]) * vsc[0], from16<F16>(sp[1]) * vsc[1]);
+      const uint32_t b1 = pack2<F16>(from16<F16>(sp[2]) * vsc[2], from16<F16>(sp[3]) * vsc[3]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        uint32_t a0, a1, a2, a3;
+        if constexpr (!FP8) {
+          // word i of a row slice = dims 16*gid+2i (low), +1 (high)
+          a0 = __byte_perm(vw[0][i], vw[1][i], 0x5410);
+          a1 = __byte_perm(vw[0][i], vw[1][i], 0x7632);
+          a2 = __byte_perm(vw[2][i], vw[3][i], 0x5410);
+          a3 = __byte_perm(vw[2][i], vw[3][i], 0x7632);
+        } else {
+          // byte 2i / 2i+1 of a row slice = dims 16*gid+2i / +1
+          const int wd = i >> 1, sh = (i & 1) * 16;
+          const uint32_t r0 = vw[0][wd] >> sh, r1 = vw[1][wd] >> sh;
+          const uint32_t r2 = vw[2][wd] >> sh, r3 = vw[3][wd] >> sh;
+          a0 = e4m3x2_f16x2(__byte_perm(r0, r1, 0x0040));
+          a1 = e4m3x2_f16x2(__byte_perm(r0, r1, 0x0051));
+          a2 = e4m3x2_f16x2(__byte_perm(r2, r3, 0x0040));
+          a3 = e4m3x2_f16x2(__byte_perm(r2, r3, 0x0051));
+        }
+        mma16816<F16>(o[nt][i], a0, a1, a2, a3, b0, b1);
+      }
+    }
+    __syncwarp();
+  }
+
+  // ---- finish: l over the lanes of a head, then (optionally) combine the
+  // WPR warps of the pair, then O = o / l, lse
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      float l = l_run[nt][e];
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+      l_run[nt][e] = l;
+    }
+  const float oscale = FP8 ? 1.f / kPScale : 1.f;
+  if constexpr (WPR == 1) {
+    if (!active) return;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int h = nt * 8 + 2 * t + e;
+        if (h >= G) continue;
+        const float l = l_run[nt][e];
+        const float inv = l > 0.f ? oscale / l : 0.f;
+        uint32_t pk[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(o[nt][i][e] * inv, o[nt][i][e + 2] * inv);
+        uint4* dst = reinterpret_cast<uint4*>(O + (r * Hq + g * G + h) * 128 + 16 * gid);
+        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        if (lse != nullptr && gid == 0)
+          lse[r * Hq + g * G + h] = l > 0.f ? (m_run[nt][e] + __log2f(l)) * kLn2 : -INFINITY;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      if (gid == 0) {
+        sM[warp][nt * 8 + 2 * t] = m_run[nt][0];
+        sM[warp][nt * 8 + 2 * t + 1] = m_run[nt][1];
+        sL[warp][nt * 8 + 2 * t] = l_run[nt][0];
+        sL[warp][nt * 8 + 2 * t + 1] = l_run[nt][1];
       }
 #pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        sO[warp][nt * 8 + 2 * t][16 * gid + 2 * i] = o[nt][i][0];
+        sO[warp][nt * 8 + 2 * t + 1][16 * gid + 2 * i] = o[nt][i][1];
+        sO[warp][nt * 8 + 2 * t][16 * gid + 2 * i + 1] = o[nt][i][2];
+        sO[warp][nt * 8 + 2 * t + 1][16 * gid + 2 * i + 1] = o[nt][i][3];
+      }
+    }
+    __syncthreads();
+    if (part == 0 && active) {
+      const int w0 = warp;  // first warp of this pair
       for (int h = 0; h < G; ++h) {
-        const float p = sp[w][h][tt];
-        acc[h][0] += p * v4[0];
-        acc[h][1] += p * v4[1];
-        acc[h][2] += p * v4[2];
-        acc[h][3] += p * v4[3];
+        float M = -INFINITY;
+        for (int w2 = 0; w2 < WPR; ++w2) M = fmaxf(M, sM[w0 + w2][h]);
+        float L = 0.f, f[WPR];
+        for (int w2 = 0; w2 < WPR; ++w2) {
+          f[w2] = M == -INFINITY ? 0.f : fast_exp2(sM[w0 + w2][h] - M);
+          L += sL[w0 + w2][h] * f[w2];
+        }
+        const float inv = L > 0.f ? oscale / L : 0.f;
+        for (int d = lane; d < 128; d += 32) {
+          float acc = 0.f;
+          for (int w2 = 0; w2 < WPR; ++w2) acc += sO[w0 + w2][h][d] * f[w2];
+          O[(r * Hq + g * G + h) * 128 + d] = __float2bfloat16_rn(acc * inv);
+        }
+        if (lse != nullptr && lane == 0)
+          lse[r * Hq + g * G + h] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
       }
     }
-    __syncwarp();
-  }
-
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    const float inv = l[h] > 0.f ? 1.f / l[h] : 0.f;
-    uint2 o;
-    o.x = pack_bf16x2(acc[h][0] * inv, acc[h][1] * inv);
-    o.y = pack_bf16x2(acc[h][2] * inv, acc[h][3] * inv);
-    *reinterpret_cast<uint2*>(O + (r * Hq + g * G + h) * 128 + lane * 4) = o;
-    if (lse != nullptr && lane == 0)
-      lse[r * Hq + g * G + h] = l[h] > 0.f ? (m[h] + __log2f(l[h])) * kLn2 : -INFINITY;
   }
 }
 
 template <int G>
 cudaError_t launch_g(const SparseArgs& a, cudaStream_t stream) {
   const int64_t pairs = a.T * a.Hkv;
-  const dim3 grid(unsigned((pairs + WARPS - 1) / WARPS));
   const float sl2 = a.scale * kLog2e;
   if (a.Kc != nullptr) {
-    sparse_attn_kernel<G, true><<<grid, WARPS * 32, 0, stream>>>(
+    // decode: few pairs, each split over the 4 warps of one CTA
+    sparse_mma_kernel<G, true, 4><<<unsigned(pairs), 128, 0, stream>>>(
         reinterpret_cast<const __nv_bfloat16*>(a.Q), a.Kc, a.Vc, a.ks, a.vs, a.idx,
         reinterpret_cast<__nv_bfloat16*>(a.O), a.lse, a.T, a.Hkv, a.kw, sl2, a.cache_T);
   } else {
-    sparse_attn_kernel<G, false><<<grid, WARPS * 32, 0, stream>>>(
+    sparse_mma_kernel<G, false, 1><<<unsigned((pairs + 3) / 4), 128, 0, stream>>>(
         reinterpret_cast<const __nv_bfloat16*>(a.Q), a.K, a.V, nullptr, nullptr, a.idx,
         reinterpret_cast<__nv_bfloat16*>(a.O), a.lse, a.T, a.Hkv, a.kw, sl2, 0);
   }
