@@ -129,6 +129,32 @@ hs2_status hs2_select_topk(const hs2_bf16* Q, const hs2_bf16* K, const float* ls
                            void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * hs2_select_topk without a workspace argument.  No counterpart on the pages:
+ * this exists for callers that cannot allocate device memory themselves, for
+ * example a host program whose device memory is owned and budgeted by another
+ * runtime's allocator, or code on a latency-critical path that must not call
+ * cudaMalloc (which may synchronise the device).  It computes exactly what
+ * hs2_select_topk computes, with the same arguments minus the workspace, and
+ * allocates nothing: its scratch is a 48 MiB array inside the library that
+ * every GPU loading the library holds until the process exits.
+ *   - The first call on a device looks up that array's device address (once
+ *     per device, with the device current); make that first call before any
+ *     stream capture.
+ *   - The array is shared by all calls on a device and keeps the last call's
+ *     contents (none of it needs to start at zero).  Calls whose kernels
+ *     overlap on the same device, e.g. on two streams, race on it: serialise
+ *     them.
+ *   - The kernel runs as many persistent CTAs as the scratch holds; each needs
+ *     4 * (128 / G) * max(2 * k_global, 256) * 8 + 65536 bytes.  A shape for
+ *     which one CTA does not fit returns HS2_ERR_UNSUPPORTED.
+ * Errors otherwise as hs2_select_topk (HS2_ERR_CUDA if the address lookup
+ * fails).
+ */
+hs2_status hs2_select_topk_noalloc(const hs2_bf16* Q, const hs2_bf16* K, const float* lse,
+                                   int32_t* idx, float* kth_score, const hs2_shape* shape,
+                                   void* stream);
+
+/*
  * Sparse attention over the shared K/V and index list (step S4, KV Reuse).
  * KV Reuse paragraph of the javabetter.cn explainer and the aitop.news
  * summary: each sparse layer has its own queries, reuses the full layer's K/V

@@ -51,6 +51,7 @@ def _load(path: str = LIB_PATH):
         "hs2_bridge_kv": [P, I32, P, P, P, P, SP, P],
         "hs2_full_attn_lse": [P, P, P, P, P, SP, P],
         "hs2_select_topk": [P, P, P, P, P, SP, P, SZ, P],
+        "hs2_select_topk_noalloc": [P, P, P, P, P, SP, P],
         "hs2_sparse_attn": [P, P, P, P, P, P, SP, P],
         "hs2_block_prefill": [P, I32, P, P, P, P, P, P, P, P, I32, PP, PP, SP, P, SZ, P],
         "hs2_block_decode": [I32, C.POINTER(C.c_int64), P, P, P, P, P, P, P, P, I32, PP, PP, SP,
@@ -72,7 +73,8 @@ def _load(path: str = LIB_PATH):
 
 _lib = _load()
 
-EXPORTED = ["hs2_bridge_kv", "hs2_full_attn_lse", "hs2_select_topk", "hs2_sparse_attn",
+EXPORTED = ["hs2_bridge_kv", "hs2_full_attn_lse", "hs2_select_topk", "hs2_select_topk_noalloc",
+            "hs2_sparse_attn",
             "hs2_block_prefill", "hs2_block_decode", "hs2_workspace_size",
             "hs2_get_device_status", "hs2_status_string", "hs2_kernel_launches"]
 
@@ -132,6 +134,15 @@ def hs2_select_topk(Q, K, lse, idx, kth, shape: Shape, workspace, stream=None):
                                 _ptr(idx, I32T, "idx"), _ptr(kth, F32, "kth", True),
                                 C.byref(shape), _ptr(workspace, U8, "workspace", True), nbytes,
                                 _stream(stream)), "hs2_select_topk")
+
+
+def hs2_select_topk_noalloc(Q, K, lse, idx, kth, shape: Shape, stream=None):
+    """hs2_select_topk on the library's own scratch, for callers that cannot
+    allocate device memory; see include/hs2.h for its limits."""
+    _check(_lib.hs2_select_topk_noalloc(_ptr(Q, BF16, "Q"), _ptr(K, BF16, "K"),
+                                        _ptr(lse, F32, "lse"), _ptr(idx, I32T, "idx"),
+                                        _ptr(kth, F32, "kth", True), C.byref(shape),
+                                        _stream(stream)), "hs2_select_topk_noalloc")
 
 
 def hs2_sparse_attn(Q, K, V, idx, O, lse, shape: Shape, stream=None):

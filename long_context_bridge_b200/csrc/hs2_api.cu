@@ -206,6 +206,19 @@ hs2_status hs2_select_topk(const hs2_bf16* Q, const hs2_bf16* K, const float* ls
   return cuda_status(launch_select(a, static_cast<cudaStream_t>(stream)));
 }
 
+hs2_status hs2_select_topk_noalloc(const hs2_bf16* Q, const hs2_bf16* K, const float* lse,
+                                   int32_t* idx, float* kth, const hs2_shape* s, void* stream) {
+  HS2_TRY(check_shape(s, true));
+  HS2_NEED(Q && K && lse && idx);
+  HS2_NEED(aligned16(Q) && aligned16(K) && aligned16(lse) && aligned16(idx));
+  HS2_NEED(kth == nullptr || aligned16(kth));
+  SelectArgs a{Q, K, lse, idx, kth, s->T, s->n_q_heads, s->n_kv_heads, s->scale,
+               s->k_global, s->window, nullptr, 0};
+  const cudaError_t e = launch_select_noalloc(a, static_cast<cudaStream_t>(stream));
+  if (e == cudaErrorNotSupported) return HS2_ERR_UNSUPPORTED;
+  return cuda_status(e);
+}
+
 hs2_status hs2_sparse_attn(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V,
                            const int32_t* idx, hs2_bf16* O, float* lse, const hs2_shape* s,
                            void* stream) {

@@ -68,6 +68,9 @@ struct SelectArgs {
 };
 size_t select_workspace_bytes(int64_t T, int Hq, int Hkv, int k, int w);
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);
+// same kernel on the library's own file-scope scratch (no workspace argument)
+size_t select_noalloc_scratch_bytes();
+cudaError_t launch_select_noalloc(const SelectArgs& a, cudaStream_t stream);
 
 struct SparseArgs {
   const void* Q;

@@ -36,6 +36,8 @@
 //     sorted ascending by a register bitonic sort.
 // Items whose every query has at most k candidates skip the scoring: all
 // candidates are selected.
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -641,6 +643,69 @@ cudaError_t launch_g(const SelectArgs& a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Variant without caller-provided workspace.  Its scratch (the per-query
+// candidate sub-buffers and the sort staging of every CTA) is this file-scope
+// array; the persistent kernel simply runs as many CTAs as the array can
+// hold.  Nothing in it has to start at zero: every word a CTA reads was
+// written earlier in the same call.  Each device has its own copy; all calls
+// on one device share it, so calls whose kernels overlap on that device (for
+// example on two streams) race on it.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = size_t(48) << 20;
+static __device__ __align__(256) unsigned char g_select_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+
+// Device address of g_select_scratch on the current device, looked up once
+// per device (host code must not use the symbol itself as an address).
+cudaError_t select_scratch_address(void** out) {
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_select_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return cudaSuccess;
+}
+
+size_t noalloc_cta_bytes(int QT, int k) {
+  return size_t(4) * QT * buffer_cap(k) * sizeof(uint2) + size_t(8) * 2048 * sizeof(uint32_t);
+}
+
+template <int G>
+cudaError_t launch_noalloc_g(const SelectArgs& a, void* scratch, cudaStream_t stream) {
+  constexpr int QT = TILE / G;
+  const int fit = int(kNoAllocScratchBytes / noalloc_cta_bytes(QT, a.k));
+  if (fit < 1) return cudaErrorNotSupported;
+  CUtensorMap tmQ, tmK;
+  if (!make_tmap_3d(&tmQ, a.Q, 128, a.Hq, a.T, 256, uint64_t(a.Hq) * 256, 64, G, QT))
+    return cudaErrorInvalidValue;
+  if (!make_tmap_3d(&tmK, a.K, 128, a.Hkv, a.T, 256, uint64_t(a.Hkv) * 256, 64, 1, TILE))
+    return cudaErrorInvalidValue;
+  const int kst = stages_for<G>();
+  const int smem = OFF_K + kst * TILE_BYTES + int(sizeof(Misc<G>)) + 1024;
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(select_kernel<G>), smem);
+  if (e != cudaSuccess) return e;
+  const int n_items = int((a.T + QT - 1) / QT) * a.Hkv;
+  const int grid = min(min(sm_count(), n_items), fit);
+  uint2* ws = reinterpret_cast<uint2*>(scratch);
+  uint32_t* wsort = reinterpret_cast<uint32_t*>(ws + size_t(grid) * 4 * QT * buffer_cap(a.k));
+  select_kernel<G><<<grid, THREADS, smem, stream>>>(tmQ, tmK, a.lse, a.idx, a.kth, ws, wsort,
+                                                    int(a.T), a.Hkv, a.k, a.w, buffer_cap(a.k),
+                                                    kst, a.scale * kLog2e);
+  count_launch();
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 size_t select_workspace_bytes(int64_t T, int Hq, int Hkv, int k, int w) {
@@ -649,6 +714,22 @@ size_t select_workspace_bytes(int64_t T, int Hq, int Hkv, int k, int w) {
   const int QT = TILE / (Hq / Hkv);
   return size_t(sm_count()) * (size_t(4) * QT * buffer_cap(k) * sizeof(uint2) +
                                size_t(8) * 2048 * sizeof(uint32_t));
+}
+
+size_t select_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+cudaError_t launch_select_noalloc(const SelectArgs& a, cudaStream_t stream) {
+  void* scratch = nullptr;
+  cudaError_t e = select_scratch_address(&scratch);
+  if (e != cudaSuccess) return e;
+  switch (a.Hq / a.Hkv) {
+    case 1: return launch_noalloc_g<1>(a, scratch, stream);
+    case 2: return launch_noalloc_g<2>(a, scratch, stream);
+    case 4: return launch_noalloc_g<4>(a, scratch, stream);
+    case 8: return launch_noalloc_g<8>(a, scratch, stream);
+    case 16: return launch_noalloc_g<16>(a, scratch, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream) {
