@@ -47,8 +47,10 @@ HS2_STATUS_ACCESSOR(status_select)
 
 namespace {
 
-constexpr int THREADS = 320;   // producer warp, MMA warp, 8 scorer warps
-constexpr int SCORERS = 256;
+constexpr int SETS = 4;                      // scorer warp sets (query quarters)
+constexpr int SCORER_WARPS = 4 * SETS;       // one warp per (set, TMEM lane quarter)
+constexpr int SCORERS = 32 * SCORER_WARPS;
+constexpr int THREADS = 64 + SCORERS;        // producer warp, MMA warp, scorers
 constexpr int TILE = 128;
 constexpr int CHUNK = TILE * 128;
 constexpr int TILE_BYTES = 2 * CHUNK;
@@ -61,13 +63,12 @@ constexpr float kLog2e = 1.4426950408889634f;
 template <int G>
 struct SelCfg {
   static constexpr int QT = TILE / G;                 // queries per item
-  static constexpr int QH = QT / 2;                   // queries per scorer half
+  static constexpr int QH = QT / SETS;                // queries per scorer set (32 columns)
   static constexpr int NB = QT <= 32 ? 256 : 64;      // histogram bins per query
   static constexpr int BSHIFT = QT <= 32 ? 20 : 22;   // bin width: 2^-3 or 2^-1 binade
-  // queries scored per group: at least one 32-column chunk, at most 8
-  static constexpr int QG = (32 / G > 8) ? 32 / G : (QH < 8 ? QH : 8);
-  static constexpr int NG = QH / QG;                  // groups per tile
-  static constexpr int CPG = QG * G / 32;             // 32-column chunks per group
+  static constexpr int QG = QH;                       // queries scored per group
+  static constexpr int NG = 1;                        // groups per tile
+  static constexpr int CPG = 1;                       // 32-column chunks per group
 };
 
 struct Bars {
@@ -85,7 +86,7 @@ struct Misc {
   uint32_t floor_bin[QT];     // candidates need bin >= floor_bin
   uint32_t cnt[4][QT];        // entries in each sub-buffer
   uint32_t hist[QT][NB];      // appended entries per score bin
-  uint32_t dig[8][256];       // per-warp radix histograms of the final select
+  uint32_t dig[SCORER_WARPS][256];  // per-warp radix histograms of the final select
 };
 
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int ks) {
@@ -93,7 +94,7 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int ks) {
 }
 
 __device__ __forceinline__ void scorer_sync() {
-  asm volatile("bar.sync 1, 256;" ::: "memory");
+  asm volatile("bar.sync 1, %0;" ::"n"(SCORERS) : "memory");
 }
 
 // Ranking key: larger is better; equal scores rank the smaller position first.
@@ -393,10 +394,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else {
     // -------------------------------- scorers -------------------------------
-    const int sw = warp - 2;          // scorer warp 0..7
-    const int half = sw >> 2;         // which half of the item's queries
+    const int sw = warp - 2;          // scorer warp 0..SCORER_WARPS-1
+    const int half = sw >> 2;         // which set (quarter) of the item's queries
     const int sub = warp & 3;         // TMEM lane quarter = key quarter of a tile
-    const int tid = threadIdx.x - 64; // 0..255
+    const int tid = threadIdx.x - 64; // 0..SCORERS-1
     const uint32_t lane_addr = uint32_t(sub * 32) << 16;
     const uint32_t lt_mask = (1u << lane) - 1u;
     uint2* my_bufs = ws + (size_t(blockIdx.x) * 4 + sub) * QT * capw;  // [QT][capw]
@@ -510,8 +511,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       scorer_sync();
       // ---- outputs of the item: one warp per query ----
-      uint32_t* sp = wsort + (size_t(blockIdx.x) * 8 + sw) * 2048;  // staging of positions
-      for (int q = sw; q < QT; q += 8) {
+      uint32_t* sp = wsort + (size_t(blockIdx.x) * SCORER_WARPS + sw) * 2048;  // staging
+      for (int q = sw; q < QT; q += SCORER_WARPS) {
         const int qpos = q0 + q;
         if (qpos >= T) continue;
         const int ncand = max(0, qpos - w + 1);
@@ -678,7 +679,7 @@ cudaError_t select_scratch_address(void** out) {
 }
 
 size_t noalloc_cta_bytes(int QT, int k) {
-  return size_t(4) * QT * buffer_cap(k) * sizeof(uint2) + size_t(8) * 2048 * sizeof(uint32_t);
+  return size_t(4) * QT * buffer_cap(k) * sizeof(uint2) + size_t(SCORER_WARPS) * 2048 * sizeof(uint32_t);
 }
 
 template <int G>
@@ -713,7 +714,7 @@ size_t select_workspace_bytes(int64_t T, int Hq, int Hkv, int k, int w) {
   (void)w;
   const int QT = TILE / (Hq / Hkv);
   return size_t(sm_count()) * (size_t(4) * QT * buffer_cap(k) * sizeof(uint2) +
-                               size_t(8) * 2048 * sizeof(uint32_t));
+                               size_t(SCORER_WARPS) * 2048 * sizeof(uint32_t));
 }
 
 size_t select_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
