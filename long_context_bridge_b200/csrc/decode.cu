@@ -77,12 +77,6 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// byte x (0..15) of a uint4
-__device__ __forceinline__ uint32_t byte_of(const uint4& v, int x) {
-  const uint32_t w = x < 4 ? v.x : x < 8 ? v.y : x < 12 ? v.z : v.w;
-  return (w >> (8 * (x & 3))) & 0xFFu;
-}
-
 // ---------------------------------------------------------------------------
 // decode_partial: grid (chunks, Hkv, B), DP_WARPS warps
 // ---------------------------------------------------------------------------
@@ -242,15 +236,21 @@ __global__ void __launch_bounds__(DP_WARPS * 32)
       const float f3 = __half2float(*reinterpret_cast<const __half*>(sp + 3)) * vsc[3];
       // vsc already carries the 2^10 factor (see below)
       const uint32_t b0 = pack_f16x2(f0, f1), b1 = pack_f16x2(f2, f3);
+      const uint32_t vw[4][4] = {{vr[0].x, vr[0].y, vr[0].z, vr[0].w},
+                                 {vr[1].x, vr[1].y, vr[1].z, vr[1].w},
+                                 {vr[2].x, vr[2].y, vr[2].z, vr[2].w},
+                                 {vr[3].x, vr[3].y, vr[3].z, vr[3].w}};
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        // dims 16*gid + 2i (MMA row gid) and 16*gid + 2i + 1 (row gid+8)
-        const uint32_t a0 = cvt_e4m3x2_f16x2(byte_of(vr[0], 2 * i) | (byte_of(vr[1], 2 * i) << 8));
-        const uint32_t a1 =
-            cvt_e4m3x2_f16x2(byte_of(vr[0], 2 * i + 1) | (byte_of(vr[1], 2 * i + 1) << 8));
-        const uint32_t a2 = cvt_e4m3x2_f16x2(byte_of(vr[2], 2 * i) | (byte_of(vr[3], 2 * i) << 8));
-        const uint32_t a3 =
-            cvt_e4m3x2_f16x2(byte_of(vr[2], 2 * i + 1) | (byte_of(vr[3], 2 * i + 1) << 8));
+        // bytes 2i / 2i+1 of a row slice = dims 16*gid + 2i (MMA row gid) and
+        // 16*gid + 2i + 1 (row gid+8); pair the two keys' bytes with a permute
+        const int wd = i >> 1, sh = (i & 1) * 16;
+        const uint32_t r0 = vw[0][wd] >> sh, r1 = vw[1][wd] >> sh;
+        const uint32_t r2 = vw[2][wd] >> sh, r3 = vw[3][wd] >> sh;
+        const uint32_t a0 = cvt_e4m3x2_f16x2(__byte_perm(r0, r1, 0x0040));
+        const uint32_t a1 = cvt_e4m3x2_f16x2(__byte_perm(r0, r1, 0x0051));
+        const uint32_t a2 = cvt_e4m3x2_f16x2(__byte_perm(r2, r3, 0x0040));
+        const uint32_t a3 = cvt_e4m3x2_f16x2(__byte_perm(r2, r3, 0x0051));
         mma_f16(o[nt][i], a0, a1, a2, a3, b0, b1);
       }
     }

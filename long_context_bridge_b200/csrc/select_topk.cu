@@ -10,7 +10,7 @@
 // Persistent kernel, one CTA per SM, work item = (128/G queries, KV head):
 //   warp 0     TMA: the item's Q tile once, K tiles into a ring
 //   warp 1     TMEM owner; one lane issues S^T = K Q^T (M = 128 keys,
-//              N = 128 (query, head) rows) into TMEM buffer t%2
+//              N = 128 (query, head) rows) into one of four TMEM buffers
 //   warps 2-9  scorers, two per TMEM lane quarter: thread = key (TMEM lane);
 //              warps 2-5 take the first half of the item's queries (columns
 //              0-63), warps 6-9 the second half; a thread sums
@@ -57,6 +57,7 @@ constexpr int TILE_BYTES = 2 * CHUNK;
 constexpr int OFF_Q = 0;
 constexpr int OFF_K = OFF_Q + TILE_BYTES;
 constexpr int MAX_STAGES = 4;
+constexpr int NSB = 4;          // S^T buffers in TMEM (128 columns each)
 constexpr uint32_t IDESC = idesc_bf16(128, 128, 0, 0);
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -74,7 +75,7 @@ struct SelCfg {
 struct Bars {
   uint64_t q_full, q_empty;
   uint64_t k_full[MAX_STAGES], k_empty[MAX_STAGES];
-  uint64_t s_full[2], s_empty[2];
+  uint64_t s_full[NSB], s_empty[NSB];
   uint32_t tmem_slot;
 };
 
@@ -320,14 +321,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&br->k_full[s], 1);
       mbar_init(&br->k_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NSB; ++b) {
       mbar_init(&br->s_full[b], 1);
       mbar_init(&br->s_empty[b], SCORERS);
     }
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(&br->tmem_slot, 256);
+    tmem_alloc(&br->tmem_slot, NSB * 128);
     tc_fence_before();
   }
   __syncthreads();
@@ -377,9 +378,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!score) continue;
         if (!mbar_wait(&br->q_full, qn & 1)) { ok = false; break; }
         for (int t = 0; t < n_tiles; ++t, ++kt, ++st) {
-          const int s = kt % kst, b = st & 1;
+          const int s = kt % kst, b = st % NSB;
           if (!mbar_wait(&br->k_full[s], (kt / kst) & 1)) { ok = false; break; }
-          if (st >= 2 && !mbar_wait(&br->s_empty[b], ((st >> 1) & 1) ^ 1)) { ok = false; break; }
+          if (st >= NSB && !mbar_wait(&br->s_empty[b], ((st / NSB) & 1) ^ 1)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sK = smem_u32(smem + OFF_K + s * TILE_BYTES);
 #pragma unroll
@@ -418,8 +419,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int i = tid; i < QT * NB; i += SCORERS) (&ms->hist[0][0])[i] = 0;
       scorer_sync();
       for (int t = 0; t < n_tiles; ++t, ++st) {
-        const int b = st & 1;
-        ok = ok && mbar_wait(&br->s_full[b], (st >> 1) & 1);
+        const int b = st % NSB;
+        ok = ok && mbar_wait(&br->s_full[b], (st / NSB) & 1);
         tc_fence_after();
         const int j = t * TILE + sub * 32 + lane;  // this thread's key
         const bool all_cand = (t + 1) * TILE - 1 + w <= q0;
@@ -601,7 +602,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, NSB * 128);
   }
 }
 
