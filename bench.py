@@ -51,32 +51,12 @@ def peaks():
 # inputs (seeded, on the device)
 # ---------------------------------------------------------------------------
 def make_inputs(cfg, device):
-    T, dm, Hq, Hkv = cfg.T, cfg.d_model, cfg.n_q_heads, cfg.n_kv_heads
-    N = Hkv * 128
-    g = lambda tid, n, sd=1.0: synth.normal_bf16_torch(cfg.seed, tid, 0, n, sd, device=device)
-    H = g(synth.TID_H, T * dm).view(T, dm)
-    Wk = g(synth.TID_WK, dm * N, dm ** -0.5).view(dm, N)
-    Wv = g(synth.TID_WV, dm * N, dm ** -0.5).view(dm, N)
-    u = torch.from_numpy(synth.needle_dirs(cfg)).to(device)            # [Hkv, d] fp64
-
-    def qmix(tid):
-        out = torch.empty(T, Hq, 128, dtype=torch.bfloat16, device=device)
-        ug = u.repeat_interleave(cfg.G, 0)[None]
-        rows = 4096
-        for r0 in range(0, T, rows):
-            n = min(rows, T - r0)
-            z = synth.normals_torch(cfg.seed, tid, r0 * Hq * 128, n * Hq * 128, device).view(n, Hq, 128)
-            out[r0:r0 + n] = (0.5 * z + 0.5 * math.sqrt(128) * ug).float().bfloat16()
-        return out
-
-    Q = qmix(synth.TID_Q)
-    Qs = [qmix(synth.TID_QS0 + l) for l in range(cfg.n_sparse)]
-    pos = synth.prefill_needles(cfg)
-    nk = torch.from_numpy(synth.needle_key_bits(cfg).view(np.int16)).to(device).view(torch.bfloat16)
-    needle_rows = torch.cat([torch.from_numpy(p) for p in pos]).to(device)
-    needle_heads = torch.cat([torch.full((len(p),), g_, dtype=torch.int64) for g_, p in enumerate(pos)]).to(device)
-    return dict(H=H, Wk=Wk, Wv=Wv, Q=Q, Qs=Qs, needle_rows=needle_rows, needle_heads=needle_heads,
-                needle_vals=nk[needle_heads])
+    H, Wk, Wv = synth.bridge_inputs_torch(cfg, device=device)
+    Q = synth.q_rows_torch(cfg, synth.TID_Q, device=device)
+    Qs = [synth.q_rows_torch(cfg, synth.TID_QS0 + l, device=device) for l in range(cfg.n_sparse)]
+    rows, heads, vals = synth.needle_scatter_torch(cfg, device=device)
+    return dict(H=H, Wk=Wk, Wv=Wv, Q=Q, Qs=Qs, needle_rows=rows, needle_heads=heads,
+                needle_vals=vals)
 
 
 # ---------------------------------------------------------------------------

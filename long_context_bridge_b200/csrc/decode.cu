@@ -9,10 +9,13 @@
 //
 // Kernels (all on `stream`):
 //   decode_partial  split-KV attention of the G query heads of (b, g) over a
-//                   4096-key chunk with mma.sync m16n8k16 (e4m3 codes -> f16
-//                   exactly, fp32 accumulation).  The dot-product dimension
-//                   and the output dims are permuted so every lane reads 16
-//                   contiguous bytes of a K or V row (fully coalesced rows).
+//                   4096-key chunk: a producer warp streams 64-row K and V
+//                   tiles by TMA (128-byte swizzle) into a shared
+//                   memory ring (3 stages); four warps each take 16 keys of a stage and
+//                   run mma.sync m16n8k16 (e4m3 codes -> f16 exactly, fp32
+//                   accumulation).  The dot-product dimension and the output
+//                   dims are permuted so every lane reads 16 contiguous bytes
+//                   of a K or V row.
 //                   Writes base-2 logits (fp32) for the scoring pass and the
 //                   chunk's (max, sum, unnormalised output).
 //   decode_merge    merges the chunks: o (bf16), lse (natural log).
@@ -63,6 +66,14 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2_f16x2(uint32_t two_bytes) {
   return uint32_t(h.x) | (uint32_t(h.y) << 16);
 }
 
+// both e4m3 pairs of a 32-bit word -> two f16x2 (low pair, high pair)
+__device__ __forceinline__ void cvt_e4m3x4_f16x2x2(uint32_t x, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 l16, h16;\n\tmov.b32 {l16, h16}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, l16;\n\tcvt.rn.f16x2.e4m3x2 %1, h16;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(x));
+}
+
 __device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                         uint32_t a3, uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -80,10 +91,14 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
 // ---------------------------------------------------------------------------
 // decode_partial: grid (chunks, Hkv, B), DP_WARPS warps
 // ---------------------------------------------------------------------------
+constexpr int DSTAGE_KEYS = 64;                   // keys per TMA stage
+constexpr int DSTAGES = 3;                        // ring depth
+constexpr int DSTAGE_BYTES = 2 * DSTAGE_KEYS * 128;  // K and V codes
+
 template <int G>
-__global__ void __launch_bounds__(DP_WARPS * 32)
-    decode_partial(const __nv_bfloat16* __restrict__ q, const uint8_t* __restrict__ Kc,
-                   const uint8_t* __restrict__ Vc, const float* __restrict__ ks,
+__global__ void __launch_bounds__((DP_WARPS + 1) * 32, 3)
+    decode_partial(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                   const __nv_bfloat16* __restrict__ q, const float* __restrict__ ks,
                    const float* __restrict__ vs, SeqLens seq_len, int64_t cap,
                    int Hkv, int nch, float scale_log2, float* __restrict__ logits,
                    Partial* __restrict__ part, float* __restrict__ part_o) {
@@ -91,16 +106,47 @@ __global__ void __launch_bounds__(DP_WARPS * 32)
   constexpr int GH = G < 8 ? G : 8;       // real heads per n-tile
   __shared__ uint16_t sP[DP_WARPS][NT][8 * 16];      // P' [head][key] f16 per warp
   __shared__ float sM[DP_WARPS][NT * 8], sL[DP_WARPS][NT * 8];
-  __shared__ float sO[DP_WARPS][NT * 8][128];
+  __shared__ uint64_t full[DSTAGES], empty[DSTAGES];
+  extern __shared__ uint8_t dsmem_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) &
+                                             ~uintptr_t(1023));
 
   const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = warp_id(), lane = lane_id();
   const int gid = lane >> 2, t = lane & 3;
   const int N = seq_len.n[b];
   const int Hq = Hkv * G;
-  const int64_t key_lo = int64_t(c) * CH + warp * (CH / DP_WARPS);
-  const int64_t key_hi = min(int64_t(c) * CH + (warp + 1) * (CH / DP_WARPS), int64_t(N));
+  const int64_t c_lo = int64_t(c) * CH;
+  const int64_t c_hi = min(c_lo + CH, int64_t(N));
+  const int n_st = c_hi > c_lo ? int((c_hi - c_lo + DSTAGE_KEYS - 1) / DSTAGE_KEYS) : 0;
   const size_t rowbase = size_t(b) * cap;  // first cache row of sequence b
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < DSTAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], DP_WARPS);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  if (warp == DP_WARPS) {
+    // ---------------- producer: K and V tiles of 64 rows -> smem ring -------
+    if (lane == 0) {
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      for (int si = 0; si < n_st; ++si) {
+        const int slot = si % DSTAGES;
+        if (si >= DSTAGES && !mbar_wait(&empty[slot], ((si / DSTAGES) & 1) ^ 1)) break;
+        uint8_t* st = ring + slot * DSTAGE_BYTES;
+        const int z = int(rowbase + c_lo) + si * DSTAGE_KEYS;
+        mbar_arrive_expect_tx(&full[slot], DSTAGE_BYTES);
+        tma_load_3d(st, &tmK, &full[slot], 0, g, z);
+        tma_load_3d(st + DSTAGE_KEYS * 128, &tmV, &full[slot], 0, g, z);
+      }
+    }
+    return;
+  }
 
   // query fragments (B operand of S^T = K q^T): dims permuted so that lane t
   // uses dims 32t .. 32t+31: MMA step s, k-slot {2t,2t+1,2t+8,2t+9} ->
@@ -133,31 +179,47 @@ __global__ void __launch_bounds__(DP_WARPS * 32)
     for (int i = 0; i < 8; ++i) o[nt][i][0] = o[nt][i][1] = o[nt][i][2] = o[nt][i][3] = 0.f;
   }
   float* lg = logits + (size_t(b) * Hkv + g) * cap * G;
+  bool ok = true;
 
-  for (int64_t key0 = key_lo; key0 < key_hi; key0 += 16) {
-    // ---- S^T = K q^T : rows key0+gid and key0+gid+8, lane bytes 32t..32t+31
-    const int64_t r0 = key0 + gid, r1 = key0 + gid + 8;
-    const bool v0 = r0 < key_hi, v1 = r1 < key_hi;
-    const uint8_t* k0 = Kc + ((rowbase + (v0 ? r0 : key_lo)) * Hkv + g) * 128 + 32 * t;
-    const uint8_t* k1 = Kc + ((rowbase + (v1 ? r1 : key_lo)) * Hkv + g) * 128 + 32 * t;
-    const uint4 ka = __ldg(reinterpret_cast<const uint4*>(k0));
-    const uint4 kb = __ldg(reinterpret_cast<const uint4*>(k0 + 16));
-    const uint4 kc = __ldg(reinterpret_cast<const uint4*>(k1));
-    const uint4 kd = __ldg(reinterpret_cast<const uint4*>(k1 + 16));
-    // ---- V rows key0 + 4t + u, bytes 16*gid .. 16*gid+15
-    uint4 vr[4];
-    float vsc[4];
+  // scales of this warp's keys in stage si (loaded one stage ahead)
+  auto load_scales = [&](int si, float (&vsc)[4], float& ks0, float& ks1) {
+    const int64_t key0 = c_lo + si * DSTAGE_KEYS + 16 * warp;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int64_t rv = key0 + 4 * t + u;
-      const bool ok = rv < key_hi;
-      vr[u] = __ldg(reinterpret_cast<const uint4*>(
-          Vc + ((rowbase + (ok ? rv : key_lo)) * Hkv + g) * 128 + 16 * gid));
-      vsc[u] = ok ? __ldg(vs + (rowbase + rv) * Hkv + g) * kPScale : 0.f;
+      const int64_t kv = key0 + 4 * t + u;
+      vsc[u] = kv < c_hi ? __ldg(vs + (rowbase + kv) * Hkv + g) * kPScale : 0.f;
     }
-    const float ks0 = v0 ? __ldg(ks + (rowbase + r0) * Hkv + g) : 0.f;
-    const float ks1 = v1 ? __ldg(ks + (rowbase + r1) * Hkv + g) : 0.f;
+    ks0 = key0 + gid < c_hi ? __ldg(ks + (rowbase + key0 + gid) * Hkv + g) : 0.f;
+    ks1 = key0 + gid + 8 < c_hi ? __ldg(ks + (rowbase + key0 + gid + 8) * Hkv + g) : 0.f;
+  };
+  float nvsc[4], nks0 = 0.f, nks1 = 0.f;
+  if (n_st > 0) load_scales(0, nvsc, nks0, nks1);
 
+  for (int si = 0; si < n_st; ++si) {
+    const int slot = si % DSTAGES;
+    float vsc[4] = {nvsc[0], nvsc[1], nvsc[2], nvsc[3]};
+    const float ks0 = nks0, ks1 = nks1;
+    if (si + 1 < n_st) load_scales(si + 1, nvsc, nks0, nks1);
+    ok = ok && mbar_wait(&full[slot], (si / DSTAGES) & 1);
+    const uint8_t* sK = ring + slot * DSTAGE_BYTES;
+    const uint8_t* sV = sK + DSTAGE_KEYS * 128;
+    // this warp's 16 keys of the stage; rows in the swizzled tile: unit u of
+    // row r sits at r*128 + ((u ^ (r & 7)) << 4)
+    const int rA = 16 * warp + gid, rB = rA + 8;
+    const int64_t key0 = c_lo + si * DSTAGE_KEYS + 16 * warp;
+    const int64_t r0 = key0 + gid, r1 = key0 + gid + 8;
+    const bool v0 = r0 < c_hi, v1 = r1 < c_hi;
+    const uint4 ka = *reinterpret_cast<const uint4*>(sK + rA * 128 + (((2 * t) ^ (rA & 7)) << 4));
+    const uint4 kb = *reinterpret_cast<const uint4*>(sK + rA * 128 + (((2 * t + 1) ^ (rA & 7)) << 4));
+    const uint4 kc = *reinterpret_cast<const uint4*>(sK + rB * 128 + (((2 * t) ^ (rB & 7)) << 4));
+    const uint4 kd = *reinterpret_cast<const uint4*>(sK + rB * 128 + (((2 * t + 1) ^ (rB & 7)) << 4));
+    // ---- V rows key0 + 4t + u, bytes 16*gid .. 16*gid+15
+    uint4 vr[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int rv = 16 * warp + 4 * t + u;
+      vr[u] = *reinterpret_cast<const uint4*>(sV + rv * 128 + ((gid ^ (rv & 7)) << 4));
+    }
     const uint32_t kw0[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
     const uint32_t kw1[8] = {kc.x, kc.y, kc.z, kc.w, kd.x, kd.y, kd.z, kd.w};
     float sacc[NT][4];
@@ -165,10 +227,10 @@ __global__ void __launch_bounds__(DP_WARPS * 32)
     for (int nt = 0; nt < NT; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
 #pragma unroll
     for (int s = 0; s < 8; ++s) {
-      const uint32_t a0 = cvt_e4m3x2_f16x2(kw0[s]);        // row gid,   slots 2t,2t+1
-      const uint32_t a1 = cvt_e4m3x2_f16x2(kw1[s]);        // row gid+8, slots 2t,2t+1
-      const uint32_t a2 = cvt_e4m3x2_f16x2(kw0[s] >> 16);  // row gid,   slots 2t+8,2t+9
-      const uint32_t a3 = cvt_e4m3x2_f16x2(kw1[s] >> 16);  // row gid+8, slots 2t+8,2t+9
+      // row gid: slots 2t,2t+1 (a0) and 2t+8,2t+9 (a2); row gid+8: a1, a3
+      uint32_t a0, a1, a2, a3;
+      cvt_e4m3x4_f16x2x2(kw0[s], a0, a2);
+      cvt_e4m3x4_f16x2x2(kw1[s], a1, a3);
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) mma_f16(sacc[nt], a0, a1, a2, a3, qf[nt][s][0], qf[nt][s][1]);
     }
@@ -243,21 +305,25 @@ __global__ void __launch_bounds__(DP_WARPS * 32)
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         // bytes 2i / 2i+1 of a row slice = dims 16*gid + 2i (MMA row gid) and
-        // 16*gid + 2i + 1 (row gid+8); pair the two keys' bytes with a permute
-        const int wd = i >> 1, sh = (i & 1) * 16;
-        const uint32_t r0 = vw[0][wd] >> sh, r1 = vw[1][wd] >> sh;
-        const uint32_t r2 = vw[2][wd] >> sh, r3 = vw[3][wd] >> sh;
-        const uint32_t a0 = cvt_e4m3x2_f16x2(__byte_perm(r0, r1, 0x0040));
-        const uint32_t a1 = cvt_e4m3x2_f16x2(__byte_perm(r0, r1, 0x0051));
-        const uint32_t a2 = cvt_e4m3x2_f16x2(__byte_perm(r2, r3, 0x0040));
-        const uint32_t a3 = cvt_e4m3x2_f16x2(__byte_perm(r2, r3, 0x0051));
+        // 16*gid + 2i + 1 (row gid+8).  One permute gathers, for two keys,
+        // [key0 dim 2i, key1 dim 2i, key0 dim 2i+1, key1 dim 2i+1].
+        const int wd = i >> 1, p = (i & 1) * 2;
+        const uint32_t sel = uint32_t(p) | uint32_t(p + 4) << 4 | uint32_t(p + 1) << 8 |
+                             uint32_t(p + 5) << 12;
+        uint32_t a0, a1, a2, a3;
+        cvt_e4m3x4_f16x2x2(__byte_perm(vw[0][wd], vw[1][wd], sel), a0, a1);
+        cvt_e4m3x4_f16x2x2(__byte_perm(vw[2][wd], vw[3][wd], sel), a2, a3);
         mma_f16(o[nt][i], a0, a1, a2, a3, b0, b1);
       }
     }
     __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[slot]);
   }
 
-  // ---- combine the warps of the CTA, then one partial per (b, h, chunk)
+  // ---- combine the warps of the CTA, then one partial per (b, h, chunk);
+  // the drained ring holds the warps' outputs
+  asm volatile("bar.sync 1, %0;" ::"n"(DP_WARPS * 32) : "memory");
+  float (*sO)[NT * 8][128] = reinterpret_cast<float (*)[NT * 8][128]>(ring);
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
@@ -281,7 +347,7 @@ __global__ void __launch_bounds__(DP_WARPS * 32)
       sO[warp][nt * 8 + 2 * t + 1][16 * gid + 2 * i + 1] = o[nt][i][3];
     }
   }
-  __syncthreads();
+  asm volatile("bar.sync 1, %0;" ::"n"(DP_WARPS * 32) : "memory");
   for (int hh = warp; hh < G; hh += DP_WARPS) {
     float M = -INFINITY;
     for (int w2 = 0; w2 < DP_WARPS; ++w2) M = fmaxf(M, sM[w2][hh]);
@@ -585,8 +651,17 @@ cudaError_t launch_dec_g(const DecodeArgs& a, const SeqLens& d_seq, int max_len,
   e = cudaMemsetAsync(ccount, 0, size_t(B) * Hkv * 4, st);
   if (e != cudaSuccess) return e;
   const float sl2 = a.scale * kLog2e;
-  decode_partial<G><<<dim3(nch_used, Hkv, B), DP_WARPS * 32, 0, st>>>(
-      reinterpret_cast<const __nv_bfloat16*>(a.q), a.Kc, a.Vc, a.ks, a.vs, d_seq, a.cap, Hkv, nch,
+  // K, V codes viewed as [B*cap tokens][Hkv][64 two-byte units]: 64-row boxes
+  CUtensorMap tmK, tmV;
+  const uint64_t rows = uint64_t(B) * a.cap;
+  if (!make_tmap_3d(&tmK, a.Kc, 64, Hkv, rows, 128, uint64_t(Hkv) * 128, 64, 1, DSTAGE_KEYS) ||
+      !make_tmap_3d(&tmV, a.Vc, 64, Hkv, rows, 128, uint64_t(Hkv) * 128, 64, 1, DSTAGE_KEYS))
+    return cudaErrorInvalidValue;
+  const int psmem = DSTAGES * DSTAGE_BYTES + 1024;
+  e = ensure_smem_attr(reinterpret_cast<const void*>(decode_partial<G>), psmem);
+  if (e != cudaSuccess) return e;
+  decode_partial<G><<<dim3(nch_used, Hkv, B), (DP_WARPS + 1) * 32, psmem, st>>>(
+      tmK, tmV, reinterpret_cast<const __nv_bfloat16*>(a.q), a.ks, a.vs, d_seq, a.cap, Hkv, nch,
       sl2, logits, part, part_o);
   decode_merge<<<dim3(Hq, B), 128, 0, st>>>(part, part_o, d_seq, Hq, nch,
                                             reinterpret_cast<__nv_bfloat16*>(a.o), a.lse, lse2);
@@ -643,7 +718,7 @@ size_t decode_workspace_bytes(int B, int64_t cap, int Hq, int Hkv, int k, int w)
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
-  if (a.B > MAX_B || a.k > CAPC / 2 || a.cap > INT32_MAX) return cudaErrorNotSupported;
+  if (a.B > MAX_B || a.k > CAPC / 2 || int64_t(a.B) * a.cap > INT32_MAX) return cudaErrorNotSupported;
   SeqLens d_seq{};
   int max_len = 0;
   for (int b = 0; b < a.B; ++b) {

@@ -15,7 +15,9 @@
 //   warps 2-5  softmax, one thread per row (TMEM lane): base-2 online softmax
 //              with a lazily raised reference max (O is rescaled only when the
 //              row max grows by more than 2^8), P_j as bf16 into shared memory
-//              (A operand of the PV MMA), epilogue O / l and lse.
+//              (A operand of the PV MMA), epilogue O / l and lse.  A quarter of
+//              the exponentials run as a polynomial on the FMA pipe so the
+//              MUFU unit is not the softmax's bound.
 // TMEM: S0 cols [0,128), S1 [128,256), O [256,384).
 #include "common.cuh"
 #include "kernels.h"
@@ -50,6 +52,27 @@ struct Bars {
   uint64_t o_done;
   uint32_t tmem_slot;
 };
+
+// 2^x on the FMA pipe, for relieving the MUFU unit: x = n + f with n the
+// nearest integer (added to x as 1.5 * 2^23, whose ulp is 1) and f in
+// [-1/2, 1/2]; 2^f from a degree-5 polynomial whose coefficients were fitted
+// here for minimum relative error on [-1/2, 1/2] (max 2.3e-7 in fp32 Horner
+// form, about the error of ex2.approx); 2^n is added to the exponent field.
+// Inputs below -126 give 0 (2^-126 is below every value that matters here).
+__device__ __forceinline__ float poly_exp2(float x) {
+  const float xc = fmaxf(x, -126.f);
+  const float t = xc + 12582912.f;
+  const float n = t - 12582912.f;
+  const float f = xc - n;
+  float p = 1.3276374666020274e-3f;
+  p = fmaf(p, f, 9.67551488429308e-3f);
+  p = fmaf(p, f, 5.550713464617729e-2f);
+  p = fmaf(p, f, 2.4022120237350464e-1f);
+  p = fmaf(p, f, 6.931469440460205e-1f);
+  p = fmaf(p, f, 1.0000001192092896f);
+  const float r = __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+  return x < -126.f ? 0.f : r;
+}
 
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int ks) {
   // K-major operand [128 rows][128 K] as two 64-column swizzled halves
@@ -201,8 +224,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t pk[64];
 #pragma unroll
       for (int e = 0; e < 128; e += 2) {
+        // one element in four on the FMA pipe, the rest on MUFU
         const float p0 = fast_exp2(fmaf(x[e], scale_log2, -m_use));
-        const float p1 = fast_exp2(fmaf(x[e + 1], scale_log2, -m_use));
+        const float p1 = (e & 2) ? poly_exp2(fmaf(x[e + 1], scale_log2, -m_use))
+                                 : fast_exp2(fmaf(x[e + 1], scale_log2, -m_use));
         sum += p0 + p1;
         pk[e >> 1] = pack_bf16x2(p0, p1);
       }
@@ -288,7 +313,19 @@ cudaError_t launch_g(const AttnArgs& a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+__global__ void poly_exp2_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
+  const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < n) y[i] = poly_exp2(x[i]);
+}
+
 }  // namespace
+
+cudaError_t launch_poly_exp2(const float* x, float* y, int64_t n, cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  poly_exp2_kernel<<<unsigned((n + 255) / 256), 256, 0, stream>>>(x, y, n);
+  count_launch();
+  return cudaGetLastError();
+}
 
 cudaError_t launch_full_attn(const AttnArgs& a, cudaStream_t stream) {
   switch (a.Hq / a.Hkv) {

@@ -344,6 +344,51 @@ def decode_cache_np(cfg: BlockConfig, N: int, batch: int | None = None) -> Decod
     return DecodeCache(Kc, Vc, S, needles)
 
 
+def q_rows_torch(cfg: BlockConfig, tid: int, T: int | None = None, device="cuda", rows: int = 4096):
+    """q_rows_np's recipe for all rows [T, Hq, d] on the device (bf16 tensor)."""
+    import torch
+    T = cfg.T if T is None else T
+    Hq, d = cfg.n_q_heads, cfg.head_dim
+    out = torch.empty(T, Hq, d, dtype=torch.bfloat16, device=device)
+    ug = torch.from_numpy(needle_dirs(cfg)).to(device).repeat_interleave(cfg.G, 0)[None]
+    for r0 in range(0, T, rows):
+        n = min(rows, T - r0)
+        z = normals_torch(cfg.seed, tid, r0 * Hq * d, n * Hq * d, device).view(n, Hq, d)
+        if cfg.q_mix:
+            z = 0.5 * z + 0.5 * math.sqrt(d) * ug
+        out[r0:r0 + n] = z.float().bfloat16()
+    return out
+
+
+def kv_torch(cfg: BlockConfig, tid: int, T: int | None = None, device="cuda"):
+    """kv_np's recipe on the device: [T, Hkv, d] bf16 tensor."""
+    T = cfg.T if T is None else T
+    return normal_bf16_torch(cfg.seed, tid, 0, T * cfg.n_kv_heads * cfg.head_dim,
+                             device=device).view(T, cfg.n_kv_heads, cfg.head_dim)
+
+
+def bridge_inputs_torch(cfg: BlockConfig, T: int | None = None, device="cuda"):
+    """bridge_inputs_np's recipe on the device: H, W_k, W_v bf16 tensors."""
+    T = cfg.T if T is None else T
+    dm, N = cfg.d_model, cfg.n_kv_heads * cfg.head_dim
+    H = normal_bf16_torch(cfg.seed, TID_H, 0, T * dm, device=device).view(T, dm)
+    sd = 1.0 / math.sqrt(dm)
+    Wk = normal_bf16_torch(cfg.seed, TID_WK, 0, dm * N, sd, device=device).view(dm, N)
+    Wv = normal_bf16_torch(cfg.seed, TID_WV, 0, dm * N, sd, device=device).view(dm, N)
+    return H, Wk, Wv
+
+
+def needle_scatter_torch(cfg: BlockConfig, T: int | None = None, device="cuda"):
+    """(rows, heads, values) of the planted needle keys for K[rows, heads] = values."""
+    import torch
+    pos = prefill_needles(cfg, T)
+    nk = torch.from_numpy(needle_key_bits(cfg).view(np.int16)).to(device).view(torch.bfloat16)
+    rows = torch.cat([torch.from_numpy(p) for p in pos]).to(device)
+    heads = torch.cat([torch.full((len(p),), g, dtype=torch.int64)
+                       for g, p in enumerate(pos)]).to(device)
+    return rows, heads, nk[heads]
+
+
 def decode_cache_torch(cfg: BlockConfig, N: int, batch: int | None = None, device="cuda"):
     """decode_cache_np's recipe on the device (torch); the e4m3 rounding is
     torch's float8_e4m3fn cast of values clamped to [-448, 448], pinned to the

@@ -67,3 +67,48 @@ def check_index_lists(gpu_idx, orc_idx, kth, rows, k, w, score_fn):
             assert not bad.any(), (f"row {i} head {g}: positions {sym[bad][:8]} differ with "
                                    f"scores {s[bad][:8]} vs k-th {tau}")
     return n_diff
+
+
+def compare_rows(orc, cfg, kv, Qr, Qsr, rows, got, k=None, w=None):
+    """Compare the GPU block's outputs on `rows` with the oracle.
+
+    Qr [n, Hq, d] and Qsr (list of [n, Hq, d]) are the rows' query bits;
+    got holds the GPU tensors (O, lse, idx, O_sparse) for all rows.  Sparse
+    outputs are compared with the oracle on its own lists where the GPU list is
+    identical, and on the GPU's list (validated by check_index_lists) where it
+    differs.  Returns the number of (row, KV head) lists that differ."""
+    import torch
+    k = cfg.k_global if k is None else k
+    w = cfg.window if w is None else w
+    sc = cfg.scale
+    ridx = torch.from_numpy(np.asarray(rows)).to(got["O"].device)
+    ref = orc.block_rows(kv, Qr, Qsr, rows, sc, k, w)
+    assert_close_bf16(host_f64(got["O"][ridx]), ref["O"], "O_full")
+    assert np.max(np.abs(got["lse"][ridx].cpu().numpy() - ref["lse"])) <= LSE_ABS
+    gi = got["idx"][ridx].cpu().numpy()
+    n_diff = check_index_lists(gi, ref["idx"], ref["kth"], rows, k, w,
+                               lambda r, g, js: orc.scores(kv, Qr[r], g, sc, ref["lse"][r], js))
+    same = np.all(gi == ref["idx"], axis=(1, 2))
+    for l, q in enumerate(Qsr):
+        gs = host_f64(got["O_sparse"][l][ridx])
+        if same.any():
+            assert_close_bf16(gs[same], ref["O_sparse"][l][same], f"O_sparse[{l}]")
+        if (~same).any():
+            o_gpu_list, _ = orc.sparse_attn(kv, q[~same], gi[~same], sc)
+            assert_close_bf16(gs[~same], o_gpu_list, f"O_sparse[{l}] on GPU lists")
+    return n_diff
+
+
+def edge_rows(T, k=1024, w=128, n_random=0, seed=0):
+    base = [0, 1, w - 1, w, w + 1, k + w - 2, k + w - 1, k + w, k + w + 1, T // 2, T - 2, T - 1]
+    rows = set(r for r in base if 0 <= r < T)
+    if n_random:
+        rng = np.random.default_rng(seed)
+        rows |= set(rng.integers(0, T, n_random).tolist())
+    return np.array(sorted(rows), np.int64)
+
+
+def bits(t):
+    """bf16 tensor -> uint16 numpy bits (host)."""
+    import torch
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)

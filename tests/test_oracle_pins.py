@@ -297,3 +297,21 @@ def test_synth_decode_cache_torch_matches_numpy():
     for got, want in ((Kc.numpy(), a.Kc), (Vc.numpy(), a.Vc)):
         nz = (want & 0x7F) != 0
         assert np.array_equal(got[nz], want[nz]) and np.all((got[~nz] & 0x7F) == 0)
+
+
+def test_synth_device_recipes_match_numpy():
+    cfg = synth.BlockConfig("t", 3, 600, 8, 2, d_model=128, n_needles=8, q_mix=True)
+    q = synth.q_rows_torch(cfg, synth.TID_Q, device="cpu", rows=128)
+    assert np.array_equal(q.view(torch.int16).numpy().view(np.uint16),
+                          synth.q_rows_np(cfg, synth.TID_Q, np.arange(600)))
+    H, Wk, Wv = synth.bridge_inputs_torch(cfg, device="cpu")
+    h2, wk2, wv2 = synth.bridge_inputs_np(cfg)
+    for a, b in ((H, h2), (Wk, wk2), (Wv, wv2)):
+        assert np.array_equal(a.view(torch.int16).numpy().view(np.uint16), b)
+    K = synth.kv_torch(cfg, synth.TID_K, device="cpu")
+    assert np.array_equal(K.view(torch.int16).numpy().view(np.uint16), synth.kv_np(cfg, synth.TID_K))
+    rows, heads, vals = synth.needle_scatter_torch(cfg, device="cpu")
+    Kn = synth.kv_np(cfg, synth.TID_K)
+    synth.plant_needles_np(cfg, Kn, synth.prefill_needles(cfg))
+    K[rows, heads] = vals
+    assert np.array_equal(K.view(torch.int16).numpy().view(np.uint16), Kn)
