@@ -56,27 +56,6 @@ struct Bars {
   uint32_t tmem_slot;
 };
 
-// 2^x on the FMA pipe, for relieving the MUFU unit: x = n + f with n the
-// nearest integer (added to x as 1.5 * 2^23, whose ulp is 1) and f in
-// [-1/2, 1/2]; 2^f from a degree-5 polynomial whose coefficients were fitted
-// here for minimum relative error on [-1/2, 1/2] (max 2.3e-7 in fp32 Horner
-// form, about the error of ex2.approx); 2^n is added to the exponent field.
-// Inputs below -126 give 0 (2^-126 is below every value that matters here).
-__device__ __forceinline__ float poly_exp2(float x) {
-  const float xc = fmaxf(x, -126.f);
-  const float t = xc + 12582912.f;
-  const float n = t - 12582912.f;
-  const float f = xc - n;
-  float p = 1.3276374666020274e-3f;
-  p = fmaf(p, f, 9.67551488429308e-3f);
-  p = fmaf(p, f, 5.550713464617729e-2f);
-  p = fmaf(p, f, 2.4022120237350464e-1f);
-  p = fmaf(p, f, 6.931469440460205e-1f);
-  p = fmaf(p, f, 1.0000001192092896f);
-  const float r = __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-  return x < -126.f ? 0.f : r;
-}
-
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int ks) {
   // K-major operand [128 rows][128 K] as two 64-column swizzled halves
   return sdesc_sw128(tile + (ks >> 2) * CHUNK + (ks & 3) * 32, 16, 1024);
@@ -240,27 +219,38 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int e = 0; e < 128; ++e)
           if (e > lim) x[e] = -INFINITY;
       }
-      float mx = x[0];
+      float mq[4] = {x[0], x[1], x[2], x[3]};
 #pragma unroll
-      for (int e = 1; e < 128; ++e) mx = fmaxf(mx, x[e]);
-      const float m_new = mx * scale_log2;
+      for (int e = 4; e < 128; e += 8)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) mq[u] = fmax3(mq[u], x[e + u], x[e + 4 + u]);
+      const float m_new = fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3])) * scale_log2;
       float alpha = 1.f;
       const bool raise = m_new > m_use + kRescaleThreshold;
       if (raise) {
         alpha = fast_exp2(m_use - m_new);  // 0 on the first tile
         m_use = m_new;
       }
-      float sum = 0.f;
+      const uint64_t sc2 = f2(scale_log2, scale_log2), nm2 = f2(-m_use, -m_use);
+      uint64_t sum2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
       uint32_t pk[64];
 #pragma unroll
       for (int e = 0; e < 128; e += 2) {
-        // one element in four on the FMA pipe, the rest on MUFU
-        const float p0 = fast_exp2(fmaf(x[e], scale_log2, -m_use));
-        const float p1 = (e & 2) ? poly_exp2(fmaf(x[e + 1], scale_log2, -m_use))
-                                 : fast_exp2(fmaf(x[e + 1], scale_log2, -m_use));
-        sum += p0 + p1;
+        float a, b, p0, p1;
+        f2_split(f2_fma(f2(x[e], x[e + 1]), sc2, nm2), a, b);
+        if ((e & 6) == 6) {  // one pair in four on the FMA pipe, the rest on MUFU
+          poly_exp2x2(a, b, p0, p1);
+        } else {
+          p0 = fast_exp2(a);
+          p1 = fast_exp2(b);
+        }
+        sum2[(e >> 1) & 1] = f2_add(sum2[(e >> 1) & 1], f2(p0, p1));
         pk[e >> 1] = pack_bf16x2(p0, p1);
       }
+      float s0, s1, s2, s3;
+      f2_split(sum2[0], s0, s1);
+      f2_split(sum2[1], s2, s3);
+      const float sum = (s0 + s1) + (s2 + s3);
       l = l * alpha + sum;
       if (j > 0 && __any_sync(0xffffffffu, raise)) {
 #pragma unroll 1
@@ -323,7 +313,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 __global__ void poly_exp2_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
   const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i < n) y[i] = poly_exp2(x[i]);
+  if (2 * i + 1 < n) {
+    poly_exp2x2(x[2 * i], x[2 * i + 1], y[2 * i], y[2 * i + 1]);
+  } else if (2 * i < n) {
+    float unused;
+    poly_exp2x2(x[2 * i], 0.f, y[2 * i], unused);
+  }
 }
 
 template <int G>
@@ -353,7 +348,7 @@ cudaError_t launch_g(const AttnArgs& a, cudaStream_t stream) {
 
 cudaError_t launch_poly_exp2(const float* x, float* y, int64_t n, cudaStream_t stream) {
   if (n <= 0) return cudaSuccess;
-  poly_exp2_kernel<<<unsigned((n + 255) / 256), 256, 0, stream>>>(x, y, n);
+  poly_exp2_kernel<<<unsigned((n + 511) / 512), 256, 0, stream>>>(x, y, n);
   count_launch();
   return cudaGetLastError();
 }

@@ -11,15 +11,15 @@
 //   warp 0     TMA: the item's Q tile once, K tiles into a ring
 //   warp 1     TMEM owner; one lane issues S^T = K Q^T (M = 128 keys,
 //              N = 128 (query, head) rows) into one of four TMEM buffers
-//   warps 2-9  scorers, two per TMEM lane quarter: thread = key (TMEM lane);
-//              warps 2-5 take the first half of the item's queries (columns
-//              0-63), warps 6-9 the second half; a thread sums
-//              exp2(s*scale*log2e - lse2) over each query's G heads in
-//              registers, so a query's score needs no shuffles.
+//   warps 2-17 scorers, four per TMEM lane quarter: thread = key (TMEM lane);
+//              scorer warp 4s + r takes the s-th quarter of the item's queries
+//              (TMEM columns 32s .. 32s + 31) for keys 32r .. 32r + 31; a
+//              thread sums exp2(s*scale*log2e - lse2) over each query's G
+//              heads in registers, so a query's score needs no shuffles.
 // Streaming exact top-k without CTA barriers in the tile loop:
 //   * every scorer warp appends the candidates of its 32 keys to its own
 //     per-query sub-buffer (ballot order = ascending position); the four
-//     warps of a query's half hold disjoint key sets;
+//     warps of a query's quarter hold disjoint key sets;
 //   * every append is also counted in a per-query histogram of score bins
 //     (eighths of a binade below the largest possible score G) in shared
 //     memory; whatever snapshot of it a warp reads, the highest bin with at
@@ -67,9 +67,6 @@ struct SelCfg {
   static constexpr int QH = QT / SETS;                // queries per scorer set (32 columns)
   static constexpr int NB = QT <= 32 ? 256 : 64;      // histogram bins per query
   static constexpr int BSHIFT = QT <= 32 ? 20 : 22;   // bin width: 2^-3 or 2^-1 binade
-  static constexpr int QG = QH;                       // queries scored per group
-  static constexpr int NG = 1;                        // groups per tile
-  static constexpr int CPG = 1;                       // 32-column chunks per group
 };
 
 struct Bars {
@@ -84,7 +81,7 @@ struct Misc {
   static constexpr int QT = SelCfg<G>::QT, NB = SelCfg<G>::NB;
   Bars bars;
   float lse2[128];            // base-2 lse of the item's 128 (query, head) rows
-  uint32_t floor_bin[QT];     // candidates need bin >= floor_bin
+  uint32_t floor_bits[QT];    // candidates need score bits >= floor_bits (a bin's lower edge)
   uint32_t cnt[4][QT];        // entries in each sub-buffer
   uint32_t hist[QT][NB];      // appended entries per score bin
   uint32_t dig[SCORER_WARPS][256];  // per-warp radix histograms of the final select
@@ -290,7 +287,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                   int T, int Hkv, int k, int w, int capw, int kst, float scale_log2) {
   using Cfg = SelCfg<G>;
   constexpr int QT = Cfg::QT, QH = Cfg::QH, NB = Cfg::NB, BSHIFT = Cfg::BSHIFT;
-  constexpr int QG = Cfg::QG, NG = Cfg::NG, CPG = Cfg::CPG;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -413,66 +409,59 @@ __global__ void __launch_bounds__(THREADS, 1)
         ms->lse2[tid] = qrow < T ? lse[size_t(qrow) * Hq + g * G + tid % G] * kLog2e : INFINITY;
       }
       for (int i = tid; i < QT; i += SCORERS) {
-        ms->floor_bin[i] = 0;
-        ms->cnt[0][i] = ms->cnt[1][i] = ms->cnt[2][i] = ms->cnt[3][i] = 0;
+        ms->floor_bits[i] = 0;
       }
       for (int i = tid; i < QT * NB; i += SCORERS) (&ms->hist[0][0])[i] = 0;
+      const int qb0 = half * QH;        // this warp's queries: qb0 .. qb0 + QH - 1
+      const int qvalid = T - q0 - qb0;  // of which those below qvalid exist
+      uint32_t n[QH];                   // entries in this warp's sub-buffers
+#pragma unroll
+      for (int ql = 0; ql < QH; ++ql) n[ql] = 0;
       scorer_sync();
       for (int t = 0; t < n_tiles; ++t, ++st) {
         const int b = st % NSB;
         ok = ok && mbar_wait(&br->s_full[b], (st / NSB) & 1);
         tc_fence_after();
         const int j = t * TILE + sub * 32 + lane;  // this thread's key
-        const bool all_cand = (t + 1) * TILE - 1 + w <= q0;
-#pragma unroll 1
-        for (int gi = 0; gi < NG; ++gi) {
-          const int qb0 = half * QH + gi * QG;  // first query of the group
-          float sc[QG];
+        // candidate test for query qb0 + ql: j + w <= its position, i.e.
+        // dpos <= ql, and the query inside the sequence (ql < qvalid)
+        const int dpos = j + w - q0 - qb0;
+        float sc[QH];
+        {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_addr + b * 128 + half * 32, r);
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(&br->s_empty[b]);
 #pragma unroll
-          for (int cc = 0; cc < CPG; ++cc) {
-            const int c = qb0 * G / 32 + cc;  // chunk: columns 32c .. 32c+31
-            uint32_t r[32];
-            tmem_ld32(tmem + lane_addr + b * 128 + c * 32, r);
-            tmem_wait_ld();
-            if (gi == NG - 1 && cc == CPG - 1) {
-              tc_fence_before();
-              mbar_arrive(&br->s_empty[b]);
-            }
+          for (int qq = 0; qq < QH; ++qq) {
+            float acc = 0.f;
 #pragma unroll
-            for (int qq = 0; qq < 32 / G; ++qq) {
-              float acc = 0.f;
-#pragma unroll
-              for (int h = 0; h < G; ++h)
-                acc += fast_exp2(fmaf(__uint_as_float(r[qq * G + h]), scale_log2,
-                                      -ms->lse2[c * 32 + qq * G + h]));
-              sc[cc * (32 / G) + qq] = acc;
-            }
+            for (int h = 0; h < G; ++h)
+              acc += fast_exp2(fmaf(__uint_as_float(r[qq * G + h]), scale_log2,
+                                    -ms->lse2[half * 32 + qq * G + h]));
+            sc[qq] = acc;
           }
-          uint32_t bal[QG], binv[QG], anymask = 0;
+        }
+        uint32_t bal[QH], anymask = 0;
 #pragma unroll
-          for (int ql = 0; ql < QG; ++ql) {
-            const int q = qb0 + ql;
-            const int qpos = q0 + q;
-            binv[ql] = bin_of<NB, BSHIFT>(__float_as_uint(sc[ql]), lo);
-            const bool pass =
-                (all_cand || j + w <= qpos) && qpos < T && binv[ql] >= ms->floor_bin[q];
-            bal[ql] = __ballot_sync(0xffffffffu, pass);
-            anymask |= uint32_t(bal[ql] != 0) << ql;
-          }
-          if (anymask == 0) continue;
-          uint32_t n[QG];
+        for (int ql = 0; ql < QH; ++ql) {
+          const bool pass = dpos <= ql && ql < qvalid &&
+                            __float_as_uint(sc[ql]) >= ms->floor_bits[qb0 + ql];
+          bal[ql] = __ballot_sync(0xffffffffu, pass);
+          anymask |= uint32_t(bal[ql] != 0) << ql;
+        }
+        if (anymask != 0) {
 #pragma unroll
-          for (int ql = 0; ql < QG; ++ql) n[ql] = ms->cnt[sub][qb0 + ql];
-#pragma unroll
-          for (int ql = 0; ql < QG; ++ql) {
+          for (int ql = 0; ql < QH; ++ql) {
             if (!((anymask >> ql) & 1u) || n[ql] + 32 <= uint32_t(capw)) continue;
             // make room: drop entries below the current floor, else keep the
             // sub-buffer's own k best (they contain its part of the top k)
+            __syncwarp();
             const int q = qb0 + ql;
             uint2* buf = my_bufs + size_t(q) * capw;
-            const uint32_t fl = ms->floor_bin[q];
-            n[ql] = warp_compact(buf, n[ql], lane,
-                                 [&](uint2 v) { return bin_of<NB, BSHIFT>(v.x, lo) >= fl; });
+            const uint32_t fl = ms->floor_bits[q];
+            n[ql] = warp_compact(buf, n[ql], lane, [&](uint2 v) { return v.x >= fl; });
             if (n[ql] + 32 > uint32_t(capw) / 2 + k / 2 && n[ql] > uint32_t(k)) {
               uint2* one[4] = {buf, buf, buf, buf};
               const uint32_t nn[4] = {n[ql], 0, 0, 0};
@@ -484,31 +473,31 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
           // append in position order; count the appends per score bin
 #pragma unroll
-          for (int ql = 0; ql < QG; ++ql) {
+          for (int ql = 0; ql < QH; ++ql) {
             if ((bal[ql] >> lane) & 1u) {
               const int q = qb0 + ql;
+              const uint32_t bits = __float_as_uint(sc[ql]);
               my_bufs[size_t(q) * capw + n[ql] + __popc(bal[ql] & lt_mask)] =
-                  make_uint2(__float_as_uint(sc[ql]), uint32_t(j));
-              atomicAdd(&ms->hist[q][binv[ql]], 1u);
+                  make_uint2(bits, uint32_t(j));
+              atomicAdd(&ms->hist[q][bin_of<NB, BSHIFT>(bits, lo)], 1u);
             }
+            n[ql] += __popc(bal[ql]);
           }
-          __syncwarp();
-          if (lane == 0) {
-#pragma unroll
-            for (int ql = 0; ql < QG; ++ql) ms->cnt[sub][qb0 + ql] = n[ql] + __popc(bal[ql]);
-          }
-          __syncwarp();
         }
         // raise the floors of this warp's queries to the highest bin with at
         // least k appended entries at or above it (any snapshot of the counts
         // gives a valid floor)
-        if ((t & 1) || t == n_tiles - 1) {
+        if ((t & 3) == 3 || t == n_tiles - 1) {
           for (int q = half * QH + sub; q < (half + 1) * QH; q += 4) {
             uint32_t above, inbin;
             const int fb = hist_cross<NB>(ms->hist[q], uint32_t(k), lane, above, inbin);
-            if (fb > 0 && lane == 0) atomicMax(&ms->floor_bin[q], uint32_t(fb));
+            if (fb > 0 && lane == 0) atomicMax(&ms->floor_bits[q], (uint32_t(fb) + lo) << BSHIFT);
           }
         }
+      }
+      if (lane == 0) {
+#pragma unroll
+        for (int ql = 0; ql < QH; ++ql) ms->cnt[sub][qb0 + ql] = n[ql];
       }
       scorer_sync();
       // ---- outputs of the item: one warp per query ----
