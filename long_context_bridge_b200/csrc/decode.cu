@@ -83,6 +83,20 @@ __device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1,
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// 4-byte asynchronous copy global -> shared; src_bytes 0 writes zeros
+__device__ __forceinline__ void cp_async4(void* dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+
+// arrive on `bar` once this thread's earlier cp.async copies have landed
+// (counts as one of the barrier's expected arrivals)
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -107,6 +121,7 @@ __global__ void __launch_bounds__((DP_WARPS + 1) * 32, 3)
   __shared__ uint16_t sP[DP_WARPS][NT][8 * 16];      // P' [head][key] f16 per warp
   __shared__ float sM[DP_WARPS][NT * 8], sL[DP_WARPS][NT * 8];
   __shared__ uint64_t full[DSTAGES], empty[DSTAGES];
+  __shared__ float sScale[DSTAGES][2][DSTAGE_KEYS];  // K and V scales of a stage's keys
   extern __shared__ uint8_t dsmem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -123,7 +138,7 @@ __global__ void __launch_bounds__((DP_WARPS + 1) * 32, 3)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < DSTAGES; ++i) {
-      mbar_init(&full[i], 1);
+      mbar_init(&full[i], 1 + 32);  // the TMA issuer, plus one per producer lane's scales
       mbar_init(&empty[i], DP_WARPS);
     }
     fence_barrier_init();
@@ -131,13 +146,28 @@ __global__ void __launch_bounds__((DP_WARPS + 1) * 32, 3)
   __syncthreads();
 
   if (warp == DP_WARPS) {
-    // ---------------- producer: K and V tiles of 64 rows -> smem ring -------
+    // ---------------- producer: K and V tiles of 64 rows -> smem ring by TMA,
+    // their per-token scales by cp.async (two keys per lane) ------------------
     if (lane == 0) {
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      for (int si = 0; si < n_st; ++si) {
-        const int slot = si % DSTAGES;
-        if (si >= DSTAGES && !mbar_wait(&empty[slot], ((si / DSTAGES) & 1) ^ 1)) break;
+    }
+    for (int si = 0; si < n_st; ++si) {
+      const int slot = si % DSTAGES;
+      bool go = true;
+      if (lane == 0 && si >= DSTAGES) go = mbar_wait(&empty[slot], ((si / DSTAGES) & 1) ^ 1);
+      if (!__shfl_sync(0xffffffffu, go, 0)) break;
+      const int64_t kbase = c_lo + int64_t(si) * DSTAGE_KEYS;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int64_t key = kbase + lane + 32 * u;
+        const bool in = key < c_hi;
+        const size_t off = (rowbase + size_t(in ? key : c_lo)) * Hkv + g;
+        cp_async4(&sScale[slot][0][lane + 32 * u], ks + off, in ? 4 : 0);
+        cp_async4(&sScale[slot][1][lane + 32 * u], vs + off, in ? 4 : 0);
+      }
+      cp_async_arrive(&full[slot]);
+      if (lane == 0) {
         uint8_t* st = ring + slot * DSTAGE_BYTES;
         const int z = int(rowbase + c_lo) + si * DSTAGE_KEYS;
         mbar_arrive_expect_tx(&full[slot], DSTAGE_BYTES);
@@ -181,26 +211,14 @@ __global__ void __launch_bounds__((DP_WARPS + 1) * 32, 3)
   float* lg = logits + (size_t(b) * Hkv + g) * cap * G;
   bool ok = true;
 
-  // scales of this warp's keys in stage si (loaded one stage ahead)
-  auto load_scales = [&](int si, float (&vsc)[4], float& ks0, float& ks1) {
-    const int64_t key0 = c_lo + si * DSTAGE_KEYS + 16 * warp;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int64_t kv = key0 + 4 * t + u;
-      vsc[u] = kv < c_hi ? __ldg(vs + (rowbase + kv) * Hkv + g) * kPScale : 0.f;
-    }
-    ks0 = key0 + gid < c_hi ? __ldg(ks + (rowbase + key0 + gid) * Hkv + g) : 0.f;
-    ks1 = key0 + gid + 8 < c_hi ? __ldg(ks + (rowbase + key0 + gid + 8) * Hkv + g) : 0.f;
-  };
-  float nvsc[4], nks0 = 0.f, nks1 = 0.f;
-  if (n_st > 0) load_scales(0, nvsc, nks0, nks1);
-
   for (int si = 0; si < n_st; ++si) {
     const int slot = si % DSTAGES;
-    float vsc[4] = {nvsc[0], nvsc[1], nvsc[2], nvsc[3]};
-    const float ks0 = nks0, ks1 = nks1;
-    if (si + 1 < n_st) load_scales(si + 1, nvsc, nks0, nks1);
     ok = ok && mbar_wait(&full[slot], (si / DSTAGES) & 1);
+    // scales of this warp's keys (zero past the chunk's end)
+    float vsc[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) vsc[u] = sScale[slot][1][16 * warp + 4 * t + u] * kPScale;
+    const float ks0 = sScale[slot][0][16 * warp + gid], ks1 = sScale[slot][0][16 * warp + gid + 8];
     const uint8_t* sK = ring + slot * DSTAGE_BYTES;
     const uint8_t* sV = sK + DSTAGE_KEYS * 128;
     // this warp's 16 keys of the stage; rows in the swizzled tile: unit u of
@@ -222,9 +240,12 @@ __global__ void __launch_bounds__((DP_WARPS + 1) * 32, 3)
     }
     const uint32_t kw0[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
     const uint32_t kw1[8] = {kc.x, kc.y, kc.z, kc.w, kd.x, kd.y, kd.z, kd.w};
-    float sacc[NT][4];
+    // two accumulation chains (even and odd steps), added at the end
+    float sacc[NT][4], sacc2[NT][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[nt][e] = sacc2[nt][e] = 0.f;
 #pragma unroll
     for (int s = 0; s < 8; ++s) {
       // row gid: slots 2t,2t+1 (a0) and 2t+8,2t+9 (a2); row gid+8: a1, a3
@@ -232,8 +253,15 @@ __global__ void __launch_bounds__((DP_WARPS + 1) * 32, 3)
       cvt_e4m3x4_f16x2x2(kw0[s], a0, a2);
       cvt_e4m3x4_f16x2x2(kw1[s], a1, a3);
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) mma_f16(sacc[nt], a0, a1, a2, a3, qf[nt][s][0], qf[nt][s][1]);
+      for (int nt = 0; nt < NT; ++nt) {
+        if (s & 1) mma_f16(sacc2[nt], a0, a1, a2, a3, qf[nt][s][0], qf[nt][s][1]);
+        else mma_f16(sacc[nt], a0, a1, a2, a3, qf[nt][s][0], qf[nt][s][1]);
+      }
     }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[nt][e] += sacc2[nt][e];
     // base-2 logits; lane holds keys r0 (c0,c1) and r1 (c2,c3), heads 2t, 2t+1
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -265,16 +293,19 @@ __global__ void __launch_bounds__((DP_WARPS + 1) * 32, 3)
       const float p10 = mn0 == -INFINITY ? 0.f : fast_exp2(s10 - mn0);
       const float p01 = mn1 == -INFINITY ? 0.f : fast_exp2(s01 - mn1);
       const float p11 = mn1 == -INFINITY ? 0.f : fast_exp2(s11 - mn1);
+      const bool grew = mn0 != m_run[nt][0] || mn1 != m_run[nt][1];
       m_run[nt][0] = mn0;
       m_run[nt][1] = mn1;
       l_run[nt][0] = l_run[nt][0] * al0 + p00 + p10;
       l_run[nt][1] = l_run[nt][1] * al1 + p01 + p11;
+      if (__any_sync(0xffffffffu, grew)) {  // rescale only after a new maximum
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        o[nt][i][0] *= al0;
-        o[nt][i][2] *= al0;
-        o[nt][i][1] *= al1;
-        o[nt][i][3] *= al1;
+        for (int i = 0; i < 8; ++i) {
+          o[nt][i][0] *= al0;
+          o[nt][i][2] *= al0;
+          o[nt][i][1] *= al1;
+          o[nt][i][3] *= al1;
+        }
       }
       // P (unscaled by V's scale yet) to shared memory, [head][key] f16;
       // local keys gid (r0) and gid+8 (r1)
@@ -413,9 +444,24 @@ __global__ void __launch_bounds__(256)
   float* sc = score + (size_t(b) * Hkv + g) * cap;
   const int64_t j_hi = min(int64_t(c + 1) * CH, ncand);
   for (int64_t j = int64_t(c) * CH + threadIdx.x; j < j_hi; j += 256) {
+    // the G logits of key j: 16-byte loads where G allows
+    float x[G];
+    if constexpr (G % 4 == 0) {
+#pragma unroll
+      for (int h = 0; h < G; h += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(lg + j * G + h);
+        x[h] = v.x;
+        x[h + 1] = v.y;
+        x[h + 2] = v.z;
+        x[h + 3] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int h = 0; h < G; ++h) x[h] = lg[j * G + h];
+    }
     float acc = 0.f;
 #pragma unroll
-    for (int h = 0; h < G; ++h) acc += fast_exp2(lg[j * G + h] - sl[h]);
+    for (int h = 0; h < G; ++h) acc += fast_exp2(x[h] - sl[h]);
     sc[j] = acc;
     atomicAdd(&sh[__float_as_uint(acc) >> 20], 1u);
   }
