@@ -60,12 +60,6 @@ struct SeqLens {  // sequence lengths, passed by value
   int n[MAX_B];
 };
 
-__device__ __forceinline__ uint32_t cvt_e4m3x2_f16x2(uint32_t two_bytes) {
-  __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_bytes & 0xFFFFu),
-                                             __NV_E4M3);
-  return uint32_t(h.x) | (uint32_t(h.y) << 16);
-}
-
 // both e4m3 pairs of a 32-bit word -> two f16x2 (low pair, high pair)
 __device__ __forceinline__ void cvt_e4m3x4_f16x2x2(uint32_t x, uint32_t& lo, uint32_t& hi) {
   asm("{\n\t.reg .b16 l16, h16;\n\tmov.b32 {l16, h16}, %2;\n\t"
@@ -400,38 +394,63 @@ __global__ void __launch_bounds__((DP_WARPS + 1) * 32, 3)
 // ---------------------------------------------------------------------------
 // decode_merge: grid (Hq, B), 128 threads
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(128)
+constexpr int MERGE_GROUPS = 4;  // groups of 128 threads, each over every 4th chunk
+
+__global__ void __launch_bounds__(128 * MERGE_GROUPS)
     decode_merge(const Partial* __restrict__ part, const float* __restrict__ part_o,
                  SeqLens seq_len, int Hq, int nch, __nv_bfloat16* __restrict__ o,
                  float* __restrict__ lse, float* __restrict__ lse2_out) {
-  const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
+  __shared__ float s_red[MERGE_GROUPS][129];
+  __shared__ float s_max[128 * MERGE_GROUPS / 32];
+  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int d = tid & 127, grp = tid >> 7;
   const int nc = (seq_len.n[b] + CH - 1) / CH;
   const size_t base = (size_t(b) * Hq + h) * nch;
+  // the largest chunk maximum
   float M = -INFINITY;
-  for (int c = 0; c < nc; ++c) M = fmaxf(M, part[base + c].m);
+  for (int c = tid; c < nc; c += 128 * MERGE_GROUPS) M = fmaxf(M, part[base + c].m);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  if ((tid & 31) == 0) s_max[tid >> 5] = M;
+  __syncthreads();
+  M = s_max[0];
+#pragma unroll
+  for (int i = 1; i < 128 * MERGE_GROUPS / 32; ++i) M = fmaxf(M, s_max[i]);
   float L = 0.f, acc = 0.f;
-  for (int c = 0; c < nc; ++c) {
+#pragma unroll 4
+  for (int c = grp; c < nc; c += MERGE_GROUPS) {
     const Partial p = part[base + c];
     const float f = p.m == -INFINITY ? 0.f : fast_exp2(p.m - M);
     L += p.l * f;
     acc += part_o[(base + c) * 128 + d] * f;
   }
-  o[(size_t(b) * Hq + h) * 128 + d] = __float2bfloat16_rn(acc / L);
-  if (d == 0) {
-    const float l2 = M + __log2f(L);
-    lse[size_t(b) * Hq + h] = l2 * kLn2;
-    lse2_out[size_t(b) * Hq + h] = l2;
+  s_red[grp][d] = acc;
+  if (d == 0) s_red[grp][128] = L;
+  __syncthreads();
+  if (grp == 0) {
+    for (int q = 1; q < MERGE_GROUPS; ++q) acc += s_red[q][d];
+    L = 0.f;
+    for (int q = 0; q < MERGE_GROUPS; ++q) L += s_red[q][128];
+    o[(size_t(b) * Hq + h) * 128 + d] = __float2bfloat16_rn(acc / L);
+    if (d == 0) {
+      const float l2 = M + __log2f(L);
+      lse[size_t(b) * Hq + h] = l2 * kLn2;
+      lse2_out[size_t(b) * Hq + h] = l2;
+    }
   }
 }
 
 // ---------------------------------------------------------------------------
 // decode_score: grid (chunks, Hkv, B), 256 threads
 // ---------------------------------------------------------------------------
+__device__ int block_kth_bucket(const uint32_t* __restrict__ gh, uint32_t k, uint32_t* s_scan);
+
 template <int G>
 __global__ void __launch_bounds__(256)
     decode_score(const float* __restrict__ logits, const float* __restrict__ lse2,
-                 SeqLens seq_len, int64_t cap, int Hkv, int w,
-                 float* __restrict__ score, uint32_t* __restrict__ hist) {
+                 SeqLens seq_len, int64_t cap, int Hkv, int k, int w,
+                 float* __restrict__ score, uint32_t* __restrict__ hist,
+                 uint32_t* __restrict__ done, int* __restrict__ kth_bucket) {
   __shared__ uint32_t sh[NBUCKET];
   __shared__ float sl[G];
   const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
@@ -469,6 +488,19 @@ __global__ void __launch_bounds__(256)
   uint32_t* gh = hist + (size_t(b) * Hkv + g) * NBUCKET;
   for (int i = threadIdx.x; i < NBUCKET; i += 256)
     if (sh[i]) atomicAdd(&gh[i], sh[i]);
+  // the last CTA of (b, g) to finish finds the bucket of the k-th best score
+  __shared__ uint32_t s_last, s_scan[256];
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = atomicAdd(&done[size_t(b) * Hkv + g], 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (s_last) {
+    __threadfence();
+    const int kb = block_kth_bucket(gh, uint32_t(k), s_scan);
+    if (threadIdx.x == 0) kth_bucket[size_t(b) * Hkv + g] = kb;
+  }
 }
 
 // bucket holding the k-th largest count from the top (NBUCKET bins, 256
@@ -479,7 +511,7 @@ __device__ int block_kth_bucket(const uint32_t* __restrict__ gh, uint32_t k, uin
   uint32_t c8[8], local = 0;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    c8[i] = gh[NBUCKET - 1 - 8 * tid - i];
+    c8[i] = __ldcg(gh + NBUCKET - 1 - 8 * tid - i);  // other CTAs' atomics, from L2
     local += c8[i];
   }
   s_scan[tid] = local;
@@ -513,10 +545,9 @@ __device__ int block_kth_bucket(const uint32_t* __restrict__ gh, uint32_t k, uin
 // decode_collect: grid (chunks, Hkv, B), 256 threads
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
-    decode_collect(const float* __restrict__ score, const uint32_t* __restrict__ hist,
+    decode_collect(const float* __restrict__ score, const int* __restrict__ kth_bucket,
                    SeqLens seq_len, int64_t cap, int Hkv, int k, int w,
                    uint2* __restrict__ cand, uint32_t* __restrict__ ccount) {
-  __shared__ uint32_t s_scan[256];
   const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int N = seq_len.n[b];
   const int64_t ncand = int64_t(N) - w;
@@ -524,7 +555,7 @@ __global__ void __launch_bounds__(256)
   const int64_t j_lo = int64_t(c) * CH;
   if (j_lo >= ncand) return;
   const size_t bg = size_t(b) * Hkv + g;
-  const int kb = block_kth_bucket(hist + bg * NBUCKET, uint32_t(k), s_scan);
+  const int kb = kth_bucket[bg];
   const uint32_t thr = kb < 0 ? 0u : uint32_t(kb);
   const float* sc = score + bg * cap;
   const int64_t j_hi = min(j_lo + CH, ncand);
@@ -689,12 +720,15 @@ cudaError_t launch_dec_g(const DecodeArgs& a, const SeqLens& d_seq, int max_len,
   float* part_o = reinterpret_cast<float*>(take(size_t(B) * Hq * nch * 128 * 4));
   float* lse2 = reinterpret_cast<float*>(take(size_t(B) * Hq * 4));
   uint32_t* hist = reinterpret_cast<uint32_t*>(take(size_t(B) * Hkv * NBUCKET * 4));
-  uint32_t* ccount = reinterpret_cast<uint32_t*>(take(size_t(B) * Hkv * 4));
+  // per (b, g): candidate count, finished scoring CTAs, k-th best bucket
+  uint32_t* ccount = reinterpret_cast<uint32_t*>(take(size_t(B) * Hkv * 12));
+  uint32_t* done = ccount + size_t(B) * Hkv;
+  int* kth_bucket = reinterpret_cast<int*>(done + size_t(B) * Hkv);
   uint2* cand = reinterpret_cast<uint2*>(take(size_t(B) * Hkv * CAPC * 8));
 
   cudaError_t e = cudaMemsetAsync(hist, 0, size_t(B) * Hkv * NBUCKET * 4, st);
   if (e != cudaSuccess) return e;
-  e = cudaMemsetAsync(ccount, 0, size_t(B) * Hkv * 4, st);
+  e = cudaMemsetAsync(ccount, 0, size_t(B) * Hkv * 8, st);  // counts and tickets
   if (e != cudaSuccess) return e;
   const float sl2 = a.scale * kLog2e;
   // K, V codes viewed as [B*cap tokens][Hkv][64 two-byte units]: 64-row boxes
@@ -709,12 +743,12 @@ cudaError_t launch_dec_g(const DecodeArgs& a, const SeqLens& d_seq, int max_len,
   decode_partial<G><<<dim3(nch_used, Hkv, B), (DP_WARPS + 1) * 32, psmem, st>>>(
       tmK, tmV, reinterpret_cast<const __nv_bfloat16*>(a.q), a.ks, a.vs, d_seq, a.cap, Hkv, nch,
       sl2, logits, part, part_o);
-  decode_merge<<<dim3(Hq, B), 128, 0, st>>>(part, part_o, d_seq, Hq, nch,
+  decode_merge<<<dim3(Hq, B), 128 * MERGE_GROUPS, 0, st>>>(part, part_o, d_seq, Hq, nch,
                                             reinterpret_cast<__nv_bfloat16*>(a.o), a.lse, lse2);
-  decode_score<G><<<dim3(nch_used, Hkv, B), 256, 0, st>>>(logits, lse2, d_seq, a.cap, Hkv, a.w,
-                                                          score, hist);
-  decode_collect<<<dim3(nch_used, Hkv, B), 256, 0, st>>>(score, hist, d_seq, a.cap, Hkv, a.k, a.w,
-                                                         cand, ccount);
+  decode_score<G><<<dim3(nch_used, Hkv, B), 256, 0, st>>>(logits, lse2, d_seq, a.cap, Hkv, a.k,
+                                                          a.w, score, hist, done, kth_bucket);
+  decode_collect<<<dim3(nch_used, Hkv, B), 256, 0, st>>>(score, kth_bucket, d_seq, a.cap, Hkv,
+                                                         a.k, a.w, cand, ccount);
   const int fsmem = CAPC * 8;
   e = ensure_smem_attr(reinterpret_cast<const void*>(decode_final), fsmem);
   if (e != cudaSuccess) return e;
@@ -751,7 +785,7 @@ size_t dec_ws_bytes(int B, int64_t cap, int Hq, int Hkv) {
   auto r = [](size_t x) { return (x + 255) / 256 * 256; };
   return r(size_t(B) * Hkv * cap * G * 4) + r(size_t(B) * Hkv * cap * 4) +
          r(size_t(B) * Hq * nch * sizeof(Partial)) + r(size_t(B) * Hq * nch * 128 * 4) +
-         r(size_t(B) * Hq * 4) + r(size_t(B) * Hkv * NBUCKET * 4) + r(size_t(B) * Hkv * 4) +
+         r(size_t(B) * Hq * 4) + r(size_t(B) * Hkv * NBUCKET * 4) + r(size_t(B) * Hkv * 12) +
          r(size_t(B) * Hkv * CAPC * 8);
 }
 

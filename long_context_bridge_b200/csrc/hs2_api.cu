@@ -118,7 +118,6 @@ hs2_status cuda_status(cudaError_t e) {
     if (!(cond)) return HS2_ERR_INVALID_ARG;      \
   } while (0)
 
-size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 }  // namespace
 

@@ -20,6 +20,7 @@
 // bytes of shared memory per warp to become the B operand.  The FP8 variant
 // converts e4m3 codes to f16 exactly, multiplies the logits by the key's
 // scale and folds the value's scale into P.
+#include <cooperative_groups.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
@@ -35,6 +36,7 @@ namespace {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kPScale = 1024.f;  // FP8: P * v_scale * 2^10 stays in f16's normal range
+constexpr int kDecodeCluster = 8;   // CTAs sharing one decode (sequence, KV head) list
 
 template <bool F16>
 __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -91,8 +93,10 @@ __device__ __forceinline__ float from16(uint16_t v) {
 }
 
 // G query heads of one KV head; FP8: e4m3 cache with per-(token, head) scales;
-// WPR warps share one (row, KV head) pair, splitting its list.
-template <int G, bool FP8, int WPR>
+// WPR warps share one (row, KV head) pair, splitting its list; with CS > 1
+// the CS CTAs of a thread-block cluster share it (CS * WPR parts) and combine
+// their partial softmax states through distributed shared memory.
+template <int G, bool FP8, int WPR, int CS = 1>
 __global__ void __launch_bounds__(128)
     sparse_mma_kernel(const __nv_bfloat16* __restrict__ Q, const void* __restrict__ Kp,
                       const void* __restrict__ Vp, const float* __restrict__ ks,
@@ -106,18 +110,23 @@ __global__ void __launch_bounds__(128)
   __shared__ uint16_t sP[NW][NT][8 * 16];
   __shared__ float sM[NW][NT * 8], sL[NW][NT * 8];
   __shared__ float sO[WPR > 1 ? NW : 1][WPR > 1 ? NT * 8 : 1][WPR > 1 ? 128 : 1];
+  // this CTA's combined state, read by the cluster's first CTA
+  __shared__ float cM[CS > 1 ? NT * 8 : 1], cL[CS > 1 ? NT * 8 : 1];
+  __shared__ float cO[CS > 1 ? NT * 8 : 1][CS > 1 ? 128 : 1];
+  static_assert(CS == 1 || WPR == 4, "a cluster splits pairs that fill their CTAs");
 
   const int warp = warp_id(), lane = lane_id();
   const int gid = lane >> 2, t = lane & 3;
-  const int64_t pair = int64_t(blockIdx.x) * PAIRS + warp / WPR;
-  const int part = warp % WPR;
+  const int64_t pair = int64_t(blockIdx.x / CS) * PAIRS + warp / WPR;
+  const int crank = int(blockIdx.x % CS);  // rank in the cluster (CS > 1)
+  const int part = crank * WPR + warp % WPR;
   const bool active = pair < rows * Hkv;
   const int64_t r = active ? pair / Hkv : 0;
   const int g = active ? int(pair % Hkv) : 0;
   const int Hq = Hkv * G;
   const int64_t tok0 = FP8 ? r * cache_T : 0;  // decode: sequence r's cache rows
   const int32_t* list = idx + (active ? pair : 0) * kw;
-  const int per = (kw + WPR - 1) / WPR;
+  const int per = (kw + WPR * CS - 1) / (WPR * CS);
   const int e_lo = part * per, e_hi = min(kw, e_lo + per);
 
   // query fragments: head nt*8+gid, dims 32t..32t+31 (words 2s, 2s+1 of step s)
@@ -360,7 +369,56 @@ __global__ void __launch_bounds__(128)
       }
     }
     __syncthreads();
-    if (part == 0 && active) {
+    if constexpr (CS > 1) {
+      // combine this CTA's warps per head (unnormalised, relative to cM)
+      for (int h = warp; h < G; h += NW) {
+        float M = -INFINITY;
+        for (int w2 = 0; w2 < WPR; ++w2) M = fmaxf(M, sM[w2][h]);
+        float L = 0.f, f[WPR];
+        for (int w2 = 0; w2 < WPR; ++w2) {
+          f[w2] = M == -INFINITY ? 0.f : fast_exp2(sM[w2][h] - M);
+          L += sL[w2][h] * f[w2];
+        }
+        for (int d = lane; d < 128; d += 32) {
+          float acc = 0.f;
+          for (int w2 = 0; w2 < WPR; ++w2) acc += sO[w2][h][d] * f[w2];
+          cO[h][d] = acc;
+        }
+        if (lane == 0) {
+          cM[h] = M;
+          cL[h] = L;
+        }
+      }
+      namespace cg = cooperative_groups;
+      cg::cluster_group cluster = cg::this_cluster();
+      cluster.sync();
+      if (crank == 0 && active) {
+        for (int h = warp; h < G; h += NW) {
+          float Mr[CS], M = -INFINITY;
+#pragma unroll
+          for (int q = 0; q < CS; ++q) {
+            Mr[q] = *cluster.map_shared_rank(&cM[h], q);
+            M = fmaxf(M, Mr[q]);
+          }
+          float L = 0.f;
+#pragma unroll
+          for (int q = 0; q < CS; ++q) {
+            Mr[q] = M == -INFINITY ? 0.f : fast_exp2(Mr[q] - M);  // weight of CTA q
+            L += *cluster.map_shared_rank(&cL[h], q) * Mr[q];
+          }
+          const float inv = L > 0.f ? oscale / L : 0.f;
+          for (int d = lane; d < 128; d += 32) {
+            float acc = 0.f;
+#pragma unroll
+            for (int q = 0; q < CS; ++q) acc += *cluster.map_shared_rank(&cO[h][d], q) * Mr[q];
+            O[(r * Hq + g * G + h) * 128 + d] = __float2bfloat16_rn(acc * inv);
+          }
+          if (lse != nullptr && lane == 0)
+            lse[r * Hq + g * G + h] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
+        }
+      }
+      cluster.sync();  // the other CTAs' shared memory stays until it has been read
+    } else if (part == 0 && active) {
       const int w0 = warp;  // first warp of this pair
       for (int h = 0; h < G; ++h) {
         float M = -INFINITY;
@@ -388,10 +446,28 @@ cudaError_t launch_g(const SparseArgs& a, cudaStream_t stream) {
   const int64_t pairs = a.T * a.Hkv;
   const float sl2 = a.scale * kLog2e;
   if (a.Kc != nullptr) {
-    // decode: few pairs, each split over the 4 warps of one CTA
-    sparse_mma_kernel<G, true, 4><<<unsigned(pairs), 128, 0, stream>>>(
-        reinterpret_cast<const __nv_bfloat16*>(a.Q), a.Kc, a.Vc, a.ks, a.vs, a.idx,
-        reinterpret_cast<__nv_bfloat16*>(a.O), a.lse, a.T, a.Hkv, a.kw, sl2, a.cache_T);
+    // decode: few pairs, each split over a cluster of kDecodeCluster CTAs of
+    // four warps
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(pairs * kDecodeCluster));
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kDecodeCluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(
+        &cfg, sparse_mma_kernel<G, true, 4, kDecodeCluster>,
+        reinterpret_cast<const __nv_bfloat16*>(a.Q), static_cast<const void*>(a.Kc),
+        static_cast<const void*>(a.Vc), static_cast<const float*>(a.ks),
+        static_cast<const float*>(a.vs), static_cast<const int32_t*>(a.idx),
+        reinterpret_cast<__nv_bfloat16*>(a.O), a.lse, int64_t(a.T), a.Hkv, a.kw, sl2,
+        int64_t(a.cache_T));
+    if (e != cudaSuccess) return e;
   } else {
     sparse_mma_kernel<G, false, 1><<<unsigned((pairs + 3) / 4), 128, 0, stream>>>(
         reinterpret_cast<const __nv_bfloat16*>(a.Q), a.K, a.V, nullptr, nullptr, a.idx,
