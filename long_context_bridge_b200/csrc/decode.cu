@@ -9,13 +9,16 @@
 //
 // Kernels (all on `stream`):
 //   decode_partial  split-KV attention of the G query heads of (b, g) over a
-//                   4096-key chunk: a producer warp streams 64-row K and V
-//                   tiles by TMA (128-byte swizzle) into a shared
-//                   memory ring (3 stages); four warps each take 16 keys of a stage and
-//                   run mma.sync m16n8k16 (e4m3 codes -> f16 exactly, fp32
-//                   accumulation).  The dot-product dimension and the output
-//                   dims are permuted so every lane reads 16 contiguous bytes
-//                   of a K or V row.
+//                   8192-key chunk: a producer warp streams 128-row K and V
+//                   tiles by TMA (128-byte swizzle) into a shared memory ring
+//                   (2 stages) and their per-token scales by cp.async; four
+//                   warps each take 32 keys of a stage and run mma.sync
+//                   m16n8k16 (e4m3 codes -> f16 exactly, fp32 accumulation).
+//                   The dot-product dimension and the output dims are
+//                   permuted so every lane reads 16 contiguous bytes of a K
+//                   or V row.  The KV heads of a chunk are neighbours in the
+//                   grid, so the head slices of the same cache rows are read
+//                   at about the same time.
 //                   Writes base-2 logits (fp32) for the scoring pass and the
 //                   chunk's (max, sum, unnormalised output).
 //   decode_merge    merges the chunks: o (bf16), lse (natural log).
@@ -42,7 +45,7 @@ HS2_STATUS_ACCESSOR(status_decode)
 
 namespace {
 
-constexpr int CH = 4096;            // keys per decode_partial CTA
+constexpr int CH = 8192;            // keys per decode_partial CTA
 constexpr int DP_WARPS = 4;         // each warp: CH / 4 keys, 16 per step
 constexpr int NBUCKET = 2048;       // score buckets (bits >> 20 of fp32 < 2^8)
 constexpr int CAPC = 8192;          // candidate list capacity per (b, g)
@@ -97,10 +100,11 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
 }
 
 // ---------------------------------------------------------------------------
-// decode_partial: grid (chunks, Hkv, B), DP_WARPS warps
+// decode_partial: grid (Hkv, chunks, B), DP_WARPS consumer warps + 1 producer
 // ---------------------------------------------------------------------------
-constexpr int DSTAGE_KEYS = 64;                   // keys per TMA stage
-constexpr int DSTAGES = 3;                        // ring depth
+constexpr int KPW = 32;                           // keys per warp per stage
+constexpr int DSTAGE_KEYS = DP_WARPS * KPW;       // keys per TMA stage
+constexpr int DSTAGES = 2;                        // ring depth
 constexpr int DSTAGE_BYTES = 2 * DSTAGE_KEYS * 128;  // K and V codes
 
 template <int G>
@@ -112,7 +116,7 @@ __global__ void __launch_bounds__((DP_WARPS + 1) * 32, 3)
                    Partial* __restrict__ part, float* __restrict__ part_o) {
   constexpr int NT = G > 8 ? G / 8 : 1;   // 8-head n-tiles
   constexpr int GH = G < 8 ? G : 8;       // real heads per n-tile
-  __shared__ uint16_t sP[DP_WARPS][NT][8 * 16];      // P' [head][key] f16 per warp
+  __shared__ uint16_t sP[DP_WARPS][NT][8 * KPW];     // P [head][key] f16 per warp
   __shared__ float sM[DP_WARPS][NT * 8], sL[DP_WARPS][NT * 8];
   __shared__ uint64_t full[DSTAGES], empty[DSTAGES];
   __shared__ float sScale[DSTAGES][2][DSTAGE_KEYS];  // K and V scales of a stage's keys
@@ -120,7 +124,9 @@ __global__ void __launch_bounds__((DP_WARPS + 1) * 32, 3)
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) &
                                              ~uintptr_t(1023));
 
-  const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  // the KV heads of a chunk are neighbours in the grid, so the 128-byte head
+  // slices of the same cache rows are read at about the same time
+  const int g = blockIdx.x, c = blockIdx.y, b = blockIdx.z;
   const int warp = warp_id(), lane = lane_id();
   const int gid = lane >> 2, t = lane & 3;
   const int N = seq_len.n[b];
@@ -153,7 +159,7 @@ __global__ void __launch_bounds__((DP_WARPS + 1) * 32, 3)
       if (!__shfl_sync(0xffffffffu, go, 0)) break;
       const int64_t kbase = c_lo + int64_t(si) * DSTAGE_KEYS;
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
+      for (int u = 0; u < DSTAGE_KEYS / 32; ++u) {
         const int64_t key = kbase + lane + 32 * u;
         const bool in = key < c_hi;
         const size_t off = (rowbase + size_t(in ? key : c_lo)) * Hkv + g;
@@ -208,73 +214,66 @@ __global__ void __launch_bounds__((DP_WARPS + 1) * 32, 3)
   for (int si = 0; si < n_st; ++si) {
     const int slot = si % DSTAGES;
     ok = ok && mbar_wait(&full[slot], (si / DSTAGES) & 1);
-    // scales of this warp's keys (zero past the chunk's end)
-    float vsc[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) vsc[u] = sScale[slot][1][16 * warp + 4 * t + u] * kPScale;
-    const float ks0 = sScale[slot][0][16 * warp + gid], ks1 = sScale[slot][0][16 * warp + gid + 8];
     const uint8_t* sK = ring + slot * DSTAGE_BYTES;
     const uint8_t* sV = sK + DSTAGE_KEYS * 128;
-    // this warp's 16 keys of the stage; rows in the swizzled tile: unit u of
-    // row r sits at r*128 + ((u ^ (r & 7)) << 4)
-    const int rA = 16 * warp + gid, rB = rA + 8;
-    const int64_t key0 = c_lo + si * DSTAGE_KEYS + 16 * warp;
-    const int64_t r0 = key0 + gid, r1 = key0 + gid + 8;
-    const bool v0 = r0 < c_hi, v1 = r1 < c_hi;
-    const uint4 ka = *reinterpret_cast<const uint4*>(sK + rA * 128 + (((2 * t) ^ (rA & 7)) << 4));
-    const uint4 kb = *reinterpret_cast<const uint4*>(sK + rA * 128 + (((2 * t + 1) ^ (rA & 7)) << 4));
-    const uint4 kc = *reinterpret_cast<const uint4*>(sK + rB * 128 + (((2 * t) ^ (rB & 7)) << 4));
-    const uint4 kd = *reinterpret_cast<const uint4*>(sK + rB * 128 + (((2 * t + 1) ^ (rB & 7)) << 4));
-    // ---- V rows key0 + 4t + u, bytes 16*gid .. 16*gid+15
-    uint4 vr[4];
+    const int wk0 = KPW * warp;  // this warp's first row of the stage
+    const int64_t key0 = c_lo + int64_t(si) * DSTAGE_KEYS + wk0;
+    // ---- S^T = K q^T for the warp's two 16-key groups (independent chains);
+    // rows in the swizzled tile: unit u of row r sits at r*128 + ((u ^ (r & 7)) << 4)
+    float sacc[2][NT][4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int rv = 16 * warp + 4 * t + u;
-      vr[u] = *reinterpret_cast<const uint4*>(sV + rv * 128 + ((gid ^ (rv & 7)) << 4));
-    }
-    const uint32_t kw0[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
-    const uint32_t kw1[8] = {kc.x, kc.y, kc.z, kc.w, kd.x, kd.y, kd.z, kd.w};
-    // two accumulation chains (even and odd steps), added at the end
-    float sacc[NT][4], sacc2[NT][4];
+    for (int q2 = 0; q2 < 2; ++q2) {
+      const int rA = wk0 + 16 * q2 + gid, rB = rA + 8;
+      const uint4 ka = *reinterpret_cast<const uint4*>(sK + rA * 128 + (((2 * t) ^ (rA & 7)) << 4));
+      const uint4 kb = *reinterpret_cast<const uint4*>(sK + rA * 128 + (((2 * t + 1) ^ (rA & 7)) << 4));
+      const uint4 kc = *reinterpret_cast<const uint4*>(sK + rB * 128 + (((2 * t) ^ (rB & 7)) << 4));
+      const uint4 kd = *reinterpret_cast<const uint4*>(sK + rB * 128 + (((2 * t + 1) ^ (rB & 7)) << 4));
+      const uint32_t kw0[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
+      const uint32_t kw1[8] = {kc.x, kc.y, kc.z, kc.w, kd.x, kd.y, kd.z, kd.w};
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+      for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) sacc[nt][e] = sacc2[nt][e] = 0.f;
+        for (int e = 0; e < 4; ++e) sacc[q2][nt][e] = 0.f;
 #pragma unroll
-    for (int s = 0; s < 8; ++s) {
-      // row gid: slots 2t,2t+1 (a0) and 2t+8,2t+9 (a2); row gid+8: a1, a3
-      uint32_t a0, a1, a2, a3;
-      cvt_e4m3x4_f16x2x2(kw0[s], a0, a2);
-      cvt_e4m3x4_f16x2x2(kw1[s], a1, a3);
+      for (int s = 0; s < 8; ++s) {
+        // row gid: slots 2t,2t+1 (a0) and 2t+8,2t+9 (a2); row gid+8: a1, a3
+        uint32_t a0, a1, a2, a3;
+        cvt_e4m3x4_f16x2x2(kw0[s], a0, a2);
+        cvt_e4m3x4_f16x2x2(kw1[s], a1, a3);
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        if (s & 1) mma_f16(sacc2[nt], a0, a1, a2, a3, qf[nt][s][0], qf[nt][s][1]);
-        else mma_f16(sacc[nt], a0, a1, a2, a3, qf[nt][s][0], qf[nt][s][1]);
+        for (int nt = 0; nt < NT; ++nt)
+          mma_f16(sacc[q2][nt], a0, a1, a2, a3, qf[nt][s][0], qf[nt][s][1]);
       }
     }
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) sacc[nt][e] += sacc2[nt][e];
-    // base-2 logits; lane holds keys r0 (c0,c1) and r1 (c2,c3), heads 2t, 2t+1
+    // ---- base-2 logits; lane holds, per group q2, keys 16q2+gid (c0,c1) and
+    // 16q2+gid+8 (c2,c3) for heads 2t, 2t+1
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const int h0 = nt * 8 + 2 * t;
-      float s00 = v0 ? sacc[nt][0] * ks0 * scale_log2 : -INFINITY;
-      float s01 = v0 ? sacc[nt][1] * ks0 * scale_log2 : -INFINITY;
-      float s10 = v1 ? sacc[nt][2] * ks1 * scale_log2 : -INFINITY;
-      float s11 = v1 ? sacc[nt][3] * ks1 * scale_log2 : -INFINITY;
-      if (h0 >= GH + nt * 8) s00 = s10 = -INFINITY;      // padded heads
-      if (h0 + 1 >= GH + nt * 8) s01 = s11 = -INFINITY;
-      if (h0 + 1 < G) {
-        if (v0) *reinterpret_cast<float2*>(lg + r0 * G + h0) = make_float2(s00, s01);
-        if (v1) *reinterpret_cast<float2*>(lg + r1 * G + h0) = make_float2(s10, s11);
-      } else if (h0 < G) {
-        if (v0) lg[r0 * G + h0] = s00;
-        if (v1) lg[r1 * G + h0] = s10;
+      float sv[2][2][2];  // [group][key gid / gid+8][head 2t / 2t+1]
+#pragma unroll
+      for (int q2 = 0; q2 < 2; ++q2) {
+        const int64_t r0 = key0 + 16 * q2 + gid, r1 = r0 + 8;
+        const bool v0 = r0 < c_hi, v1 = r1 < c_hi;
+        const float c0 = sScale[slot][0][wk0 + 16 * q2 + gid] * scale_log2;
+        const float c1 = sScale[slot][0][wk0 + 16 * q2 + gid + 8] * scale_log2;
+        sv[q2][0][0] = v0 ? sacc[q2][nt][0] * c0 : -INFINITY;
+        sv[q2][0][1] = v0 ? sacc[q2][nt][1] * c0 : -INFINITY;
+        sv[q2][1][0] = v1 ? sacc[q2][nt][2] * c1 : -INFINITY;
+        sv[q2][1][1] = v1 ? sacc[q2][nt][3] * c1 : -INFINITY;
+        if (h0 >= GH + nt * 8) sv[q2][0][0] = sv[q2][1][0] = -INFINITY;  // padded heads
+        if (h0 + 1 >= GH + nt * 8) sv[q2][0][1] = sv[q2][1][1] = -INFINITY;
+        if (h0 + 1 < G) {
+          if (v0) *reinterpret_cast<float2*>(lg + r0 * G + h0) = make_float2(sv[q2][0][0], sv[q2][0][1]);
+          if (v1) *reinterpret_cast<float2*>(lg + r1 * G + h0) = make_float2(sv[q2][1][0], sv[q2][1][1]);
+        } else if (h0 < G) {
+          if (v0) lg[r0 * G + h0] = sv[q2][0][0];
+          if (v1) lg[r1 * G + h0] = sv[q2][1][0];
+        }
       }
-      // online softmax over this step's 16 keys for heads h0, h0+1
-      float mx0 = fmaxf(s00, s10), mx1 = fmaxf(s01, s11);
+      // online softmax over the warp's 32 keys of the stage for heads h0, h0+1
+      float mx0 = fmaxf(fmaxf(sv[0][0][0], sv[0][1][0]), fmaxf(sv[1][0][0], sv[1][1][0]));
+      float mx1 = fmaxf(fmaxf(sv[0][0][1], sv[0][1][1]), fmaxf(sv[1][0][1], sv[1][1][1]));
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1) {
         mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
@@ -283,15 +282,19 @@ __global__ void __launch_bounds__((DP_WARPS + 1) * 32, 3)
       const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
       const float al0 = mn0 == -INFINITY ? 1.f : fast_exp2(m_run[nt][0] - mn0);
       const float al1 = mn1 == -INFINITY ? 1.f : fast_exp2(m_run[nt][1] - mn1);
-      const float p00 = mn0 == -INFINITY ? 0.f : fast_exp2(s00 - mn0);
-      const float p10 = mn0 == -INFINITY ? 0.f : fast_exp2(s10 - mn0);
-      const float p01 = mn1 == -INFINITY ? 0.f : fast_exp2(s01 - mn1);
-      const float p11 = mn1 == -INFINITY ? 0.f : fast_exp2(s11 - mn1);
       const bool grew = mn0 != m_run[nt][0] || mn1 != m_run[nt][1];
+      float pv[2][2][2];
+#pragma unroll
+      for (int q2 = 0; q2 < 2; ++q2)
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          pv[q2][kk][0] = mn0 == -INFINITY ? 0.f : fast_exp2(sv[q2][kk][0] - mn0);
+          pv[q2][kk][1] = mn1 == -INFINITY ? 0.f : fast_exp2(sv[q2][kk][1] - mn1);
+        }
       m_run[nt][0] = mn0;
       m_run[nt][1] = mn1;
-      l_run[nt][0] = l_run[nt][0] * al0 + p00 + p10;
-      l_run[nt][1] = l_run[nt][1] * al1 + p01 + p11;
+      l_run[nt][0] = l_run[nt][0] * al0 + ((pv[0][0][0] + pv[0][1][0]) + (pv[1][0][0] + pv[1][1][0]));
+      l_run[nt][1] = l_run[nt][1] * al1 + ((pv[0][0][1] + pv[0][1][1]) + (pv[1][0][1] + pv[1][1][1]));
       if (__any_sync(0xffffffffu, grew)) {  // rescale only after a new maximum
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -301,44 +304,57 @@ __global__ void __launch_bounds__((DP_WARPS + 1) * 32, 3)
           o[nt][i][3] *= al1;
         }
       }
-      // P (unscaled by V's scale yet) to shared memory, [head][key] f16;
-      // local keys gid (r0) and gid+8 (r1)
+      // P (not yet times V's scale) to shared memory, [head][32 keys] f16
       uint16_t* sp = sP[warp][nt];
-      const __half hp00 = __float2half_rn(p00), hp01 = __float2half_rn(p01);
-      const __half hp10 = __float2half_rn(p10), hp11 = __float2half_rn(p11);
-      sp[(2 * t) * 16 + gid] = *reinterpret_cast<const uint16_t*>(&hp00);
-      sp[(2 * t + 1) * 16 + gid] = *reinterpret_cast<const uint16_t*>(&hp01);
-      sp[(2 * t) * 16 + gid + 8] = *reinterpret_cast<const uint16_t*>(&hp10);
-      sp[(2 * t + 1) * 16 + gid + 8] = *reinterpret_cast<const uint16_t*>(&hp11);
+#pragma unroll
+      for (int q2 = 0; q2 < 2; ++q2)
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const __half hp = __float2half_rn(pv[q2][kk][e]);
+            sp[(2 * t + e) * KPW + 16 * q2 + 8 * kk + gid] = *reinterpret_cast<const uint16_t*>(&hp);
+          }
     }
     __syncwarp();
-    // ---- O^T += V^T P'^T: M = 16 dims (permuted), K = 16 keys (4t+u), N = heads
-    // B fragment: P'[head gid][keys 4t, 4t+1] and [4t+2, 4t+3], times V scale
+    // ---- O^T += V^T P'^T per 16-key group: M = 16 dims (permuted), K = 16
+    // keys (4t+u), N = heads; B fragment: P'[head gid][keys 4t, 4t+1] and
+    // [4t+2, 4t+3], times V's scale (which carries the 2^10 factor)
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const uint16_t* sp = sP[warp][nt] + gid * 16 + 4 * t;
-      const float f0 = __half2float(*reinterpret_cast<const __half*>(sp + 0)) * vsc[0];
-      const float f1 = __half2float(*reinterpret_cast<const __half*>(sp + 1)) * vsc[1];
-      const float f2 = __half2float(*reinterpret_cast<const __half*>(sp + 2)) * vsc[2];
-      const float f3 = __half2float(*reinterpret_cast<const __half*>(sp + 3)) * vsc[3];
-      // vsc already carries the 2^10 factor (see below)
-      const uint32_t b0 = pack_f16x2(f0, f1), b1 = pack_f16x2(f2, f3);
+    for (int q2 = 0; q2 < 2; ++q2) {
+      uint4 vr[4];
+      float vsc[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int rv = wk0 + 16 * q2 + 4 * t + u;
+        vr[u] = *reinterpret_cast<const uint4*>(sV + rv * 128 + ((gid ^ (rv & 7)) << 4));
+        vsc[u] = sScale[slot][1][rv] * kPScale;
+      }
       const uint32_t vw[4][4] = {{vr[0].x, vr[0].y, vr[0].z, vr[0].w},
                                  {vr[1].x, vr[1].y, vr[1].z, vr[1].w},
                                  {vr[2].x, vr[2].y, vr[2].z, vr[2].w},
                                  {vr[3].x, vr[3].y, vr[3].z, vr[3].w}};
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        // bytes 2i / 2i+1 of a row slice = dims 16*gid + 2i (MMA row gid) and
-        // 16*gid + 2i + 1 (row gid+8).  One permute gathers, for two keys,
-        // [key0 dim 2i, key1 dim 2i, key0 dim 2i+1, key1 dim 2i+1].
-        const int wd = i >> 1, p = (i & 1) * 2;
-        const uint32_t sel = uint32_t(p) | uint32_t(p + 4) << 4 | uint32_t(p + 1) << 8 |
-                             uint32_t(p + 5) << 12;
-        uint32_t a0, a1, a2, a3;
-        cvt_e4m3x4_f16x2x2(__byte_perm(vw[0][wd], vw[1][wd], sel), a0, a1);
-        cvt_e4m3x4_f16x2x2(__byte_perm(vw[2][wd], vw[3][wd], sel), a2, a3);
-        mma_f16(o[nt][i], a0, a1, a2, a3, b0, b1);
+      for (int nt = 0; nt < NT; ++nt) {
+        const uint16_t* sp = sP[warp][nt] + gid * KPW + 16 * q2 + 4 * t;
+        const float f0 = __half2float(*reinterpret_cast<const __half*>(sp + 0)) * vsc[0];
+        const float f1 = __half2float(*reinterpret_cast<const __half*>(sp + 1)) * vsc[1];
+        const float f2 = __half2float(*reinterpret_cast<const __half*>(sp + 2)) * vsc[2];
+        const float f3 = __half2float(*reinterpret_cast<const __half*>(sp + 3)) * vsc[3];
+        const uint32_t b0 = pack_f16x2(f0, f1), b1 = pack_f16x2(f2, f3);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          // bytes 2i / 2i+1 of a row slice = dims 16*gid + 2i (MMA row gid) and
+          // 16*gid + 2i + 1 (row gid+8).  One permute gathers, for two keys,
+          // [key0 dim 2i, key1 dim 2i, key0 dim 2i+1, key1 dim 2i+1].
+          const int wd = i >> 1, p = (i & 1) * 2;
+          const uint32_t sel = uint32_t(p) | uint32_t(p + 4) << 4 | uint32_t(p + 1) << 8 |
+                               uint32_t(p + 5) << 12;
+          uint32_t a0, a1, a2, a3;
+          cvt_e4m3x4_f16x2x2(__byte_perm(vw[0][wd], vw[1][wd], sel), a0, a1);
+          cvt_e4m3x4_f16x2x2(__byte_perm(vw[2][wd], vw[3][wd], sel), a2, a3);
+          mma_f16(o[nt][i], a0, a1, a2, a3, b0, b1);
+        }
       }
     }
     __syncwarp();
@@ -560,21 +576,38 @@ __global__ void __launch_bounds__(256)
   const float* sc = score + bg * cap;
   const int64_t j_hi = min(j_lo + CH, ncand);
   const int lane = lane_id();
-  for (int64_t base = j_lo; base < j_hi; base += 256) {
-    const int64_t j = base + threadIdx.x;
-    float v = 0.f;
-    bool take = false;
-    if (j < j_hi) {
-      v = sc[j];
-      take = (__float_as_uint(v) >> 20) >= thr;
+  const bool vec = (cap & 3) == 0;  // rows of scores start 16-byte aligned
+  // rounds of 2048 keys: thread owns keys j0 .. j0+3 and j0+1024 .. j0+1027;
+  // all eight loads are issued before any is used
+  for (int64_t base = j_lo; base < j_hi; base += 2048) {
+    float v[8];
+#pragma unroll
+    for (int hlf = 0; hlf < 2; ++hlf) {
+      const int64_t j0 = base + 1024 * hlf + 4 * threadIdx.x;
+      if (vec && j0 + 3 < j_hi) {
+        const float4 x = __ldcs(reinterpret_cast<const float4*>(sc + j0));
+        v[4 * hlf] = x.x;
+        v[4 * hlf + 1] = x.y;
+        v[4 * hlf + 2] = x.z;
+        v[4 * hlf + 3] = x.w;
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) v[4 * hlf + u] = j0 + u < j_hi ? sc[j0 + u] : 0.f;
+      }
     }
-    const uint32_t bal = __ballot_sync(0xffffffffu, take);
-    if (bal) {
-      uint32_t pos = 0;
-      if (lane == __ffs(bal) - 1) pos = atomicAdd(&ccount[bg], __popc(bal));
-      pos = __shfl_sync(0xffffffffu, pos, __ffs(bal) - 1);
-      const uint32_t p = pos + __popc(bal & ((1u << lane) - 1u));
-      if (take && p < uint32_t(CAPC)) cand[bg * CAPC + p] = make_uint2(__float_as_uint(v), uint32_t(j));
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int64_t j = base + 1024 * (e >> 2) + 4 * threadIdx.x + (e & 3);
+      const bool take = j < j_hi && (__float_as_uint(v[e]) >> 20) >= thr;
+      const uint32_t bal = __ballot_sync(0xffffffffu, take);
+      if (bal) {
+        uint32_t pos = 0;
+        if (lane == __ffs(bal) - 1) pos = atomicAdd(&ccount[bg], __popc(bal));
+        pos = __shfl_sync(0xffffffffu, pos, __ffs(bal) - 1);
+        const uint32_t p = pos + __popc(bal & ((1u << lane) - 1u));
+        if (take && p < uint32_t(CAPC))
+          cand[bg * CAPC + p] = make_uint2(__float_as_uint(v[e]), uint32_t(j));
+      }
     }
   }
 }
@@ -740,7 +773,7 @@ cudaError_t launch_dec_g(const DecodeArgs& a, const SeqLens& d_seq, int max_len,
   const int psmem = DSTAGES * DSTAGE_BYTES + 1024;
   e = ensure_smem_attr(reinterpret_cast<const void*>(decode_partial<G>), psmem);
   if (e != cudaSuccess) return e;
-  decode_partial<G><<<dim3(nch_used, Hkv, B), (DP_WARPS + 1) * 32, psmem, st>>>(
+  decode_partial<G><<<dim3(Hkv, nch_used, B), (DP_WARPS + 1) * 32, psmem, st>>>(
       tmK, tmV, reinterpret_cast<const __nv_bfloat16*>(a.q), a.ks, a.vs, d_seq, a.cap, Hkv, nch,
       sl2, logits, part, part_o);
   decode_merge<<<dim3(Hq, B), 128 * MERGE_GROUPS, 0, st>>>(part, part_o, d_seq, Hq, nch,
