@@ -302,8 +302,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t lo = top - (NB - 1);
 
   auto item = [&](int it, int& q0, int& g, int& n_tiles, bool& score) {
-    const int qb = nqb - 1 - it / Hkv;  // heaviest items first
-    g = it % Hkv;
+    // KV-head-major, heaviest query blocks first within a head, so that the
+    // CTAs running at one time stream the same head's K through L2
+    const int qb = nqb - 1 - it % nqb;
+    g = it / nqb;
     q0 = qb * QT;
     const int q_last = min(q0 + QT, T) - 1;
     score = k > 0 && (q_last - w + 1) > k;

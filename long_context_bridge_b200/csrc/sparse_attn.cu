@@ -121,11 +121,13 @@ __global__ void __launch_bounds__(128)
   const int crank = int(blockIdx.x % CS);  // rank in the cluster (CS > 1)
   const int part = crank * WPR + warp % WPR;
   const bool active = pair < rows * Hkv;
-  const int64_t r = active ? pair / Hkv : 0;
-  const int g = active ? int(pair % Hkv) : 0;
+  // KV-head-major pairs: a CTA's warps take consecutive rows of one KV head,
+  // whose lists share the window and much of the rest
+  const int64_t r = active ? pair % rows : 0;
+  const int g = active ? int(pair / rows) : 0;
   const int Hq = Hkv * G;
   const int64_t tok0 = FP8 ? r * cache_T : 0;  // decode: sequence r's cache rows
-  const int32_t* list = idx + (active ? pair : 0) * kw;
+  const int32_t* list = idx + (r * Hkv + g) * kw;
   const int per = (kw + WPR * CS - 1) / (WPR * CS);
   const int e_lo = part * per, e_hi = min(kw, e_lo + per);
 
