@@ -11,12 +11,15 @@
 // The dot-product dimension and the output dims are permuted (a sum does not
 // care about the order of its terms, and the output permutation is undone at
 // the store) so that every lane's fragment words are contiguous in memory:
-//   * QK^T: lane (gid, t) reads dims 32t..32t+31 of gathered key rows gid and
-//     gid+8 -- for bf16 these words are the A registers as they are;
-//   * PV: lane (gid, t) reads dims 16*gid..16*gid+15 of gathered value rows
-//     4t..4t+3, paired into A registers with one byte permute each.
+//   * QK^T: lane (gid, t) reads 32 dims of gathered key rows gid and gid+8 --
+//     bf16: dims 32u + 8t .. +7 for u = 0..3, FP8: dims 32t .. 32t+31; for
+//     bf16 these words are the A registers as they are;
+//   * PV: lane (gid, t) reads 16 dims of gathered value rows 4t..4t+3 --
+//     bf16: dims 8*gid .. +7 and 64 + 8*gid .. +7, FP8: 16*gid .. +15 --
+//     paired into A registers with one byte permute each.
 // Each gathered row is read by four (K) or eight (V) lanes with 16-byte loads
-// that cover it exactly.  Softmax is online and base 2; P goes through 256
+// that cover it exactly; in the bf16 layout the lanes of one load instruction
+// read whole 32-byte sectors of each row.  Softmax is online and base 2; P goes through 256
 // bytes of shared memory per warp to become the B operand.  The FP8 variant
 // converts e4m3 codes to f16 exactly, multiplies the logits by the key's
 // scale and folds the value's scale into P.
@@ -131,17 +134,18 @@ __global__ void __launch_bounds__(128)
   const int per = (kw + WPR * CS - 1) / (WPR * CS);
   const int e_lo = part * per, e_hi = min(kw, e_lo + per);
 
-  // query fragments: head nt*8+gid, dims 32t..32t+31 (words 2s, 2s+1 of step s)
+  // query fragments: head nt*8+gid; step s = 2u + h2 uses the dims that lane
+  // t's K loads hold: bf16 dims 8t + 32u + 4*h2 + {0..3}, FP8 dims 32t + 4s + {0..3}
   uint32_t qf[NT][8][2];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const int hh = nt * 8 + gid;
     const bool real = hh < G && active;
     const uint4* qr = reinterpret_cast<const uint4*>(Q + (r * Hq + g * G + (real ? hh : 0)) * 128 +
-                                                     32 * t);
+                                                     (FP8 ? 32 * t : 8 * t));
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const uint4 w = real ? __ldg(qr + u) : make_uint4(0, 0, 0, 0);
+      const uint4 w = real ? __ldg(qr + (FP8 ? u : 4 * u)) : make_uint4(0, 0, 0, 0);
       const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2) {
@@ -184,22 +188,26 @@ __global__ void __launch_bounds__(128)
     float vsc[4] = {0.f, 0.f, 0.f, 0.f};
     float ksA = 1.f, ksB = 1.f;
     if constexpr (!FP8) {
+      // lanes t = 0..3 of a row read 64 contiguous bytes per load (dims
+      // 32u + 8t .. +7): every 32-byte sector they touch is used whole
       const uint4* pa = reinterpret_cast<const uint4*>(
-          reinterpret_cast<const __nv_bfloat16*>(Kp) + rowA * 128 + 32 * t);
+          reinterpret_cast<const __nv_bfloat16*>(Kp) + rowA * 128 + 8 * t);
       const uint4* pb = reinterpret_cast<const uint4*>(
-          reinterpret_cast<const __nv_bfloat16*>(Kp) + rowB * 128 + 32 * t);
+          reinterpret_cast<const __nv_bfloat16*>(Kp) + rowB * 128 + 8 * t);
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const uint4 x = __ldg(pa + u), y = __ldg(pb + u);
+        const uint4 x = __ldg(pa + 4 * u), y = __ldg(pb + 4 * u);
         ka[4 * u] = x.x; ka[4 * u + 1] = x.y; ka[4 * u + 2] = x.z; ka[4 * u + 3] = x.w;
         kb[4 * u] = y.x; kb[4 * u + 1] = y.y; kb[4 * u + 2] = y.z; kb[4 * u + 3] = y.w;
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int64_t rv = (tok0 + (jP[u] >= 0 ? jP[u] : 0)) * Hkv + g;
+        // lanes gid = 0..7 read 128 contiguous bytes per load: dims
+        // 8*gid .. +7 and 64 + 8*gid .. +7
         const uint4* pv = reinterpret_cast<const uint4*>(
-            reinterpret_cast<const __nv_bfloat16*>(Vp) + rv * 128 + 16 * gid);
-        const uint4 x = __ldg(pv), y = __ldg(pv + 1);
+            reinterpret_cast<const __nv_bfloat16*>(Vp) + rv * 128 + 8 * gid);
+        const uint4 x = __ldg(pv), y = __ldg(pv + 8);
         vw[u][0] = x.x; vw[u][1] = x.y; vw[u][2] = x.z; vw[u][3] = x.w;
         vw[u][4] = y.x; vw[u][5] = y.y; vw[u][6] = y.z; vw[u][7] = y.w;
         vsc[u] = jP[u] >= 0 ? 1.f : 0.f;
@@ -290,7 +298,8 @@ __global__ void __launch_bounds__(128)
     }
     __syncwarp();
     // ---- O^T += V^T P^T: K slots {2t,2t+1,2t+8,2t+9} = keys 4t+{0,1,2,3};
-    // MMA i, row gid -> dim 16*gid+2i, row gid+8 -> dim 16*gid+2i+1
+    // MMA i, row gid -> dim D(i) = 16*gid + 2i (FP8) or
+    // 8*gid + 64*(i/4) + 2*(i%4) (bf16); row gid+8 -> D(i) + 1
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const uint16_t* sp = sP[warp][nt] + gid * 16 + 4 * t;
@@ -300,7 +309,7 @@ __global__ void __launch_bounds__(128)
       for (int i = 0; i < 8; ++i) {
         uint32_t a0, a1, a2, a3;
         if constexpr (!FP8) {
-          // word i of a row slice = dims 16*gid+2i (low), +1 (high)
+          // word i of the lane's row slices = dims D(i) (low), D(i) + 1 (high)
           a0 = __byte_perm(vw[0][i], vw[1][i], 0x5410);
           a1 = __byte_perm(vw[0][i], vw[1][i], 0x7632);
           a2 = __byte_perm(vw[2][i], vw[3][i], 0x5410);
@@ -346,9 +355,12 @@ __global__ void __launch_bounds__(128)
         uint32_t pk[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(o[nt][i][e] * inv, o[nt][i][e + 2] * inv);
-        uint4* dst = reinterpret_cast<uint4*>(O + (r * Hq + g * G + h) * 128 + 16 * gid);
-        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        __nv_bfloat16* orow = O + (r * Hq + g * G + h) * 128;
+        // pk[i] holds dims D(i), D(i) + 1
+        uint4* d0 = reinterpret_cast<uint4*>(orow + (FP8 ? 16 * gid : 8 * gid));
+        uint4* d1 = reinterpret_cast<uint4*>(orow + (FP8 ? 16 * gid + 8 : 8 * gid + 64));
+        *d0 = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *d1 = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         if (lse != nullptr && gid == 0)
           lse[r * Hq + g * G + h] = l > 0.f ? (m_run[nt][e] + __log2f(l)) * kLn2 : -INFINITY;
       }
@@ -364,10 +376,11 @@ __global__ void __launch_bounds__(128)
       }
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        sO[warp][nt * 8 + 2 * t][16 * gid + 2 * i] = o[nt][i][0];
-        sO[warp][nt * 8 + 2 * t + 1][16 * gid + 2 * i] = o[nt][i][1];
-        sO[warp][nt * 8 + 2 * t][16 * gid + 2 * i + 1] = o[nt][i][2];
-        sO[warp][nt * 8 + 2 * t + 1][16 * gid + 2 * i + 1] = o[nt][i][3];
+        const int d = FP8 ? 16 * gid + 2 * i : 8 * gid + 64 * (i >> 2) + 2 * (i & 3);
+        sO[warp][nt * 8 + 2 * t][d] = o[nt][i][0];
+        sO[warp][nt * 8 + 2 * t + 1][d] = o[nt][i][1];
+        sO[warp][nt * 8 + 2 * t][d + 1] = o[nt][i][2];
+        sO[warp][nt * 8 + 2 * t + 1][d + 1] = o[nt][i][3];
       }
     }
     __syncthreads();
