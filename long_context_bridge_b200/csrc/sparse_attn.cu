@@ -170,10 +170,13 @@ __global__ void __launch_bounds__(128)
     for (int i = 0; i < 8; ++i) o[nt][i][0] = o[nt][i][1] = o[nt][i][2] = o[nt][i][3] = 0.f;
   }
 
+  // positions of a step's 16 list entries (lanes 16-31 repeat 0-15), loaded
+  // one step ahead so that a step's gathers do not wait for its list load
+  int jl_next = (active && e_lo + (lane & 15) < e_hi) ? __ldg(list + e_lo + (lane & 15)) : -1;
   for (int e0 = e_lo; e0 < e_hi && active; e0 += 16) {
-    // positions of this step's 16 list entries (lanes 16-31 repeat 0-15)
-    const int ee = e0 + (lane & 15);
-    const int jl = ee < e_hi ? __ldg(list + ee) : -1;
+    const int jl = jl_next;
+    const int en = e0 + 16 + (lane & 15);
+    jl_next = en < e_hi ? __ldg(list + en) : -1;
     const int jA = __shfl_sync(0xffffffffu, jl, gid), jB = __shfl_sync(0xffffffffu, jl, gid + 8);
     int jP[4];
 #pragma unroll
