@@ -221,12 +221,6 @@ const char* hs2_status_string(hs2_status status);
 /* Launch count of the library's kernels since load (all devices). */
 uint64_t hs2_kernel_launches(void);
 
-/* Self-test of the library's own exp2 (the polynomial that takes a quarter of
- * the full-attention softmax's exponentials off the MUFU unit): y[i] = 2^x[i]
- * for n device floats, 0 below -126.  Not part of the block; exposed so its
- * error bound can be checked. */
-hs2_status hs2_selftest_exp2(const float* x, float* y, int64_t n, void* stream);
-
 #ifdef __cplusplus
 }
 #endif

@@ -68,8 +68,6 @@ def _load(path: str = LIB_PATH):
     L.hs2_status_string.argtypes = [C.c_int]
     L.hs2_status_string.restype = C.c_char_p
     L.hs2_kernel_launches.restype = C.c_uint64
-    L.hs2_selftest_exp2.argtypes = [P, P, I64, P]
-    L.hs2_selftest_exp2.restype = C.c_int
     return L
 
 
@@ -78,8 +76,7 @@ _lib = _load()
 EXPORTED = ["hs2_bridge_kv", "hs2_full_attn_lse", "hs2_select_topk", "hs2_select_topk_noalloc",
             "hs2_sparse_attn",
             "hs2_block_prefill", "hs2_block_decode", "hs2_workspace_size",
-            "hs2_get_device_status", "hs2_status_string", "hs2_kernel_launches",
-            "hs2_selftest_exp2"]
+            "hs2_get_device_status", "hs2_status_string", "hs2_kernel_launches"]
 
 
 def _ptr(t, dtype, what, nullable=False):
@@ -188,10 +185,6 @@ def hs2_block_decode(seq_len, q_full, Kc, Vc, k_scale, v_scale, o_full, lse, idx
         _ptr(lse, F32, "lse"), _ptr(idx, I32T, "idx"), len(q_sparse), qs, os_, C.byref(shape),
         _ptr(workspace, U8, "workspace", True), nbytes, _stream(stream)), "hs2_block_decode")
 
-
-def hs2_selftest_exp2(x, y, stream=None):
-    _check(_lib.hs2_selftest_exp2(_ptr(x, F32, "x"), _ptr(y, F32, "y"), x.numel(),
-                                  _stream(stream)), "hs2_selftest_exp2")
 
 
 def hs2_get_device_status(stream=None) -> int:

@@ -282,44 +282,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// The coefficients of poly_exp2x2 (highest degree first), each duplicated
-// into both halves of a pair, then the rounding constant 1.5 * 2^23, its
-// negation and -1, so that FFMA2 can take them from the constant bank.
-static __constant__ __align__(16) float kPoly2[18] = {
-    1.3276374666020274e-3f, 1.3276374666020274e-3f, 9.67551488429308e-3f, 9.67551488429308e-3f,
-    5.550713464617729e-2f,  5.550713464617729e-2f,  2.4022120237350464e-1f, 2.4022120237350464e-1f,
-    6.931469440460205e-1f,  6.931469440460205e-1f,  1.0000001192092896f,   1.0000001192092896f,
-    12582912.f,             12582912.f,             -12582912.f,           -12582912.f,
-    -1.f,                   -1.f};
-
-__device__ __forceinline__ uint64_t kp2(int i) {
-  return reinterpret_cast<const uint64_t*>(kPoly2)[i];
-}
-
-// 2^x for a pair of arguments on the FMA pipe, for relieving the MUFU unit:
-// x = n + f with n the nearest integer (added to x as 1.5 * 2^23, whose ulp
-// is 1) and f in [-1/2, 1/2]; 2^f from a degree-5 polynomial whose
-// coefficients were fitted here for minimum relative error on [-1/2, 1/2]
-// (max 2.3e-7 in fp32 Horner form, about the error of ex2.approx); 2^n is
-// added to the exponent field.  The arithmetic runs on packed pairs (FFMA2).
-// Arguments below -126 give 0 (2^-126 is below every value that matters).
-__device__ __forceinline__ void poly_exp2x2(float a, float b, float& ya, float& yb) {
-  const uint64_t xc = f2(fmaxf(a, -126.f), fmaxf(b, -126.f));
-  const uint64_t t = f2_add(xc, kp2(6));
-  const uint64_t n = f2_add(t, kp2(7));
-  const uint64_t f = f2_fma(n, kp2(8), xc);
-  uint64_t p = f2_fma(kp2(0), f, kp2(1));
-#pragma unroll
-  for (int i = 2; i < 6; ++i) p = f2_fma(p, f, kp2(i));
-  float pa, pb, ta, tb;
-  f2_split(p, pa, pb);
-  f2_split(t, ta, tb);
-  ya = __int_as_float(__float_as_int(pa) + (__float_as_int(ta) << 23));
-  yb = __int_as_float(__float_as_int(pb) + (__float_as_int(tb) << 23));
-  ya = a < -126.f ? 0.f : ya;
-  yb = b < -126.f ? 0.f : yb;
-}
-
 __device__ __forceinline__ bool elect_one_lane() { return (threadIdx.x & 31) == 0; }
 
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }

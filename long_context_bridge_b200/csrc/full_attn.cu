@@ -20,8 +20,8 @@
 //   warps 2-5  softmax of tile A, warps 6-9 softmax of tile B: one thread per
 //              row (TMEM lane), base-2 online softmax with a lazily raised
 //              reference max (O is rescaled only when the row max grows by
-//              more than 2^8), a quarter of the exponentials as a polynomial on
-//              the FMA pipe, P as bf16 into TMEM, epilogue O / l and lse.
+//              more than 2^8), scale-and-shift and row sums on packed fp32
+//              pairs, P as bf16 into TMEM, epilogue O / l and lse.
 // TMEM: S_A [0,128), O_A [128,256), S_B [256,384), O_B [384,512).
 #include "common.cuh"
 #include "kernels.h"
@@ -238,12 +238,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int e = 0; e < 128; e += 2) {
         float a, b, p0, p1;
         f2_split(f2_fma(f2(x[e], x[e + 1]), sc2, nm2), a, b);
-        if ((e & 6) == 6) {  // one pair in four on the FMA pipe, the rest on MUFU
-          poly_exp2x2(a, b, p0, p1);
-        } else {
-          p0 = fast_exp2(a);
-          p1 = fast_exp2(b);
-        }
+        p0 = fast_exp2(a);
+        p1 = fast_exp2(b);
         sum2[(e >> 1) & 1] = f2_add(sum2[(e >> 1) & 1], f2(p0, p1));
         pk[e >> 1] = pack_bf16x2(p0, p1);
       }
@@ -311,16 +307,6 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-__global__ void poly_exp2_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
-  const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (2 * i + 1 < n) {
-    poly_exp2x2(x[2 * i], x[2 * i + 1], y[2 * i], y[2 * i + 1]);
-  } else if (2 * i < n) {
-    float unused;
-    poly_exp2x2(x[2 * i], 0.f, y[2 * i], unused);
-  }
-}
-
 template <int G>
 cudaError_t launch_g(const AttnArgs& a, cudaStream_t stream) {
   constexpr int QT = TILE / G;
@@ -345,13 +331,6 @@ cudaError_t launch_g(const AttnArgs& a, cudaStream_t stream) {
 }
 
 }  // namespace
-
-cudaError_t launch_poly_exp2(const float* x, float* y, int64_t n, cudaStream_t stream) {
-  if (n <= 0) return cudaSuccess;
-  poly_exp2_kernel<<<unsigned((n + 511) / 512), 256, 0, stream>>>(x, y, n);
-  count_launch();
-  return cudaGetLastError();
-}
 
 cudaError_t launch_full_attn(const AttnArgs& a, cudaStream_t stream) {
   switch (a.Hq / a.Hkv) {

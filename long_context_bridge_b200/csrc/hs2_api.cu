@@ -137,11 +137,6 @@ const char* hs2_status_string(hs2_status s) {
 
 uint64_t hs2_kernel_launches(void) { return g_launches.load(); }
 
-hs2_status hs2_selftest_exp2(const float* x, float* y, int64_t n, void* stream) {
-  HS2_NEED(n >= 0 && (n == 0 || (x && y)));
-  return cuda_status(launch_poly_exp2(x, y, n, static_cast<cudaStream_t>(stream)));
-}
-
 hs2_status hs2_get_device_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return HS2_ERR_CUDA;

@@ -52,8 +52,6 @@ struct AttnArgs {
   float scale;
 };
 cudaError_t launch_full_attn(const AttnArgs& a, cudaStream_t stream);
-// the FMA-pipe exp2 of the full-attention softmax, element-wise (self-test)
-cudaError_t launch_poly_exp2(const float* x, float* y, int64_t n, cudaStream_t stream);
 
 struct SelectArgs {
   const void* Q;

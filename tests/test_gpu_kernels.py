@@ -115,20 +115,3 @@ def test_select_matches_oracle(hs2, orc, T, Hq, Hkv, k, w):
     assert np.all(gk[~sel] == -1.0)
     if sel.any():
         np.testing.assert_allclose(gk[sel], kth_o[sel], rtol=1e-4)
-
-
-def test_poly_exp2_error_bound(hs2):
-    """The softmax's FMA-pipe exp2 against fp64 exp2: relative error within
-    3e-7 on the softmax's argument range, exact 0 below -126."""
-    import torch
-    x = torch.cat([torch.linspace(-126, 8, 2_000_001), torch.tensor([0.0, -0.5, 0.5, 1.0, -1.0]),
-                   torch.randn(100_000) * 3]).clamp(-126, 8).float().cuda()
-    y = torch.empty_like(x)
-    hs2.hs2_selftest_exp2(x, y)
-    ref = torch.exp2(x.double())
-    rel = ((y.double() - ref).abs() / ref).max().item()
-    assert rel < 3e-7, rel
-    z = torch.tensor([-127.0, -200.0, -float("inf")], device="cuda")
-    yz = torch.empty_like(z)
-    hs2.hs2_selftest_exp2(z, yz)
-    assert torch.all(yz == 0)
