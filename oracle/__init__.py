@@ -44,6 +44,9 @@ def lib():
         L.orc_e4m3_value.argtypes = [I32]
         L.orc_e4m3_value.restype = D
         L.orc_bf16_round.argtypes = [P, I64, P]
+        L.orc_e4m3_encode.argtypes = [C.c_float]
+        L.orc_e4m3_encode.restype = C.c_uint8
+        L.orc_quantize_rows.argtypes = [P, P, I64, I32, P, P, P]
         L.orc_threads.restype = I32
         L.orc_set_threads.argtypes = [I32]
         _lib = L
@@ -86,6 +89,29 @@ def bridge(H, W) -> np.ndarray:
     out = np.empty((T, N), np.uint16)
     lib().orc_bridge(_p(H), T, dm, _p(W), N, _p(out))
     return out
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """e4m3 codes of fp32 values: nearest, ties to the even code, saturated at
+    448, sign kept (f1's rounding rule)."""
+    L = lib()
+    x = np.asarray(x, dtype=np.float32).ravel()
+    return np.array([L.orc_e4m3_encode(C.c_float(float(v))) for v in x], dtype=np.uint8)
+
+
+def bridge_fp8(H, Wk, Wv, Hkv: int, d: int = 128):
+    """f1, bridge-only prefill into the FP8 cache: K/V = bf16(H W) as in S1,
+    then one fp32 scale per (token, KV head) and e4m3 codes of x / scale.
+    Returns (Kc, Vc uint8 [T, Hkv, d], scale float32 [T, Hkv], K, V bf16 bits)."""
+    K = bridge(H, Wk)
+    V = bridge(H, Wv)
+    T = K.shape[0]
+    rows = T * Hkv
+    Kc = np.empty((T, Hkv, d), np.uint8)
+    Vc = np.empty((T, Hkv, d), np.uint8)
+    S = np.empty((T, Hkv), np.float32)
+    lib().orc_quantize_rows(_p(K), _p(V), rows, d, _p(Kc), _p(Vc), _p(S))
+    return Kc, Vc, S, K.reshape(T, Hkv, d), V.reshape(T, Hkv, d)
 
 
 class KV:

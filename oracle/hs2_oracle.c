@@ -181,6 +181,59 @@ void orc_bridge(const uint16_t* H, int64_t T, int dm, const uint16_t* W, int N, 
 }
 
 /* ------------------------------------------------------------------------ */
+/* f1  bridge-only prefill into the FP8 cache                                 */
+/* [P5 KV Bridging] K/V of the cross-decoder come from the self-decoder's     */
+/* hidden states at prefill; [P2 tbl] the cache is FP8.  K = bf16(H W_k) and  */
+/* V = bf16(H W_v) exactly as in S1, then per (token t, KV head g) one fp32   */
+/* scale s = max(amax|K[t,g,:]|, amax|V[t,g,:]|) / 448 (1 when that amax is   */
+/* 0), and each code = e4m3(x / s): the quotient taken as an fp32 division,   */
+/* rounded to the nearest e4m3 value (ties to the even code), magnitudes      */
+/* above 448 saturated, the sign kept (a negative value that rounds to zero   */
+/* gives the negative zero code).                                             */
+/* ------------------------------------------------------------------------ */
+uint8_t orc_e4m3_encode(float x) {
+  const double a = fabs((double)x);
+  int code;
+  if (a >= 448.0) {
+    code = 0x7E;
+  } else {
+    int lo = 0; /* largest finite positive code whose value is <= a */
+    while (lo < 0x7E && orc_e4m3_value(lo + 1) <= a) ++lo;
+    if (orc_e4m3_value(lo) == a) {
+      code = lo;
+    } else {
+      const double dlo = a - orc_e4m3_value(lo), dhi = orc_e4m3_value(lo + 1) - a;
+      code = dlo < dhi ? lo : dhi < dlo ? lo + 1 : (lo % 2 == 0 ? lo : lo + 1);
+    }
+  }
+  return (uint8_t)(code | (signbit(x) ? 0x80 : 0));
+}
+
+/* rows: K and V bf16 bits [rows, d] (a row = one (token, KV head)) -> codes
+ * [rows, d] and scales [rows] */
+void orc_quantize_rows(const uint16_t* K, const uint16_t* V, int64_t rows, int d, uint8_t* Kc,
+                       uint8_t* Vc, float* scale) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r) {
+    float amax = 0.0f;
+    for (int e = 0; e < d; ++e) {
+      const float k = fabsf((float)bf16_value(K[r * d + e]));
+      const float v = fabsf((float)bf16_value(V[r * d + e]));
+      if (k > amax) amax = k;
+      if (v > amax) amax = v;
+    }
+    const float s = amax > 0.0f ? amax / 448.0f : 1.0f;
+    scale[r] = s;
+    for (int e = 0; e < d; ++e) {
+      const float qk = (float)bf16_value(K[r * d + e]) / s;
+      const float qv = (float)bf16_value(V[r * d + e]) / s;
+      Kc[r * d + e] = orc_e4m3_encode(qk);
+      Vc[r * d + e] = orc_e4m3_encode(qv);
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------ */
 /* S2  causal GQA full attention with log-sum-exp                             */
 /* [P5 Cross-Decoder]: each block starts with one full-attention layer that   */
 /* looks at every earlier token; [P2 原理] its complete attention scores pick */

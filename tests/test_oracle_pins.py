@@ -74,6 +74,50 @@ def test_synth_e4m3_quantiser_matches_torch_cast():
     assert np.all((ours[zero] & 0x7F) == 0)
 
 
+def test_oracle_e4m3_encoder_matches_torch_cast(orc):
+    # f1's rounding rule (nearest, ties to the even code, saturation, sign of
+    # zero kept) against torch's float8_e4m3fn cast of values clamped to 448
+    tab = orc.e4m3_table()
+    pos = tab[:0x7F]
+    mids = ((pos[:-1] + pos[1:]) / 2).astype(np.float32)       # exact ties
+    x = np.concatenate([np.linspace(-460, 460, 20001), RNG.standard_normal(20000) * 3,
+                        RNG.standard_normal(20000) * 1e-2, pos, -pos, mids, -mids,
+                        [0.0, -0.0, 1e-30, -1e-30, 449.0, -1e9]]).astype(np.float32)
+    ours = orc.e4m3_encode(x)
+    ref = torch.from_numpy(np.clip(x, -448, 448)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(ours, ref)
+
+
+def test_bridge_fp8_is_nearest_code_of_scaled_row(orc):
+    # brute force on a small case: the scale is the row pair's amax / 448 in
+    # fp32 and each code is the nearest e4m3 value of x / scale (fp32 quotient)
+    T, dm, Hkv = 48, 128, 2
+    H = rand_bf16((T, dm))
+    Wk, Wv = rand_bf16((dm, Hkv * 128), 1 / 16), rand_bf16((dm, Hkv * 128), 1 / 16)
+    H[3] = 0                                               # an all-zero row: scale 1
+    Kc, Vc, S, K, V = orc.bridge_fp8(H, Wk, Wv, Hkv)
+    assert np.array_equal(K.reshape(T, -1), orc.bridge(H, Wk))
+    kf = synth.bf16_bits_to_f32(K)
+    vf = synth.bf16_bits_to_f32(V)
+    amax = np.maximum(np.abs(kf).max(axis=2), np.abs(vf).max(axis=2)).astype(np.float32)
+    want_s = np.where(amax > 0, amax / np.float32(448), np.float32(1)).astype(np.float32)
+    assert np.array_equal(S, want_s) and np.all(S[3] == 1)
+    tab = orc.e4m3_table()
+    vals = tab[:0x7F]
+    for codes, x in ((Kc, kf), (Vc, vf)):
+        q = (x / S[:, :, None]).astype(np.float32).astype(np.float64)
+        dist = np.abs(np.abs(q)[..., None] - vals)            # [T, Hkv, d, 127]
+        best = dist.min(axis=-1)
+        mag = codes & 0x7F
+        assert np.all(np.abs(np.abs(q) - vals[mag]) == best)  # a nearest value
+        tie = (dist == best[..., None]).sum(axis=-1) > 1
+        assert np.all(mag[tie] % 2 == 0)                      # ties to the even code
+        assert np.array_equal(codes >> 7, np.signbit(q).astype(np.uint8))
+    # the largest magnitude of each row pair maps to 448
+    top = np.maximum((Kc & 0x7F).max(axis=2), (Vc & 0x7F).max(axis=2))
+    assert np.all(top[amax > 0] == 0x7E)
+
+
 # --------------------------------------------------------------------------
 # S1 bridge
 # --------------------------------------------------------------------------
