@@ -187,6 +187,47 @@ class OracleSample:
 # ---------------------------------------------------------------------------
 # decode step at 1M context (8 sequences, FP8 cache)
 # ---------------------------------------------------------------------------
+def bench_bridge_fp8(hs2, dev, steps, warmup):
+    """Bridge-only prefill into the FP8 cache at 1M tokens (the C3 block's
+    bridge shapes: d_model 2048, 4 KV heads), against the tensor roofline."""
+    cfg = synth.CONFIGS["C3"]
+    T, Hkv, dm = 1 << 20, cfg.n_kv_heads, cfg.d_model
+    H, Wk, Wv = synth.bridge_inputs_torch(cfg, T=T, device=dev)
+    Kc = torch.empty(T, Hkv, 128, dtype=torch.uint8, device=dev)
+    Vc = torch.empty_like(Kc)
+    S = torch.empty(T, Hkv, dtype=torch.float32, device=dev)
+    shape = hs2.Shape.make(T, Hkv, Hkv)
+    for _ in range(max(warmup, 3)):
+        hs2.hs2_bridge_kv_fp8(H, Wk, Wv, Kc, Vc, S, shape)
+    n0 = hs2.hs2_kernel_launches()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        hs2.hs2_bridge_kv_fp8(H, Wk, Wv, Kc, Vc, S, shape)  # H (4 GiB) is larger than L2
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    flop = 2.0 * T * dm * 2 * Hkv * 128
+    # a few ms timed on its own: the burst bf16 figure is the denominator
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            tfl, src = float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        tfl, src = 1590.0, "fallback"
+    tf = flop / (ms / 1e3) / 1e12
+    out = {"metric": "bridge-only prefill into the FP8 cache tokens/s @1M", "value": T / (ms / 1e3),
+           "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
+           "config": {"workload": "bridge T=1048576 d_model 2048 -> e4m3 K/V cache, 4 KV heads",
+                      "l2": "inputs larger than L2 (H is 4 GiB)"},
+           "gpu_launches_per_step": (hs2.hs2_kernel_launches() - n0) / steps,
+           "roofline": {"bound": "tensor", "achieved": tf, "peak": tfl, "unit": "TFLOP/s",
+                        "frac": tf / tfl, "flop": flop, "peak_source": f"{src} (bf16 burst)"}}
+    del H, Wk, Wv, Kc, Vc, S
+    torch.cuda.empty_cache()
+    return out
+
+
 def bench_decode(hs2, dev, steps, warmup):
     cfg = synth.CONFIGS["C5"]
     B, N, Hq, Hkv = cfg.batch, cfg.T, cfg.n_q_heads, cfg.n_kv_heads
@@ -486,6 +527,7 @@ def main():
         del inp, K, V, O, Os, lse, idx, ws
         torch.cuda.empty_cache()
         dec = bench_decode(hs2, dev, args.steps, args.warmup)
+    f1 = bench_bridge_fp8(hs2, dev, args.steps, args.warmup) if not args.no_decode else None
     cpu = None
     if not args.no_cpu and world == 1:
         cpu = OracleSample(cfg).run(320, seed=5)
@@ -494,7 +536,7 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": config, "clocks": clk.summary(), "e2e": e2e,
             "gpu_launches": int(n_launch), "roofline": roof, "kernels": per_kernel,
-            "decode": dec, "cpu_baseline": cpu}
+            "decode": dec, "bridge_fp8": f1, "cpu_baseline": cpu}
     print(json.dumps(line), flush=True)
     if pg:
         torch.distributed.destroy_process_group()

@@ -97,6 +97,24 @@ hs2_status hs2_bridge_kv(const hs2_bf16* H, int32_t d_model, const hs2_bf16* W_k
                          const hs2_shape* shape, void* stream);
 
 /*
+ * Bridge-only prefill into the FP8 cache.  The javabetter.cn explainer's KV
+ * Bridging paragraph (at prefill the cross-decoder's K/V come from the
+ * self-decoder's hidden states) and the FP8 KV cache of the zgeo.com.cn
+ * comparison table: step S1 fused with the cache's quantisation.
+ *   K, V = bf16(H W_k), bf16(H W_v)            exactly as hs2_bridge_kv, then
+ *   scale[t, g] = max(amax|K[t,g,:]|, amax|V[t,g,:]|) / 448   (fp32; 1 if 0)
+ *   Kc[t, g, e] = e4m3(K[t, g, e] / scale[t, g])  (fp32 quotient, nearest,
+ *                 ties to the even code, saturated at 448), likewise Vc.
+ * H, W_k, W_v as in hs2_bridge_kv.  Kc, Vc [T, n_kv_heads, 128] e4m3 codes
+ * and scale [T, n_kv_heads] fp32: the layout of one sequence of the decode
+ * cache (hs2_block_decode reads scale as k_scale and v_scale).  Pointers
+ * 16-byte aligned; d_model a positive multiple of 64.  No workspace.
+ */
+hs2_status hs2_bridge_kv_fp8(const hs2_bf16* H, int32_t d_model, const hs2_bf16* W_k,
+                             const hs2_bf16* W_v, hs2_fp8e4m3* Kc, hs2_fp8e4m3* Vc,
+                             float* scale, const hs2_shape* shape, void* stream);
+
+/*
  * Causal GQA full attention with per-row log-sum-exp (step S2).  The block's
  * full-attention layer (Cross-Decoder paragraph of the javabetter.cn
  * explainer); its complete attention scores later rank tokens (section

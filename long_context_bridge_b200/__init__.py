@@ -49,6 +49,7 @@ def _load(path: str = LIB_PATH):
     PP = C.POINTER(C.c_void_p)
     sigs = {
         "hs2_bridge_kv": [P, I32, P, P, P, P, SP, P],
+        "hs2_bridge_kv_fp8": [P, I32, P, P, P, P, P, SP, P],
         "hs2_full_attn_lse": [P, P, P, P, P, SP, P],
         "hs2_select_topk": [P, P, P, P, P, SP, P, SZ, P],
         "hs2_select_topk_noalloc": [P, P, P, P, P, SP, P],
@@ -73,7 +74,7 @@ def _load(path: str = LIB_PATH):
 
 _lib = _load()
 
-EXPORTED = ["hs2_bridge_kv", "hs2_full_attn_lse", "hs2_select_topk", "hs2_select_topk_noalloc",
+EXPORTED = ["hs2_bridge_kv", "hs2_bridge_kv_fp8", "hs2_full_attn_lse", "hs2_select_topk", "hs2_select_topk_noalloc",
             "hs2_sparse_attn",
             "hs2_block_prefill", "hs2_block_decode", "hs2_workspace_size",
             "hs2_get_device_status", "hs2_status_string", "hs2_kernel_launches"]
@@ -120,6 +121,13 @@ def hs2_bridge_kv(H, W_k, W_v, K, V, shape: Shape, stream=None):
     _check(_lib.hs2_bridge_kv(_ptr(H, BF16, "H"), H.shape[-1], _ptr(W_k, BF16, "W_k"),
                               _ptr(W_v, BF16, "W_v"), _ptr(K, BF16, "K"), _ptr(V, BF16, "V"),
                               C.byref(shape), _stream(stream)), "hs2_bridge_kv")
+
+
+def hs2_bridge_kv_fp8(H, W_k, W_v, Kc, Vc, scale, shape: Shape, stream=None):
+    _check(_lib.hs2_bridge_kv_fp8(_ptr(H, BF16, "H"), H.shape[-1], _ptr(W_k, BF16, "W_k"),
+                                  _ptr(W_v, BF16, "W_v"), _ptr(Kc, U8, "Kc"), _ptr(Vc, U8, "Vc"),
+                                  _ptr(scale, F32, "scale"), C.byref(shape), _stream(stream)),
+           "hs2_bridge_kv_fp8")
 
 
 def hs2_full_attn_lse(Q, K, V, O, lse, shape: Shape, stream=None):

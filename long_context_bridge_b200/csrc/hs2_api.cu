@@ -181,6 +181,18 @@ hs2_status hs2_bridge_kv(const hs2_bf16* H, int32_t d_model, const hs2_bf16* W_k
   return cuda_status(launch_bridge(a, static_cast<cudaStream_t>(stream)));
 }
 
+hs2_status hs2_bridge_kv_fp8(const hs2_bf16* H, int32_t d_model, const hs2_bf16* W_k,
+                             const hs2_bf16* W_v, hs2_fp8e4m3* Kc, hs2_fp8e4m3* Vc, float* scale,
+                             const hs2_shape* s, void* stream) {
+  HS2_TRY(check_shape(s, false));
+  HS2_NEED(H && W_k && W_v && Kc && Vc && scale);
+  HS2_NEED(aligned16(H) && aligned16(W_k) && aligned16(W_v) && aligned16(Kc) && aligned16(Vc) &&
+           aligned16(scale));
+  HS2_NEED(d_model > 0 && d_model % 64 == 0);
+  BridgeFp8Args a{H, W_k, W_v, Kc, Vc, scale, s->T, d_model, s->n_kv_heads * 128};
+  return cuda_status(launch_bridge_fp8(a, static_cast<cudaStream_t>(stream)));
+}
+
 hs2_status hs2_full_attn_lse(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V,
                              hs2_bf16* O, float* lse, const hs2_shape* s, void* stream) {
   HS2_TRY(check_shape(s, false));

@@ -41,6 +41,19 @@ struct BridgeArgs {
 };
 cudaError_t launch_bridge(const BridgeArgs& a, cudaStream_t stream);
 
+struct BridgeFp8Args {
+  const void* H;
+  const void* Wk;
+  const void* Wv;
+  uint8_t* Kc;   // [T, Hkv, 128] e4m3 codes
+  uint8_t* Vc;
+  float* scale;  // [T, Hkv]
+  int64_t T;
+  int dm;
+  int Nkv;       // n_kv_heads * 128
+};
+cudaError_t launch_bridge_fp8(const BridgeFp8Args& a, cudaStream_t stream);
+
 struct AttnArgs {
   const void* Q;
   const void* K;

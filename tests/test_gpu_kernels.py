@@ -51,6 +51,48 @@ def test_bridge_matches_oracle(hs2, orc, T, dm, Hkv):
         assert np.mean(g == want) > 0.99
 
 
+@pytest.mark.parametrize("T,dm,Hkv", [(300, 256, 2), (1000, 2048, 4), (130, 128, 1)])
+def test_bridge_fp8_matches_oracle(hs2, orc, T, dm, Hkv):
+    """Bridge-only prefill into the FP8 cache.  Scales and codes are the
+    oracle's bit for bit on every (token, KV head) whose bf16 K/V cannot differ:
+    no element's exact product lies within the fp32 summation bound of a bf16
+    rounding boundary.  Elsewhere (rare) the decoded values agree to one e4m3
+    step.  A zero code counts with either sign."""
+    import torch
+    H = rand_bf16((T, dm))
+    Wk, Wv = rand_bf16((dm, Hkv * 128), dm ** -0.5), rand_bf16((dm, Hkv * 128), dm ** -0.5)
+    H[min(5, T - 1)] = 0                                   # an all-zero row: scale 1
+    Kc = torch.empty(T, Hkv, 128, dtype=torch.uint8, device="cuda")
+    Vc = torch.empty_like(Kc)
+    S = torch.empty(T, Hkv, dtype=torch.float32, device="cuda")
+    shape = hs2.Shape.make(T, Hkv, Hkv)
+    hs2.hs2_bridge_kv_fp8(dev_bf16(H), dev_bf16(Wk), dev_bf16(Wv), Kc, Vc, S, shape)
+    assert hs2.hs2_get_device_status() == hs2.OK
+    Kc_o, Vc_o, S_o, K_o, V_o = orc.bridge_fp8(H, Wk, Wv, Hkv)
+    hf = synth.bf16_bits_to_f32(H).astype(np.float64)
+    ambiguous = np.zeros((T, Hkv), bool)
+    for W, Xo in ((Wk, K_o), (Wv, V_o)):
+        wf = synth.bf16_bits_to_f32(W).astype(np.float64)
+        exact = (hf @ wf).reshape(T, Hkv, 128)
+        bound = (dm * 2.0 ** -24 * (np.abs(hf) @ np.abs(wf))).reshape(T, Hkv, 128)
+        xo = synth.bf16_bits_to_f32(Xo).astype(np.float64)
+        half_ulp = np.spacing(np.abs(xo).astype(np.float32)).astype(np.float64) * 2.0 ** 15
+        ambiguous |= (half_ulp - np.abs(exact - xo) <= bound).any(axis=2)
+    assert ambiguous.mean() < 0.05
+    Sg, Kg, Vg = S.cpu().numpy(), Kc.cpu().numpy(), Vc.cpu().numpy()
+    ok = ~ambiguous
+    assert np.array_equal(Sg[ok], S_o[ok])
+    for g_codes, o_codes in ((Kg, Kc_o), (Vg, Vc_o)):
+        same = (g_codes == o_codes) | (((g_codes | o_codes) & 0x7F) == 0)
+        assert same[ok].all()
+        tab = orc.e4m3_table()
+        dg = tab[g_codes] * Sg[..., None]
+        do = tab[o_codes] * S_o[..., None]
+        step = np.maximum(np.abs(do), np.abs(dg)) * 2.0 ** -3 + S_o[..., None] * 2.0 ** -9
+        assert np.all(np.abs(dg - do) <= step)
+    assert np.all(Sg[min(5, T - 1)] == 1.0)
+
+
 @pytest.mark.parametrize("T,Hq,Hkv", [(2048, 4, 1), (1000, 16, 2), (333, 2, 1), (700, 16, 1),
                                       (130, 4, 4)])
 def test_full_attn_matches_oracle(hs2, orc, T, Hq, Hkv):
