@@ -306,6 +306,10 @@ def kernels_once(dev):
     idx = torch.empty(T, Hkv, 1152, dtype=torch.int32, device=dev)
     hs2.hs2_select_topk(Q, K, lse, idx, None, sh, ws)
     hs2.hs2_sparse_attn(g(synth.TID_QS0, T * Hq * 128).view(T, Hq, 128), K, V, idx, O, None, sh)
+    K8 = torch.empty(T, Hkv, 128, dtype=torch.uint8, device=dev)
+    hs2.hs2_bridge_kv_fp8(H, Wk, Wv, K8, torch.empty_like(K8),
+                          torch.empty(T, Hkv, dtype=torch.float32, device=dev),
+                          hs2.Shape.make(T, Hkv, Hkv))
     dcfg = synth.CONFIGS["C5"]
     N, B = 262144, dcfg.batch
     Kc, Vc, S = synth.decode_cache_torch(dcfg, N, device=dev)
@@ -319,8 +323,8 @@ def kernels_once(dev):
                          torch.empty(B, Hkv, 1152, dtype=torch.int32, device=dev), q[1:], os_, shd, wsd)
     torch.cuda.synchronize()
     assert hs2.hs2_get_device_status() == hs2.OK
-    print("kernels-once: 32K block (bridge, full attention, selection, one sparse layer) and "
-          "one decode step of 8 x 262144 tokens", flush=True)
+    print("kernels-once: 32K block (bridge, full attention, selection, one sparse layer, "
+          "bridge into the FP8 cache) and one decode step of 8 x 262144 tokens", flush=True)
 
 
 # ---------------------------------------------------------------------------

@@ -53,11 +53,13 @@ def test_bridge_matches_oracle(hs2, orc, T, dm, Hkv):
 
 @pytest.mark.parametrize("T,dm,Hkv", [(300, 256, 2), (1000, 2048, 4), (130, 128, 1)])
 def test_bridge_fp8_matches_oracle(hs2, orc, T, dm, Hkv):
-    """Bridge-only prefill into the FP8 cache.  Scales and codes are the
-    oracle's bit for bit on every (token, KV head) whose bf16 K/V cannot differ:
-    no element's exact product lies within the fp32 summation bound of a bf16
-    rounding boundary.  Elsewhere (rare) the decoded values agree to one e4m3
-    step.  A zero code counts with either sign."""
+    """Bridge-only prefill into the FP8 cache against the oracle.  An element
+    is ambiguous when its exact product lies within the fp32 summation bound
+    dm * 2^-24 * sum|h||w| of a bf16 rounding boundary: there the GPU's bf16
+    K/V may differ from the oracle's by one ulp.  Scales are bit-exact wherever
+    the row pair's largest element is unambiguous; codes are bit-exact (a zero
+    code with either sign) except at ambiguous elements, which stay within one
+    e4m3 step, as do all decoded values."""
     import torch
     H = rand_bf16((T, dm))
     Wk, Wv = rand_bf16((dm, Hkv * 128), dm ** -0.5), rand_bf16((dm, Hkv * 128), dm ** -0.5)
@@ -70,22 +72,28 @@ def test_bridge_fp8_matches_oracle(hs2, orc, T, dm, Hkv):
     assert hs2.hs2_get_device_status() == hs2.OK
     Kc_o, Vc_o, S_o, K_o, V_o = orc.bridge_fp8(H, Wk, Wv, Hkv)
     hf = synth.bf16_bits_to_f32(H).astype(np.float64)
-    ambiguous = np.zeros((T, Hkv), bool)
+    amb, mag = [], []
     for W, Xo in ((Wk, K_o), (Wv, V_o)):
         wf = synth.bf16_bits_to_f32(W).astype(np.float64)
         exact = (hf @ wf).reshape(T, Hkv, 128)
         bound = (dm * 2.0 ** -24 * (np.abs(hf) @ np.abs(wf))).reshape(T, Hkv, 128)
         xo = synth.bf16_bits_to_f32(Xo).astype(np.float64)
         half_ulp = np.spacing(np.abs(xo).astype(np.float32)).astype(np.float64) * 2.0 ** 15
-        ambiguous |= (half_ulp - np.abs(exact - xo) <= bound).any(axis=2)
-    assert ambiguous.mean() < 0.05
+        amb.append(half_ulp - np.abs(exact - xo) <= bound)
+        mag.append(np.abs(xo))
+    amax = np.maximum(mag[0].max(axis=2), mag[1].max(axis=2))
+    top_amb = ((mag[0] == amax[..., None]) & amb[0]).any(axis=2) | \
+              ((mag[1] == amax[..., None]) & amb[1]).any(axis=2)
     Sg, Kg, Vg = S.cpu().numpy(), Kc.cpu().numpy(), Vc.cpu().numpy()
-    ok = ~ambiguous
-    assert np.array_equal(Sg[ok], S_o[ok])
-    for g_codes, o_codes in ((Kg, Kc_o), (Vg, Vc_o)):
+    assert np.array_equal(Sg[~top_amb], S_o[~top_amb])
+    same_s = Sg == S_o
+    assert same_s.mean() > 0.99
+    tab = orc.e4m3_table()
+    for g_codes, o_codes, a in ((Kg, Kc_o, amb[0]), (Vg, Vc_o, amb[1])):
         same = (g_codes == o_codes) | (((g_codes | o_codes) & 0x7F) == 0)
-        assert same[ok].all()
-        tab = orc.e4m3_table()
+        assert same[same_s & ~a.any(axis=2)].all()            # rows with no ambiguity
+        assert not (~same & ~a & same_s[..., None]).any()     # elsewhere only ambiguous ones
+        assert same.mean() > 0.99                             # and those seldom differ
         dg = tab[g_codes] * Sg[..., None]
         do = tab[o_codes] * S_o[..., None]
         step = np.maximum(np.abs(do), np.abs(dg)) * 2.0 ** -3 + S_o[..., None] * 2.0 ** -9
