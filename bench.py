@@ -526,6 +526,24 @@ def main():
                          ("TFLOP/s" if b == "tensor" else "GB/s"):
                              (a / s / 1e12) if b == "tensor" else (a / s / 1e9),
                          "frac": ((a / s / 1e12) / tfl) if b == "tensor" else ((a / s / 1e9) / hbm)}
+    # f4, a separate labelled figure: the same three sparse layers in one pass
+    # over the gathered rows (valid only when all layers' queries exist up
+    # front, so it is not part of the step above)
+    sp = work["sparse_attn"][1]
+    torch.cuda.synchronize()
+    fa, fb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    hs2.hs2_sparse_attn_layers(inp["Qs"], K, V, idx, Os, None, shape)
+    fa.record()
+    for _ in range(args.steps):
+        hs2.hs2_sparse_attn_layers(inp["Qs"], K, V, idx, Os, None, shape)
+    fb.record()
+    torch.cuda.synchronize()
+    fused_ms = fa.elapsed_time(fb) / args.steps
+    fused = {"metric": "3 sparse layers in one pass over the gathered rows, ms @128K",
+             "value": fused_ms, "unit": "ms", "separate_ms": kern_ms["sparse_attn"] * cfg.n_sparse,
+             "GB/s": cfg.n_sparse * sp / (fused_ms / 1e3) / 1e9,
+             "note": "algorithmic bytes of the three separate layers over the fused time; "
+                     "not in the step (a model's layer l+1 queries depend on layer l)"}
     dec = None
     if not args.no_decode:
         del inp, K, V, O, Os, lse, idx, ws
@@ -540,7 +558,7 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": config, "clocks": clk.summary(), "e2e": e2e,
             "gpu_launches": int(n_launch), "roofline": roof, "kernels": per_kernel,
-            "decode": dec, "bridge_fp8": f1, "cpu_baseline": cpu}
+            "decode": dec, "bridge_fp8": f1, "sparse_layers_fused": fused, "cpu_baseline": cpu}
     print(json.dumps(line), flush=True)
     if pg:
         torch.distributed.destroy_process_group()

@@ -188,6 +188,22 @@ hs2_status hs2_sparse_attn(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16*
                            const hs2_shape* shape, void* stream);
 
 /*
+ * Several sparse layers in one pass over the gathered rows (variant of
+ * hs2_sparse_attn; no counterpart on the pages).  Layer l computes exactly
+ * what hs2_sparse_attn(Q[l], K, V, idx, O[l], lse[l]) computes, but every
+ * gathered K/V row serves all the layers' queries (up to three per pass when
+ * G <= 8, one otherwise).  Valid only when every layer's queries exist before
+ * the call: in a model's forward pass layer l+1's queries depend on layer l's
+ * output, so the block (hs2_block_prefill) runs the layers one by one.
+ * Q, O: HOST arrays of n_layers DEVICE pointers; lse: NULL or a HOST array of
+ * n_layers nullable DEVICE pointers.  No workspace.
+ */
+hs2_status hs2_sparse_attn_layers(int32_t n_layers, const hs2_bf16* const* Q,
+                                  const hs2_bf16* K, const hs2_bf16* V, const int32_t* idx,
+                                  hs2_bf16* const* O, float* const* lse,
+                                  const hs2_shape* shape, void* stream);
+
+/*
  * The whole block at prefill: bridge (if H != NULL), full attention, selection
  * and n_sparse sparse layers sharing K/V and idx (all of the above, in order,
  * on `stream`).  Q_sparse and O_sparse are HOST arrays of n_sparse DEVICE

@@ -54,6 +54,7 @@ def _load(path: str = LIB_PATH):
         "hs2_select_topk": [P, P, P, P, P, SP, P, SZ, P],
         "hs2_select_topk_noalloc": [P, P, P, P, P, SP, P],
         "hs2_sparse_attn": [P, P, P, P, P, P, SP, P],
+        "hs2_sparse_attn_layers": [I32, PP, P, P, P, PP, PP, SP, P],
         "hs2_block_prefill": [P, I32, P, P, P, P, P, P, P, P, I32, PP, PP, SP, P, SZ, P],
         "hs2_block_decode": [I32, C.POINTER(C.c_int64), P, P, P, P, P, P, P, P, I32, PP, PP, SP,
                              P, SZ, P],
@@ -75,7 +76,7 @@ def _load(path: str = LIB_PATH):
 _lib = _load()
 
 EXPORTED = ["hs2_bridge_kv", "hs2_bridge_kv_fp8", "hs2_full_attn_lse", "hs2_select_topk", "hs2_select_topk_noalloc",
-            "hs2_sparse_attn",
+            "hs2_sparse_attn", "hs2_sparse_attn_layers",
             "hs2_block_prefill", "hs2_block_decode", "hs2_workspace_size",
             "hs2_get_device_status", "hs2_status_string", "hs2_kernel_launches"]
 
@@ -165,6 +166,17 @@ def _ptr_array(ts, dtype, what):
     for i, t in enumerate(ts):
         arr[i] = _ptr(t, dtype, f"{what}[{i}]").value
     return C.cast(arr, C.POINTER(C.c_void_p)), arr
+
+
+def hs2_sparse_attn_layers(Qs, K, V, idx, Os, lses, shape: Shape, stream=None):
+    qs, _keep_q = _ptr_array(Qs, BF16, "Q")
+    os_, _keep_o = _ptr_array(Os, BF16, "O")
+    ls = None
+    if lses is not None:
+        ls = (C.c_void_p * max(1, len(lses)))(*[_ptr(t, F32, "lse", True) for t in lses])
+    _check(_lib.hs2_sparse_attn_layers(len(Qs), qs, _ptr(K, BF16, "K"), _ptr(V, BF16, "V"),
+                                       _ptr(idx, I32T, "idx"), os_, ls, C.byref(shape),
+                                       _stream(stream)), "hs2_sparse_attn_layers")
 
 
 def hs2_block_prefill(H, W_k, W_v, K, V, Q_full, O_full, lse, idx, Q_sparse, O_sparse,

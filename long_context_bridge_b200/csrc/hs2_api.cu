@@ -3,6 +3,7 @@
 // in the kernels of this library; nothing here computes results on the host.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 #include <set>
@@ -249,6 +250,49 @@ hs2_status hs2_sparse_attn(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16*
   a.scale = s->scale;
   a.kw = s->k_global + s->window;
   return cuda_status(launch_sparse(a, static_cast<cudaStream_t>(stream)));
+}
+
+hs2_status hs2_sparse_attn_layers(int32_t n_layers, const hs2_bf16* const* Q,
+                                  const hs2_bf16* K, const hs2_bf16* V, const int32_t* idx,
+                                  hs2_bf16* const* O, float* const* lse, const hs2_shape* s,
+                                  void* stream) {
+  HS2_TRY(check_shape(s, true));
+  HS2_NEED(n_layers >= 1 && Q && O && K && V && idx);
+  HS2_NEED(aligned16(K) && aligned16(V) && aligned16(idx));
+  for (int l = 0; l < n_layers; ++l) {
+    HS2_NEED(Q[l] && O[l] && aligned16(Q[l]) && aligned16(O[l]));
+    HS2_NEED(lse == nullptr || lse[l] == nullptr || aligned16(lse[l]));
+  }
+  SparseArgs a{};
+  a.K = K;
+  a.V = V;
+  a.idx = idx;
+  a.T = s->T;
+  a.Hq = s->n_q_heads;
+  a.Hkv = s->n_kv_heads;
+  a.scale = s->scale;
+  a.kw = s->k_global + s->window;
+  const int per = max_fused_layers(s->n_q_heads / s->n_kv_heads);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (int l0 = 0; l0 < n_layers;) {
+    const int L = std::min(per, n_layers - l0);
+    if (L == 1) {
+      a.Q = Q[l0];
+      a.O = O[l0];
+      a.lse = lse ? lse[l0] : nullptr;
+      HS2_TRY(cuda_status(launch_sparse(a, st)));
+    } else {
+      SparseLayers lp{};
+      for (int i = 0; i < L; ++i) {
+        lp.Q[i] = Q[l0 + i];
+        lp.O[i] = O[l0 + i];
+        lp.lse[i] = lse ? lse[l0 + i] : nullptr;
+      }
+      HS2_TRY(cuda_status(launch_sparse_fused(a, lp, L, st)));
+    }
+    l0 += L;
+  }
+  return HS2_OK;
 }
 
 hs2_status hs2_block_prefill(const hs2_bf16* H, int32_t d_model, const hs2_bf16* W_k,

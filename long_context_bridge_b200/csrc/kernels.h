@@ -105,6 +105,18 @@ struct SparseArgs {
 };
 cudaError_t launch_sparse(const SparseArgs& a, cudaStream_t stream);
 
+// Fused sparse layers (bf16 K/V): the Q, O and (nullable) lse of each layer
+constexpr int kMaxFusedLayers = 3;
+struct SparseLayers {
+  const void* Q[kMaxFusedLayers];  // bf16 [T, Hq, 128]
+  void* O[kMaxFusedLayers];        // bf16 [T, Hq, 128]
+  float* lse[kMaxFusedLayers];     // [T, Hq] or null
+};
+// most layers one fused launch takes for G query heads per KV head (1 = none)
+int max_fused_layers(int G);
+cudaError_t launch_sparse_fused(const SparseArgs& a, const SparseLayers& lp, int L,
+                                cudaStream_t stream);
+
 struct DecodeArgs {
   int B;
   const int64_t* seq_len_host;

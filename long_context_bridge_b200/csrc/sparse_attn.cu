@@ -98,15 +98,21 @@ __device__ __forceinline__ float from16(uint16_t v) {
 // G query heads of one KV head; FP8: e4m3 cache with per-(token, head) scales;
 // WPR warps share one (row, KV head) pair, splitting its list; with CS > 1
 // the CS CTAs of a thread-block cluster share it (CS * WPR parts) and combine
-// their partial softmax states through distributed shared memory.
-template <int G, bool FP8, int WPR, int CS = 1>
+// their partial softmax states through distributed shared memory.  L > 1
+// fuses L sparse layers: the pair's L * G heads (layer e / G, head e % G of
+// pair head e) share every gathered K/V row; their Q, O and lse come from
+// `lp`.
+template <int G, bool FP8, int WPR, int CS = 1, int L = 1>
 __global__ void __launch_bounds__(128)
     sparse_mma_kernel(const __nv_bfloat16* __restrict__ Q, const void* __restrict__ Kp,
                       const void* __restrict__ Vp, const float* __restrict__ ks,
                       const float* __restrict__ vs, const int32_t* __restrict__ idx,
                       __nv_bfloat16* __restrict__ O, float* __restrict__ lse, int64_t rows,
-                      int Hkv, int kw, float scale_log2, int64_t cache_T) {
-  constexpr int NT = G > 8 ? G / 8 : 1;  // 8-head n-tiles
+                      int Hkv, int kw, float scale_log2, int64_t cache_T,
+                      const __grid_constant__ SparseLayers lp) {
+  constexpr int HE = L * G;                       // heads of a pair
+  constexpr int NT = (HE + 7) / 8;                // 8-head n-tiles
+  static_assert(L == 1 || (WPR == 1 && !FP8), "layers are fused on the prefill path only");
   constexpr int NW = 4;                  // warps per CTA
   constexpr int PAIRS = NW / WPR;        // (row, KV head) pairs per CTA
   constexpr bool F16 = FP8;              // FP8 path: f16 MMA; bf16 path: bf16 MMA
@@ -139,9 +145,11 @@ __global__ void __launch_bounds__(128)
   uint32_t qf[NT][8][2];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
-    const int hh = nt * 8 + gid;
-    const bool real = hh < G && active;
-    const uint4* qr = reinterpret_cast<const uint4*>(Q + (r * Hq + g * G + (real ? hh : 0)) * 128 +
+    const int hh = nt * 8 + gid;  // pair head
+    const bool real = hh < HE && active;
+    const __nv_bfloat16* Qh =
+        L == 1 ? Q : reinterpret_cast<const __nv_bfloat16*>(lp.Q[real ? hh / G : 0]);
+    const uint4* qr = reinterpret_cast<const uint4*>(Qh + (r * Hq + g * G + (real ? hh % G : 0)) * 128 +
                                                      (FP8 ? 32 * t : 8 * t));
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -267,8 +275,8 @@ __global__ void __launch_bounds__(128)
       const float cA = scale_log2 * ksA, cB = scale_log2 * ksB;
       float s00 = vA ? sacc[nt][0] * cA : -INFINITY, s01 = vA ? sacc[nt][1] * cA : -INFINITY;
       float s10 = vB ? sacc[nt][2] * cB : -INFINITY, s11 = vB ? sacc[nt][3] * cB : -INFINITY;
-      if (h0 >= G) s00 = s10 = -INFINITY;
-      if (h0 + 1 >= G) s01 = s11 = -INFINITY;
+      if (h0 >= HE) s00 = s10 = -INFINITY;
+      if (h0 + 1 >= HE) s01 = s11 = -INFINITY;
       float mx0 = fmaxf(s00, s10), mx1 = fmaxf(s01, s11);
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1) {
@@ -351,21 +359,23 @@ __global__ void __launch_bounds__(128)
     for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const int h = nt * 8 + 2 * t + e;
-        if (h >= G) continue;
+        const int h = nt * 8 + 2 * t + e;  // pair head: layer h / G, head h % G
+        if (h >= HE) continue;
+        __nv_bfloat16* Oh = L == 1 ? O : reinterpret_cast<__nv_bfloat16*>(lp.O[h / G]);
+        float* lseh = L == 1 ? lse : lp.lse[h / G];
         const float l = l_run[nt][e];
         const float inv = l > 0.f ? oscale / l : 0.f;
         uint32_t pk[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(o[nt][i][e] * inv, o[nt][i][e + 2] * inv);
-        __nv_bfloat16* orow = O + (r * Hq + g * G + h) * 128;
+        __nv_bfloat16* orow = Oh + (r * Hq + g * G + h % G) * 128;
         // pk[i] holds dims D(i), D(i) + 1
         uint4* d0 = reinterpret_cast<uint4*>(orow + (FP8 ? 16 * gid : 8 * gid));
         uint4* d1 = reinterpret_cast<uint4*>(orow + (FP8 ? 16 * gid + 8 : 8 * gid + 64));
         *d0 = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         *d1 = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-        if (lse != nullptr && gid == 0)
-          lse[r * Hq + g * G + h] = l > 0.f ? (m_run[nt][e] + __log2f(l)) * kLn2 : -INFINITY;
+        if (lseh != nullptr && gid == 0)
+          lseh[r * Hq + g * G + h % G] = l > 0.f ? (m_run[nt][e] + __log2f(l)) * kLn2 : -INFINITY;
       }
     }
   } else {
@@ -484,18 +494,53 @@ cudaError_t launch_g(const SparseArgs& a, cudaStream_t stream) {
         static_cast<const void*>(a.Vc), static_cast<const float*>(a.ks),
         static_cast<const float*>(a.vs), static_cast<const int32_t*>(a.idx),
         reinterpret_cast<__nv_bfloat16*>(a.O), a.lse, int64_t(a.T), a.Hkv, a.kw, sl2,
-        int64_t(a.cache_T));
+        int64_t(a.cache_T), SparseLayers{});
     if (e != cudaSuccess) return e;
   } else {
     sparse_mma_kernel<G, false, 1><<<unsigned((pairs + 3) / 4), 128, 0, stream>>>(
         reinterpret_cast<const __nv_bfloat16*>(a.Q), a.K, a.V, nullptr, nullptr, a.idx,
-        reinterpret_cast<__nv_bfloat16*>(a.O), a.lse, a.T, a.Hkv, a.kw, sl2, 0);
+        reinterpret_cast<__nv_bfloat16*>(a.O), a.lse, a.T, a.Hkv, a.kw, sl2, 0, SparseLayers{});
   }
   count_launch();
   return cudaGetLastError();
 }
 
+// L layers in one pass over the gathered rows (bf16 K/V)
+template <int G, int L>
+cudaError_t launch_fused(const SparseArgs& a, const SparseLayers& lp, cudaStream_t stream) {
+  const int64_t pairs = a.T * a.Hkv;
+  sparse_mma_kernel<G, false, 1, 1, L><<<unsigned((pairs + 3) / 4), 128, 0, stream>>>(
+      nullptr, a.K, a.V, nullptr, nullptr, a.idx, nullptr, nullptr, a.T, a.Hkv, a.kw,
+      a.scale * kLog2e, 0, lp);
+  count_launch();
+  return cudaGetLastError();
+}
+
+template <int G>
+cudaError_t launch_fused_g(const SparseArgs& a, const SparseLayers& lp, int L,
+                           cudaStream_t stream) {
+  switch (L) {
+    case 2: return launch_fused<G, 2>(a, lp, stream);
+    case 3: return launch_fused<G, 3>(a, lp, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 }  // namespace
+
+int max_fused_layers(int G) { return G <= 8 ? kMaxFusedLayers : 1; }
+
+cudaError_t launch_sparse_fused(const SparseArgs& a, const SparseLayers& lp, int L,
+                                cudaStream_t stream) {
+  if (L < 2 || L > max_fused_layers(a.Hq / a.Hkv)) return cudaErrorInvalidValue;
+  switch (a.Hq / a.Hkv) {
+    case 1: return launch_fused_g<1>(a, lp, L, stream);
+    case 2: return launch_fused_g<2>(a, lp, L, stream);
+    case 4: return launch_fused_g<4>(a, lp, L, stream);
+    case 8: return launch_fused_g<8>(a, lp, L, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
 
 cudaError_t launch_sparse(const SparseArgs& a, cudaStream_t stream) {
   switch (a.Hq / a.Hkv) {

@@ -137,6 +137,34 @@ def test_sparse_attn_on_oracle_lists(hs2, orc, T, Hq, Hkv, k, w):
     assert np.max(np.abs(lse_s.cpu().numpy() - lo)) <= LSE_ABS
 
 
+@pytest.mark.parametrize("T,Hq,Hkv,k,w,L", [(1500, 16, 2, 1024, 128, 3), (700, 4, 1, 64, 16, 2),
+                                            (900, 32, 4, 100, 32, 4), (500, 32, 2, 64, 64, 3)])
+def test_sparse_layers_fused_on_oracle_lists(hs2, orc, T, Hq, Hkv, k, w, L):
+    """Several sparse layers in one pass over the gathered rows: each layer's
+    output against the oracle's sparse attention with that layer's queries
+    (G <= 8 fuses up to three layers per pass, G = 16 none; four layers mix
+    a fused pass with a single one)."""
+    import torch
+    Q, K, V = rand_bf16((T, Hq, 128)), rand_bf16((T, Hkv, 128)), rand_bf16((T, Hkv, 128))
+    Qs = [rand_bf16((T, Hq, 128)) for _ in range(L)]
+    kv, sc = orc.KV(K, V), 1 / math.sqrt(128)
+    rows = np.arange(T)
+    _, lse = orc.full_attn(kv, Q, rows, sc)
+    idx, _ = orc.select(kv, Q, rows, sc, lse, k, w)
+    Os = [torch.empty(T, Hq, 128, dtype=torch.bfloat16, device="cuda") for _ in range(L)]
+    lses = [torch.empty(T, Hq, dtype=torch.float32, device="cuda") for _ in range(L)]
+    lses[-1] = None                                        # lse is optional per layer
+    shape = hs2.Shape.make(T, Hq, Hkv, k_global=k, window=w)
+    hs2.hs2_sparse_attn_layers([dev_bf16(q) for q in Qs], dev_bf16(K), dev_bf16(V), dev(idx), Os,
+                               lses, shape)
+    assert hs2.hs2_get_device_status() == hs2.OK
+    for l in range(L):
+        Oo, lo = orc.sparse_attn(kv, Qs[l], idx, sc)
+        assert_close_bf16(host_f64(Os[l]), Oo, f"O_sparse[{l}]")
+        if lses[l] is not None:
+            assert np.max(np.abs(lses[l].cpu().numpy() - lo)) <= LSE_ABS
+
+
 @pytest.mark.parametrize("T,Hq,Hkv,k,w", [(2048, 4, 1, 1024, 128), (1500, 16, 2, 64, 16),
                                           (900, 2, 1, 100, 32), (700, 16, 1, 32, 128),
                                           (333, 8, 1, 1024, 128), (1200, 4, 2, 0, 128)])
