@@ -12,14 +12,14 @@
 // care about the order of its terms, and the output permutation is undone at
 // the store) so that every lane's fragment words are contiguous in memory:
 //   * QK^T: lane (gid, t) reads 32 dims of gathered key rows gid and gid+8 --
-//     bf16: dims 32u + 8t .. +7 for u = 0..3, FP8: dims 32t .. 32t+31; for
-//     bf16 these words are the A registers as they are;
-//   * PV: lane (gid, t) reads 16 dims of gathered value rows 4t..4t+3 --
-//     bf16: dims 8*gid .. +7 and 64 + 8*gid .. +7, FP8: 16*gid .. +15 --
-//     paired into A registers with one byte permute each.
-// Each gathered row is read by four (K) or eight (V) lanes with 16-byte loads
-// that cover it exactly; in the bf16 layout the lanes of one load instruction
-// read whole 32-byte sectors of each row.  Softmax is online and base 2; P goes through 256
+//     bf16: dims 64u + 16t .. +15 for u = 0, 1 (two 32-byte loads), FP8:
+//     dims 32t .. 32t+31; for bf16 these words are the A registers as they are;
+//   * PV: lane (gid, t) reads dims 16*gid .. +15 of gathered value rows
+//     4t..4t+3 (bf16: one 32-byte load per row), paired into A registers with
+//     one byte permute each.
+// Each gathered row is read by four (K) or eight (V) lanes with loads that
+// cover it exactly; in the bf16 layout the lanes of one load instruction read
+// whole 32-byte sectors of each row.  Softmax is online and base 2; P goes through 256
 // bytes of shared memory per warp to become the B operand.  The FP8 variant
 // converts e4m3 codes to f16 exactly, multiplies the logits by the key's
 // scale and folds the value's scale into P.
@@ -95,6 +95,14 @@ __device__ __forceinline__ float from16(uint16_t v) {
   }
 }
 
+// 32 contiguous bytes (32-byte aligned) from global memory, read-only path
+__device__ __forceinline__ void ldg256(const void* p, uint32_t (&r)[8]) {
+  asm volatile("ld.global.nc.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "l"(p));
+}
+
 // G query heads of one KV head; FP8: e4m3 cache with per-(token, head) scales;
 // WPR warps share one (row, KV head) pair, splitting its list; with CS > 1
 // the CS CTAs of a thread-block cluster share it (CS * WPR parts) and combine
@@ -140,8 +148,8 @@ __global__ void __launch_bounds__(128)
   const int per = (kw + WPR * CS - 1) / (WPR * CS);
   const int e_lo = part * per, e_hi = min(kw, e_lo + per);
 
-  // query fragments: head nt*8+gid; step s = 2u + h2 uses the dims that lane
-  // t's K loads hold: bf16 dims 8t + 32u + 4*h2 + {0..3}, FP8 dims 32t + 4s + {0..3}
+  // query fragments: head nt*8+gid; step s uses the dims that lane t's K
+  // loads hold: bf16 dims 64(s/4) + 16t + 4(s%4) + {0..3}, FP8 dims 32t + 4s + {0..3}
   uint32_t qf[NT][8][2];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
@@ -150,10 +158,11 @@ __global__ void __launch_bounds__(128)
     const __nv_bfloat16* Qh =
         L == 1 ? Q : reinterpret_cast<const __nv_bfloat16*>(lp.Q[real ? hh / G : 0]);
     const uint4* qr = reinterpret_cast<const uint4*>(Qh + (r * Hq + g * G + (real ? hh % G : 0)) * 128 +
-                                                     (FP8 ? 32 * t : 8 * t));
+                                                     (FP8 ? 32 * t : 16 * t));
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const uint4 w = real ? __ldg(qr + (FP8 ? u : 4 * u)) : make_uint4(0, 0, 0, 0);
+      // bf16: 16-byte pieces u of the lane's two 32-byte runs at 64(u/2) + 16t
+      const uint4 w = real ? __ldg(qr + (FP8 ? u : (u & 1) + 8 * (u >> 1))) : make_uint4(0, 0, 0, 0);
       const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2) {
@@ -199,28 +208,27 @@ __global__ void __launch_bounds__(128)
     float vsc[4] = {0.f, 0.f, 0.f, 0.f};
     float ksA = 1.f, ksB = 1.f;
     if constexpr (!FP8) {
-      // lanes t = 0..3 of a row read 64 contiguous bytes per load (dims
-      // 32u + 8t .. +7): every 32-byte sector they touch is used whole
-      const uint4* pa = reinterpret_cast<const uint4*>(
-          reinterpret_cast<const __nv_bfloat16*>(Kp) + rowA * 128 + 8 * t);
-      const uint4* pb = reinterpret_cast<const uint4*>(
-          reinterpret_cast<const __nv_bfloat16*>(Kp) + rowB * 128 + 8 * t);
+      // lanes t = 0..3 of a row read 128 contiguous bytes per 32-byte load
+      // (dims 64u + 16t .. +15): every sector they touch is used whole
+      const __nv_bfloat16* pa = reinterpret_cast<const __nv_bfloat16*>(Kp) + rowA * 128 + 16 * t;
+      const __nv_bfloat16* pb = reinterpret_cast<const __nv_bfloat16*>(Kp) + rowB * 128 + 16 * t;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const uint4 x = __ldg(pa + 4 * u), y = __ldg(pb + 4 * u);
-        ka[4 * u] = x.x; ka[4 * u + 1] = x.y; ka[4 * u + 2] = x.z; ka[4 * u + 3] = x.w;
-        kb[4 * u] = y.x; kb[4 * u + 1] = y.y; kb[4 * u + 2] = y.z; kb[4 * u + 3] = y.w;
+      for (int u = 0; u < 2; ++u) {
+        uint32_t x[8], y[8];
+        ldg256(pa + 64 * u, x);
+        ldg256(pb + 64 * u, y);
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+          ka[8 * u + w] = x[w];
+          kb[8 * u + w] = y[w];
+        }
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int64_t rv = (tok0 + (jP[u] >= 0 ? jP[u] : 0)) * Hkv + g;
-        // lanes gid = 0..7 read 128 contiguous bytes per load: dims
-        // 8*gid .. +7 and 64 + 8*gid .. +7
-        const uint4* pv = reinterpret_cast<const uint4*>(
-            reinterpret_cast<const __nv_bfloat16*>(Vp) + rv * 128 + 8 * gid);
-        const uint4 x = __ldg(pv), y = __ldg(pv + 8);
-        vw[u][0] = x.x; vw[u][1] = x.y; vw[u][2] = x.z; vw[u][3] = x.w;
-        vw[u][4] = y.x; vw[u][5] = y.y; vw[u][6] = y.z; vw[u][7] = y.w;
+        // lanes gid = 0..7 read a whole 256-byte row, 32 bytes each: dims
+        // 16*gid .. +15
+        ldg256(reinterpret_cast<const __nv_bfloat16*>(Vp) + rv * 128 + 16 * gid, vw[u]);
         vsc[u] = jP[u] >= 0 ? 1.f : 0.f;
       }
     } else {
@@ -309,8 +317,7 @@ __global__ void __launch_bounds__(128)
     }
     __syncwarp();
     // ---- O^T += V^T P^T: K slots {2t,2t+1,2t+8,2t+9} = keys 4t+{0,1,2,3};
-    // MMA i, row gid -> dim D(i) = 16*gid + 2i (FP8) or
-    // 8*gid + 64*(i/4) + 2*(i%4) (bf16); row gid+8 -> D(i) + 1
+    // MMA i, row gid -> dim D(i) = 16*gid + 2i; row gid+8 -> D(i) + 1
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const uint16_t* sp = sP[warp][nt] + gid * 16 + 4 * t;
@@ -370,8 +377,8 @@ __global__ void __launch_bounds__(128)
         for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(o[nt][i][e] * inv, o[nt][i][e + 2] * inv);
         __nv_bfloat16* orow = Oh + (r * Hq + g * G + h % G) * 128;
         // pk[i] holds dims D(i), D(i) + 1
-        uint4* d0 = reinterpret_cast<uint4*>(orow + (FP8 ? 16 * gid : 8 * gid));
-        uint4* d1 = reinterpret_cast<uint4*>(orow + (FP8 ? 16 * gid + 8 : 8 * gid + 64));
+        uint4* d0 = reinterpret_cast<uint4*>(orow + 16 * gid);
+        uint4* d1 = reinterpret_cast<uint4*>(orow + 16 * gid + 8);
         *d0 = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         *d1 = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         if (lseh != nullptr && gid == 0)
@@ -389,7 +396,7 @@ __global__ void __launch_bounds__(128)
       }
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const int d = FP8 ? 16 * gid + 2 * i : 8 * gid + 64 * (i >> 2) + 2 * (i & 3);
+        const int d = 16 * gid + 2 * i;
         sO[warp][nt * 8 + 2 * t][d] = o[nt][i][0];
         sO[warp][nt * 8 + 2 * t + 1][d] = o[nt][i][1];
         sO[warp][nt * 8 + 2 * t][d + 1] = o[nt][i][2];
