@@ -61,6 +61,23 @@ def test_host_side_errors(hs2):
     assert L.hs2_sparse_attn(ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr, None, C.byref(sw), None) == hs2.ERR_INVALID_ARG
     # bridge: d_model must be a positive multiple of 64
     assert L.hs2_bridge_kv(ok_ptr, 100, ok_ptr, ok_ptr, ok_ptr, ok_ptr, C.byref(s), None) == hs2.ERR_INVALID_ARG
+    # bridge into the FP8 cache: null output, misaligned scale, bad d_model
+    assert L.hs2_bridge_kv_fp8(ok_ptr, 128, ok_ptr, ok_ptr, None, ok_ptr, ok_ptr, C.byref(s),
+                               None) == hs2.ERR_INVALID_ARG
+    assert L.hs2_bridge_kv_fp8(ok_ptr, 128, ok_ptr, ok_ptr, ok_ptr, ok_ptr, bad_ptr, C.byref(s),
+                               None) == hs2.ERR_INVALID_ARG
+    assert L.hs2_bridge_kv_fp8(ok_ptr, 96, ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr, C.byref(s),
+                               None) == hs2.ERR_INVALID_ARG
+    assert L.hs2_bridge_kv_fp8(ok_ptr, 128, ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr, C.byref(s64),
+                               None) == hs2.ERR_UNSUPPORTED
+    # fused sparse layers: no layers, a null or misaligned layer pointer
+    two = (C.c_void_p * 2)(0x10000, 0x20000)
+    one_null = (C.c_void_p * 2)(0x10000, None)
+    one_bad = (C.c_void_p * 2)(0x10000, 0x20001)
+    P = C.POINTER(C.c_void_p)
+    for n, q, o in ((0, two, two), (2, one_null, two), (2, two, one_bad)):
+        assert L.hs2_sparse_attn_layers(n, C.cast(q, P), ok_ptr, ok_ptr, ok_ptr, C.cast(o, P), None,
+                                        C.byref(s), None) == hs2.ERR_INVALID_ARG
     # workspace too small for selection
     need = hs2.workspace_size(hs2.OP_SELECT, s)
     if need > 0:
