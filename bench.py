@@ -48,6 +48,35 @@ def peaks():
 
 
 # ---------------------------------------------------------------------------
+# ranks: one process per GPU, independent replicas of the block
+# ---------------------------------------------------------------------------
+def init_ranks(world, backend="nccl"):
+    """Join the process group when there is more than one rank (env://
+    rendezvous from MASTER_ADDR/MASTER_PORT); returns whether one was joined."""
+    if world <= 1:
+        return False
+    import datetime
+    torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return True
+
+
+def max_over_ranks(x, device, joined):
+    """The largest value of x over all ranks (a step time: the slowest rank
+    sets the job's time)."""
+    if not joined:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank, world, ms):
+    """Whole-job tokens/s: every rank processes its own tokens_per_rank in
+    the (max over ranks) step time ms."""
+    return tokens_per_rank * world / (ms / 1e3)
+
+
+# ---------------------------------------------------------------------------
 # inputs (seeded, on the device)
 # ---------------------------------------------------------------------------
 def make_inputs(cfg, device):
@@ -378,11 +407,7 @@ def main():
     import long_context_bridge_b200 as hs2
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    pg = None
-    if world > 1:
-        import datetime
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-        pg = True
+    pg = init_ranks(world)
 
     T, Hq, Hkv = cfg.T, cfg.n_q_heads, cfg.n_kv_heads
     inp = make_inputs(cfg, dev)
@@ -446,11 +471,7 @@ def main():
         end.record()
         barrier()
         n_launch = hs2.hs2_kernel_launches() - n0
-    ms = start.elapsed_time(end) / args.steps
-    if pg:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(start.elapsed_time(end) / args.steps, dev, pg)
     kern_ms = {n: float(np.mean([a.elapsed_time(b) for a, b in ev[n]])) for n in names}
     st = hs2.hs2_get_device_status()
     assert st == hs2.OK, f"device status {st}"
@@ -489,14 +510,10 @@ def main():
             e2e_step()
         t2.record()
         barrier()
-        ms_e2e = s2.elapsed_time(t2) / n_e2e
-        if pg:
-            t = torch.tensor([ms_e2e], device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            ms_e2e = float(t.item())
+        ms_e2e = max_over_ranks(s2.elapsed_time(t2) / n_e2e, dev, pg)
         h2d = sum(x.numel() * x.element_size() for x in [hH, hQ, *hQs])
         d2h = sum(x.numel() * x.element_size() for x in [hO, *hOs, hidx, hlse])
-        e2e = {"value": T * world / (ms_e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        e2e = {"value": job_throughput(T, world, ms_e2e), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
                "note": "hs2_block_prefill (bridge inside) with pinned-host inputs and outputs; "
                        "needles not planted on this path"}
@@ -553,7 +570,7 @@ def main():
     cpu = None
     if not args.no_cpu and world == 1:
         cpu = OracleSample(cfg).run(320, seed=5)
-    line = {"metric": METRIC, "value": T * world / (ms / 1e3), "unit": UNIT, "n_gpus": world,
+    line = {"metric": METRIC, "value": job_throughput(T, world, ms), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": config, "clocks": clk.summary(), "e2e": e2e,
