@@ -10,6 +10,8 @@
 //   warp 1     allocates TMEM, one lane issues tcgen05.mma 128xBNx16 and
 //              commits each stage back to the producer
 //   warps 2-5  epilogue: TMEM -> registers -> bf16 -> global
+// bridge_fp8_kernel (further down) is the same GEMM with the K and V tiles of
+// one KV head in one CTA and an epilogue that writes the FP8 decode cache.
 #include <cuda_fp8.h>
 
 #include "common.cuh"
