@@ -118,7 +118,7 @@ def test_full_attn_matches_oracle(hs2, orc, T, Hq, Hkv):
 
 
 @pytest.mark.parametrize("T,Hq,Hkv,k,w", [(2048, 4, 1, 1024, 128), (500, 16, 2, 64, 16),
-                                          (300, 8, 1, 0, 128)])
+                                          (300, 8, 1, 0, 128), (2600, 8, 1, 2048, 256)])
 def test_sparse_attn_on_oracle_lists(hs2, orc, T, Hq, Hkv, k, w):
     import torch
     Q, K, V = rand_bf16((T, Hq, 128)), rand_bf16((T, Hkv, 128)), rand_bf16((T, Hkv, 128))
@@ -167,7 +167,8 @@ def test_sparse_layers_fused_on_oracle_lists(hs2, orc, T, Hq, Hkv, k, w, L):
 
 @pytest.mark.parametrize("T,Hq,Hkv,k,w", [(2048, 4, 1, 1024, 128), (1500, 16, 2, 64, 16),
                                           (900, 2, 1, 100, 32), (700, 16, 1, 32, 128),
-                                          (333, 8, 1, 1024, 128), (1200, 4, 2, 0, 128)])
+                                          (333, 8, 1, 1024, 128), (1200, 4, 2, 0, 128),
+                                          (3000, 8, 1, 2048, 256)])
 def test_select_matches_oracle(hs2, orc, T, Hq, Hkv, k, w):
     import torch
     from helpers import check_index_lists
