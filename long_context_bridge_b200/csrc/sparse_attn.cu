@@ -106,11 +106,11 @@ __device__ __forceinline__ void ldg256(const void* p, uint32_t (&r)[8]) {
 // G query heads of one KV head; FP8: e4m3 cache with per-(token, head) scales;
 // WPR warps share one (row, KV head) pair, splitting its list; with CS > 1
 // the CS CTAs of a thread-block cluster share it (CS * WPR parts) and combine
-// their partial softmax states through distributed shared memory.  L > 1
-// fuses L sparse layers: the pair's L * G heads (layer e / G, head e % G of
+// their partial softmax states through distributed shared memory.  NL > 1
+// fuses NL sparse layers: the pair's NL * G heads (layer e / G, head e % G of
 // pair head e) share every gathered K/V row; their Q, O and lse come from
 // `lp`.
-template <int G, bool FP8, int WPR, int CS = 1, int L = 1>
+template <int G, bool FP8, int WPR, int CS = 1, int NL = 1>
 __global__ void __launch_bounds__(128)
     sparse_mma_kernel(const __nv_bfloat16* __restrict__ Q, const void* __restrict__ Kp,
                       const void* __restrict__ Vp, const float* __restrict__ ks,
@@ -118,9 +118,9 @@ __global__ void __launch_bounds__(128)
                       __nv_bfloat16* __restrict__ O, float* __restrict__ lse, int64_t rows,
                       int Hkv, int kw, float scale_log2, int64_t cache_T,
                       const __grid_constant__ SparseLayers lp) {
-  constexpr int HE = L * G;                       // heads of a pair
+  constexpr int HE = NL * G;                      // heads of a pair
   constexpr int NT = (HE + 7) / 8;                // 8-head n-tiles
-  static_assert(L == 1 || (WPR == 1 && !FP8), "layers are fused on the prefill path only");
+  static_assert(NL == 1 || (WPR == 1 && !FP8), "layers are fused on the prefill path only");
   constexpr int NW = 4;                  // warps per CTA
   constexpr int PAIRS = NW / WPR;        // (row, KV head) pairs per CTA
   constexpr bool F16 = FP8;              // FP8 path: f16 MMA; bf16 path: bf16 MMA
@@ -156,7 +156,7 @@ __global__ void __launch_bounds__(128)
     const int hh = nt * 8 + gid;  // pair head
     const bool real = hh < HE && active;
     const __nv_bfloat16* Qh =
-        L == 1 ? Q : reinterpret_cast<const __nv_bfloat16*>(lp.Q[real ? hh / G : 0]);
+        NL == 1 ? Q : reinterpret_cast<const __nv_bfloat16*>(lp.Q[real ? hh / G : 0]);
     const uint4* qr = reinterpret_cast<const uint4*>(Qh + (r * Hq + g * G + (real ? hh % G : 0)) * 128 +
                                                      (FP8 ? 32 * t : 16 * t));
 #pragma unroll
@@ -368,8 +368,8 @@ __global__ void __launch_bounds__(128)
       for (int e = 0; e < 2; ++e) {
         const int h = nt * 8 + 2 * t + e;  // pair head: layer h / G, head h % G
         if (h >= HE) continue;
-        __nv_bfloat16* Oh = L == 1 ? O : reinterpret_cast<__nv_bfloat16*>(lp.O[h / G]);
-        float* lseh = L == 1 ? lse : lp.lse[h / G];
+        __nv_bfloat16* Oh = NL == 1 ? O : reinterpret_cast<__nv_bfloat16*>(lp.O[h / G]);
+        float* lseh = NL == 1 ? lse : lp.lse[h / G];
         const float l = l_run[nt][e];
         const float inv = l > 0.f ? oscale / l : 0.f;
         uint32_t pk[8];
