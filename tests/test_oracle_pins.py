@@ -118,6 +118,28 @@ def test_bridge_fp8_is_nearest_code_of_scaled_row(orc):
     assert np.all(top[amax > 0] == 0x7E)
 
 
+def test_bridge_fp8_rule_equals_decode_cache_recipe(orc):
+    # the cache f1 writes follows the same rule as the decode workload's input
+    # recipe: on the same bf16 rows, equal scales and codes (zero codes with
+    # either sign: the recipe's numpy quantiser writes +0)
+    T, Hkv = 64, 2
+    K = rand_bf16((T * Hkv, 128))
+    V = rand_bf16((T * Hkv, 128))
+    Kc = np.empty((T * Hkv, 128), np.uint8)
+    Vc = np.empty_like(Kc)
+    S = np.empty(T * Hkv, np.float32)
+    orc.lib().orc_quantize_rows(orc._p(K), orc._p(V), T * Hkv, 128, orc._p(Kc), orc._p(Vc),
+                                orc._p(S))
+    kf, vf = synth.bf16_bits_to_f32(K), synth.bf16_bits_to_f32(V)
+    amax = np.maximum(np.abs(kf).max(axis=1), np.abs(vf).max(axis=1)).astype(np.float32)
+    s_rec = np.where(amax > 0, amax / np.float32(448.0), np.float32(1.0)).astype(np.float32)
+    assert np.array_equal(S, s_rec)
+    for codes, x in ((Kc, kf), (Vc, vf)):
+        rec = synth.e4m3_quantize_np((x / s_rec[:, None]).astype(np.float32))
+        same = (codes == rec) | (((codes | rec) & 0x7F) == 0)
+        assert same.all()
+
+
 # --------------------------------------------------------------------------
 # S1 bridge
 # --------------------------------------------------------------------------
