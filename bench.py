@@ -543,6 +543,10 @@ def main():
                          ("TFLOP/s" if b == "tensor" else "GB/s"):
                              (a / s / 1e12) if b == "tensor" else (a / s / 1e9),
                          "frac": ((a / s / 1e12) / tfl) if b == "tensor" else ((a / s / 1e9) / hbm)}
+    per_kernel["sparse_attn"]["note"] = (
+        "algorithmic bytes (every gathered row counted once per list) over time, against "
+        "the HBM copy peak; the rows are mostly served from L2 (ncu: DRAM bytes about 1.5% "
+        "of the gathered bytes), so the fraction can exceed 1")
     # f4, a separate labelled figure: the same three sparse layers in one pass
     # over the gathered rows (valid only when all layers' queries exist up
     # front, so it is not part of the step above)
