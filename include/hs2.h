@@ -34,8 +34,13 @@
  * - Device-side waits are bounded.  A wait that runs out sets a sticky device
  *   status word, the kernel returns early, and the next
  *   hs2_get_device_status() reports HS2_ERR_TIMEOUT.
- * - Supported: head_dim == 128; G in {1, 2, 4, 8, 16}; 0 <= k_global <= 2048;
- *   1 <= window <= 2048; 1 <= T <= 2^31 - 1 (T * n_q_heads * 128 < 2^40).
+ * - Index lists passed in by the caller are checked entry by entry on the
+ *   device: an entry other than -1 outside [0, T) is skipped like -1 and
+ *   recorded, and the next hs2_get_device_status() reports HS2_ERR_BAD_INDEX.
+ * - Supported: head_dim == 128; G in {1, 2, 4, 8, 16} (a query tile packs
+ *   128 / G whole queries of one KV head, so G must divide 128);
+ *   0 <= k_global <= 2048; 1 <= window <= 2048; 1 <= T <= 2^31 - 1
+ *   (T * n_q_heads * 128 < 2^40).  Other shapes return HS2_ERR_UNSUPPORTED.
  * - Thread safety: calls on different streams may run concurrently; the only
  *   global state is one-time kernel attribute set-up per device.
  */
@@ -55,7 +60,8 @@ typedef enum {
   HS2_ERR_UNSUPPORTED = 2, /* head_dim != 128, G not in {1,2,4,8,16}, ...      */
   HS2_ERR_WORKSPACE = 3,   /* workspace pointer null or smaller than required  */
   HS2_ERR_CUDA = 4,        /* a CUDA runtime/driver call or launch failed      */
-  HS2_ERR_TIMEOUT = 5      /* a device-side bounded wait ran out               */
+  HS2_ERR_TIMEOUT = 5,     /* a device-side bounded wait ran out               */
+  HS2_ERR_BAD_INDEX = 6    /* an index-list entry outside [-1, T) was skipped  */
 } hs2_status;
 
 typedef uint16_t hs2_bf16;    /* raw bf16 bits */
@@ -163,7 +169,7 @@ hs2_status hs2_select_topk(const hs2_bf16* Q, const hs2_bf16* K, const float* ls
  *     overlap on the same device, e.g. on two streams, race on it: serialise
  *     them.
  *   - The kernel runs as many persistent CTAs as the scratch holds; each needs
- *     4 * (128 / G) * max(2 * k_global, 256) * 8 + 65536 bytes.  A shape for
+ *     4 * (128 / G) * max(2 * k_global, 256) * 8 + 131072 bytes.  A shape for
  *     which one CTA does not fit returns HS2_ERR_UNSUPPORTED.
  * Errors otherwise as hs2_select_topk (HS2_ERR_CUDA if the address lookup
  * fails).
@@ -177,11 +183,13 @@ hs2_status hs2_select_topk_noalloc(const hs2_bf16* Q, const hs2_bf16* K, const f
  * KV Reuse paragraph of the javabetter.cn explainer and the aitop.news
  * summary: each sparse layer has its own queries, reuses the full layer's K/V
  * cache and selection indices, and stores no K/V.  For row i, head h:
- *   s_j = scale * Q[i,h] . K[j,g] for j in idx[i,g,:] (entries < 0 skipped)
+ *   s_j = scale * Q[i,h] . K[j,g] for j in idx[i,g,:] (entries -1 skipped)
  *   O[i,h] = sum_j softmax_j(s) V[j,g];  lse (nullable) = ln sum_j exp(s_j).
- * Entries must satisfy -1 <= idx < T; lists hold no duplicates (as written by
- * hs2_select_topk).  A row whose list is entirely -1 gets O = 0, lse = -inf.
- * No workspace.
+ * Entries should satisfy -1 <= idx < T and a list should hold no duplicates
+ * (as written by hs2_select_topk).  Any other entry is skipped like -1 and
+ * reported as HS2_ERR_BAD_INDEX by the next hs2_get_device_status(); K and V
+ * are never read outside their T rows.  A row whose list is entirely -1 gets
+ * O = 0, lse = -inf.  No workspace.
  */
 hs2_status hs2_sparse_attn(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V,
                            const int32_t* idx, hs2_bf16* O, float* lse,
@@ -225,6 +233,8 @@ hs2_status hs2_block_prefill(const hs2_bf16* H, int32_t d_model, const hs2_bf16*
  * and the block (full attention, selection, n_sparse sparse layers) runs on
  *   K^[t,g,:] = e4m3(Kc[b,t,g,:]) * k_scale[b,t,g],  likewise V with v_scale.
  * seq_len: HOST array [batch], 1 <= seq_len[b] <= shape->T.
+ * Limits: batch <= 64 and batch * shape->T <= 2^31 - 1 (HS2_ERR_UNSUPPORTED
+ * otherwise, before any launch).
  * Kc, Vc [batch, shape->T, n_kv_heads, 128] e4m3; k_scale, v_scale
  * [batch, shape->T, n_kv_heads] fp32 (they may alias).
  * q_full, o_full [batch, n_q_heads, 128] bf16; lse [batch, n_q_heads] fp32;
@@ -244,8 +254,9 @@ hs2_status hs2_block_decode(int32_t batch, const int64_t* seq_len, const hs2_bf1
  * the op needs none.  Returns (size_t)-1 for invalid arguments. */
 size_t hs2_workspace_size(int32_t op, const hs2_shape* shape, int32_t batch, int32_t d_model);
 
-/* Synchronises `stream` and reports a sticky device-side error (a bounded
- * wait that ran out) as HS2_ERR_TIMEOUT, clearing it; CUDA errors as
+/* Synchronises `stream` and reports a sticky device-side error, clearing it:
+ * a bounded wait that ran out as HS2_ERR_TIMEOUT, otherwise a skipped
+ * out-of-range index entry as HS2_ERR_BAD_INDEX; CUDA errors as
  * HS2_ERR_CUDA. */
 hs2_status hs2_get_device_status(void* stream);
 

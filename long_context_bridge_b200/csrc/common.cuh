@@ -29,8 +29,9 @@ enum : unsigned { DEV_OK = 0, DEV_TIMEOUT = 1, DEV_BAD_INDEX = 2 };
     return v;                                                         \
   }
 
+// Codes are bits: a timeout and a bad index entry can both be recorded.
 __device__ __forceinline__ void set_dev_status(unsigned code) {
-  atomicCAS(&g_dev_status, 0u, code);
+  atomicOr(&g_dev_status, code);
 }
 
 // Spin budget for one wait: ~2^31 cycles (about a second at 1.9 GHz).

@@ -52,7 +52,7 @@ constexpr int CAPC = 8192;          // candidate list capacity per (b, g)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-constexpr int MAX_B = 64;
+constexpr int MAX_B = kDecodeMaxBatch;
 constexpr float kPScale = 1024.f;   // P' = p * v_scale * 2^10 keeps f16 products normal
 
 struct Partial {  // per (b, h, chunk)

@@ -132,6 +132,7 @@ const char* hs2_status_string(hs2_status s) {
     case HS2_ERR_WORKSPACE: return "workspace too small";
     case HS2_ERR_CUDA: return "CUDA error";
     case HS2_ERR_TIMEOUT: return "device-side wait timed out";
+    case HS2_ERR_BAD_INDEX: return "index list entry out of range (skipped)";
   }
   return "unknown status";
 }
@@ -148,7 +149,8 @@ hs2_status hs2_get_device_status(void* stream) {
   v |= status_sparse(true);
   v |= status_decode(true);
   if (v == ~0u) return HS2_ERR_CUDA;
-  if (v != 0) return HS2_ERR_TIMEOUT;
+  if (v & DEV_TIMEOUT) return HS2_ERR_TIMEOUT;
+  if (v & DEV_BAD_INDEX) return HS2_ERR_BAD_INDEX;
   return HS2_OK;
 }
 
@@ -164,7 +166,8 @@ size_t hs2_workspace_size(int32_t op, const hs2_shape* s, int32_t batch, int32_t
     case HS2_OP_BLOCK_PREFILL:
       return select_workspace_bytes(s->T, s->n_q_heads, s->n_kv_heads, s->k_global, s->window);
     case HS2_OP_BLOCK_DECODE:
-      if (batch <= 0) return size_t(-1);
+      if (batch <= 0 || batch > kDecodeMaxBatch || int64_t(batch) * s->T > INT32_MAX)
+        return size_t(-1);
       return decode_workspace_bytes(batch, s->T, s->n_q_heads, s->n_kv_heads, s->k_global,
                                     s->window);
   }
@@ -328,6 +331,7 @@ hs2_status hs2_block_decode(int32_t batch, const int64_t* seq_len, const hs2_bf1
            aligned16(lse) && aligned16(idx));
   HS2_NEED((reinterpret_cast<uintptr_t>(k_scale) & 3) == 0 &&
            (reinterpret_cast<uintptr_t>(v_scale) & 3) == 0);
+  if (batch > kDecodeMaxBatch || int64_t(batch) * s->T > INT32_MAX) return HS2_ERR_UNSUPPORTED;
   for (int b = 0; b < batch; ++b) HS2_NEED(seq_len[b] >= 1 && seq_len[b] <= s->T);
   HS2_NEED(n_sparse >= 0 && (n_sparse == 0 || (q_sparse && o_sparse)));
   for (int l = 0; l < n_sparse; ++l)

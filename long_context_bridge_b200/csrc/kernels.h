@@ -138,6 +138,8 @@ struct DecodeArgs {
   void* ws;
   size_t ws_bytes;
 };
+// decode limits, checked on the host before any launch
+constexpr int kDecodeMaxBatch = 64;
 size_t decode_workspace_bytes(int B, int64_t cap, int Hq, int Hkv, int k, int w);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 

@@ -36,8 +36,6 @@
 //     sorted ascending by a register bitonic sort.
 // Items whose every query has at most k candidates skip the scoring: all
 // candidates are selected.
-#include <mutex>
-
 #include "common.cuh"
 #include "kernels.h"
 
@@ -648,31 +646,26 @@ cudaError_t launch_g(const SelectArgs& a, cudaStream_t stream) {
 constexpr size_t kNoAllocScratchBytes = size_t(48) << 20;
 static __device__ __align__(256) unsigned char g_select_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
-
-// Device address of g_select_scratch on the current device, looked up once
-// per device (host code must not use the symbol itself as an address).
+// Device address of g_select_scratch in the current context.  Host code must
+// not use the symbol itself as an address.  The lookup runs on every call, so
+// a context that was reset and re-created never sees a stale address; the
+// first call in a context also loads the module, which is why that call
+// should come before any stream capture.
 cudaError_t select_scratch_address(void** out) {
-  static std::mutex mu;
-  static void* addr[kMaxDevices] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_select_scratch);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_select_scratch);
-    if (e != cudaSuccess) return e;
-    addr[dev] = p;
-  }
-  *out = addr[dev];
+  *out = p;
   return cudaSuccess;
 }
 
+// bytes of the file-scope scratch taken by one CTA (the documented figure:
+// 4 * (128 / G) * max(2k, 256) * 8 + 131072)
 size_t noalloc_cta_bytes(int QT, int k) {
   return size_t(4) * QT * buffer_cap(k) * sizeof(uint2) + size_t(SCORER_WARPS) * 2048 * sizeof(uint32_t);
 }
+static_assert(size_t(SCORER_WARPS) * 2048 * sizeof(uint32_t) == 131072,
+              "the per-CTA staging term documented for hs2_select_topk_noalloc");
 
 template <int G>
 cudaError_t launch_noalloc_g(const SelectArgs& a, void* scratch, cudaStream_t stream) {

@@ -95,6 +95,15 @@ __device__ __forceinline__ float from16(uint16_t v) {
   }
 }
 
+// A list entry as the gather uses it: -1 (no token) and positions in
+// [0, bound) pass unchanged; anything else is recorded as DEV_BAD_INDEX and
+// skipped like -1, so a caller's bad list never reads outside K/V.
+__device__ __forceinline__ int checked_entry(int j, int bound) {
+  if (j == -1 || unsigned(j) < unsigned(bound)) return j;
+  set_dev_status(DEV_BAD_INDEX);
+  return -1;
+}
+
 // 32 contiguous bytes (32-byte aligned) from global memory, read-only path
 __device__ __forceinline__ void ldg256(const void* p, uint32_t (&r)[8]) {
   asm volatile("ld.global.nc.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
@@ -147,6 +156,8 @@ __global__ void __launch_bounds__(128)
   const int32_t* list = idx + (r * Hkv + g) * kw;
   const int per = (kw + WPR * CS - 1) / (WPR * CS);
   const int e_lo = part * per, e_hi = min(kw, e_lo + per);
+  // valid positions: rows of K/V (prefill) or of a sequence's cache (decode)
+  const int jbound = int(FP8 ? cache_T : rows);
 
   // query fragments: head nt*8+gid; step s uses the dims that lane t's K
   // loads hold: bf16 dims 64(s/4) + 16t + 4(s%4) + {0..3}, FP8 dims 32t + 4s + {0..3}
@@ -191,7 +202,7 @@ __global__ void __launch_bounds__(128)
   // one step ahead so that a step's gathers do not wait for its list load
   int jl_next = (active && e_lo + (lane & 15) < e_hi) ? __ldg(list + e_lo + (lane & 15)) : -1;
   for (int e0 = e_lo; e0 < e_hi && active; e0 += 16) {
-    const int jl = jl_next;
+    const int jl = checked_entry(jl_next, jbound);
     const int en = e0 + 16 + (lane & 15);
     jl_next = en < e_hi ? __ldg(list + en) : -1;
     const int jA = __shfl_sync(0xffffffffu, jl, gid), jB = __shfl_sync(0xffffffffu, jl, gid + 8);

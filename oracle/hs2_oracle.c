@@ -108,21 +108,22 @@ typedef struct {
   int Hkv, d;
 } kv_src;
 
+/* Value of every e4m3 code, filled once when the library is loaded (before
+ * any parallel region reads it). */
+static double e4m3_table[256];
+__attribute__((constructor)) static void fill_e4m3_table(void) {
+  for (int c = 0; c < 256; ++c) e4m3_table[c] = orc_e4m3_value(c);
+}
+
 static void fetch_row(const kv_src* s, int64_t t, int g, double* out) {
   int64_t base = (t * s->Hkv + g) * (int64_t)s->d;
   if (s->kind == ORC_BF16) {
     const uint16_t* p = (const uint16_t*)s->data + base;
     for (int c = 0; c < s->d; ++c) out[c] = bf16_value(p[c]);
   } else {
-    static double table[256];
-    static int ready = 0;
-    if (!ready) { /* benign race: every thread writes the same values */
-      for (int c = 0; c < 256; ++c) table[c] = orc_e4m3_value(c);
-      ready = 1;
-    }
     const uint8_t* p = (const uint8_t*)s->data + base;
     double sc = (double)s->scale[t * s->Hkv + g];
-    for (int c = 0; c < s->d; ++c) out[c] = table[p[c]] * sc; /* exact in fp64 */
+    for (int c = 0; c < s->d; ++c) out[c] = e4m3_table[p[c]] * sc; /* exact in fp64 */
   }
 }
 

@@ -301,6 +301,52 @@ def bridge_inputs_np(cfg: BlockConfig, T: int | None = None):
     return H, Wk, Wv
 
 
+# The bridge recipe on a coarse dyadic grid: H = round(2 z) / 2 clipped to
+# [-8, 8] and W = round(2^9 z / sqrt(d_model)) / 2^9 clipped to [-1/8, 1/8]
+# (z the same N(0,1) draws as bridge_inputs_np).  Every product H W is then
+# an integer multiple of 2^-10 of magnitude <= 1, so every partial sum of a
+# row's d_model <= 2^11 products is an integer multiple of 2^-10 below 2^11:
+# at most 21 significant bits, exact in fp32 whatever the order of summation.
+# An fp32-accumulating bridge and an fp64 one then round the same exact
+# value to bf16.
+def _dyadic_h(z):
+    return np.clip(np.round(2.0 * z), -16, 16) / 2.0
+
+
+def _dyadic_w(z, dm):
+    return np.clip(np.round(z * (512.0 / math.sqrt(dm))), -64, 64) / 512.0
+
+
+def bridge_inputs_dyadic_np(cfg: BlockConfig, T: int | None = None):
+    """H [T, d_model], W_k, W_v [d_model, Hkv*d] bf16 bits on the dyadic grid."""
+    T = cfg.T if T is None else T
+    dm, N = cfg.d_model, cfg.n_kv_heads * cfg.head_dim
+    H = f64_to_bf16_bits(_dyadic_h(normals_np(cfg.seed, TID_H, 0, T * dm))).reshape(T, dm)
+    Wk = f64_to_bf16_bits(_dyadic_w(normals_np(cfg.seed, TID_WK, 0, dm * N), dm)).reshape(dm, N)
+    Wv = f64_to_bf16_bits(_dyadic_w(normals_np(cfg.seed, TID_WV, 0, dm * N), dm)).reshape(dm, N)
+    return H, Wk, Wv
+
+
+def bridge_inputs_dyadic_torch(cfg: BlockConfig, T: int | None = None, device="cuda",
+                               chunk: int = 1 << 26):
+    """bridge_inputs_dyadic_np's tensors generated on the device (bf16)."""
+    import torch
+    T = cfg.T if T is None else T
+    dm, N = cfg.d_model, cfg.n_kv_heads * cfg.head_dim
+
+    def gen(tid, count, grid):
+        out = torch.empty(count, dtype=torch.bfloat16, device=device)
+        for s0 in range(0, count, chunk):
+            c = min(chunk, count - s0)
+            out[s0:s0 + c] = grid(normals_torch(cfg.seed, tid, s0, c, device)).float().bfloat16()
+        return out
+
+    h = lambda z: torch.clamp(torch.round(2.0 * z), -16, 16) / 2.0
+    w = lambda z: torch.clamp(torch.round(z * (512.0 / math.sqrt(dm))), -64, 64) / 512.0
+    return (gen(TID_H, T * dm, h).view(T, dm), gen(TID_WK, dm * N, w).view(dm, N),
+            gen(TID_WV, dm * N, w).view(dm, N))
+
+
 def plant_needles_np(cfg: BlockConfig, K: np.ndarray, positions: list[np.ndarray]) -> None:
     """Overwrite needle rows of K [T, Hkv, d] (bf16 bits) in place."""
     rows = needle_key_bits(cfg)
@@ -342,6 +388,34 @@ def decode_cache_np(cfg: BlockConfig, N: int, batch: int | None = None) -> Decod
         Kc[b] = e4m3_quantize_np((K / s[:, :, None]).astype(np.float32))
         Vc[b] = e4m3_quantize_np((V / s[:, :, None]).astype(np.float32))
     return DecodeCache(Kc, Vc, S, needles)
+
+
+def decode_cache_split_scales_np(cfg: BlockConfig, N: int, batch: int | None = None,
+                                 v_gain: float = 8.0):
+    """FP8 cache whose K and V rows have their own scales: bf16 N(0,1) K plus
+    needles and v_gain * N(0,1) V, k_scale = amax|K row| / 448 and v_scale =
+    amax|V row| / 448 per (token, KV head), codes = e4m3(x / scale).
+    Returns (Kc, Vc, k_scale, v_scale)."""
+    B = cfg.batch if batch is None else batch
+    Hkv, d = cfg.n_kv_heads, cfg.head_dim
+    Kc = np.empty((B, N, Hkv, d), np.uint8)
+    Vc = np.empty((B, N, Hkv, d), np.uint8)
+    KS = np.empty((B, N, Hkv), np.float32)
+    VS = np.empty((B, N, Hkv), np.float32)
+    nrows = needle_key_bits(cfg)
+    for b in range(B):
+        K = bf16_bits_to_f32(normal_bf16_np(cfg.seed, TID_DEC_K0 + b, 0, N * Hkv * d)).reshape(N, Hkv, d)
+        V = bf16_bits_to_f32(normal_bf16_np(cfg.seed, TID_DEC_V0 + b, 0, N * Hkv * d,
+                                            v_gain)).reshape(N, Hkv, d)
+        for g in range(Hkv):
+            pos = needle_positions(cfg.seed, TID_DEC_POS0 + b, g, min(cfg.n_needles, N), N)
+            K[pos, g, :] = bf16_bits_to_f32(nrows[g])
+        for X, S, C in ((K, KS, Kc), (V, VS, Vc)):
+            amax = np.abs(X).max(axis=2).astype(np.float32)
+            s = np.where(amax > 0, amax / np.float32(448.0), np.float32(1.0)).astype(np.float32)
+            S[b] = s
+            C[b] = e4m3_quantize_np((X / s[:, :, None]).astype(np.float32))
+    return Kc, Vc, KS, VS
 
 
 def q_rows_torch(cfg: BlockConfig, tid: int, T: int | None = None, device="cuda", rows: int = 4096):

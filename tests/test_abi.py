@@ -93,7 +93,22 @@ def test_host_side_errors(hs2):
                               ok_ptr, 0, C.cast(arr, C.POINTER(C.c_void_p)),
                               C.cast(arr, C.POINTER(C.c_void_p)), C.byref(sd), ok_ptr, 1 << 40,
                               None) == hs2.ERR_INVALID_ARG
+    # decode limits, checked before any launch: batch > 64, batch * capacity >= 2^31
+    lens65 = (C.c_int64 * 65)(*([10] * 65))
+    assert L.hs2_block_decode(65, lens65, ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr,
+                              ok_ptr, 0, C.cast(arr, C.POINTER(C.c_void_p)),
+                              C.cast(arr, C.POINTER(C.c_void_p)), C.byref(sd), ok_ptr, 1 << 40,
+                              None) == hs2.ERR_UNSUPPORTED
+    big = hs2.Shape.make(1 << 28, 8, 2)
+    lens8 = (C.c_int64 * 8)(*([10] * 8))
+    assert L.hs2_block_decode(8, lens8, ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr,
+                              ok_ptr, 0, C.cast(arr, C.POINTER(C.c_void_p)),
+                              C.cast(arr, C.POINTER(C.c_void_p)), C.byref(big), ok_ptr, 1 << 40,
+                              None) == hs2.ERR_UNSUPPORTED
+    with pytest.raises(hs2.HS2Error):
+        hs2.workspace_size(hs2.OP_BLOCK_DECODE, sd, 65)
     assert hs2.hs2_status_string(hs2.ERR_TIMEOUT) == "device-side wait timed out"
+    assert hs2.hs2_status_string(hs2.ERR_BAD_INDEX) == "index list entry out of range (skipped)"
 
 
 def test_workspace_size_queries(hs2):
