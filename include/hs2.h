@@ -169,7 +169,7 @@ hs2_status hs2_select_topk(const hs2_bf16* Q, const hs2_bf16* K, const float* ls
  *     overlap on the same device, e.g. on two streams, race on it: serialise
  *     them.
  *   - The kernel runs as many persistent CTAs as the scratch holds; each needs
- *     4 * (128 / G) * max(2 * k_global, 256) * 8 + 131072 bytes.  A shape for
+ *     4 * (128 / G) * max(2 * k_global, 256) * 8 + 262144 bytes.  A shape for
  *     which one CTA does not fit returns HS2_ERR_UNSUPPORTED.
  * Errors otherwise as hs2_select_topk (HS2_ERR_CUDA if the address lookup
  * fails).
@@ -259,6 +259,16 @@ size_t hs2_workspace_size(int32_t op, const hs2_shape* shape, int32_t batch, int
  * out-of-range index entry as HS2_ERR_BAD_INDEX; CUDA errors as
  * HS2_ERR_CUDA. */
 hs2_status hs2_get_device_status(void* stream);
+
+/* Testing hook, not part of the block: sets the spin budget (GPU clock
+ * cycles) of every bounded wait in the library's kernels on the current
+ * device, for launches that follow; cycles <= 0 restores the default of
+ * 2^31.  A tiny budget makes waits run out, so a test can check that the
+ * kernels unwind cleanly (they first wait, with a fixed budget, for their own
+ * copies and MMAs in flight, then release tensor memory and exit) and that
+ * hs2_get_device_status() reports HS2_ERR_TIMEOUT.  Synchronous; not for use
+ * while library kernels run. */
+hs2_status hs2_debug_set_wait_budget(int64_t cycles);
 
 /* Static English text for a status code. */
 const char* hs2_status_string(hs2_status status);

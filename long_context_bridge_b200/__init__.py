@@ -70,6 +70,8 @@ def _load(path: str = LIB_PATH):
     L.hs2_status_string.argtypes = [C.c_int]
     L.hs2_status_string.restype = C.c_char_p
     L.hs2_kernel_launches.restype = C.c_uint64
+    L.hs2_debug_set_wait_budget.argtypes = [C.c_int64]
+    L.hs2_debug_set_wait_budget.restype = C.c_int
     return L
 
 
@@ -78,7 +80,8 @@ _lib = _load()
 EXPORTED = ["hs2_bridge_kv", "hs2_bridge_kv_fp8", "hs2_full_attn_lse", "hs2_select_topk", "hs2_select_topk_noalloc",
             "hs2_sparse_attn", "hs2_sparse_attn_layers",
             "hs2_block_prefill", "hs2_block_decode", "hs2_workspace_size",
-            "hs2_get_device_status", "hs2_status_string", "hs2_kernel_launches"]
+            "hs2_get_device_status", "hs2_status_string", "hs2_kernel_launches",
+            "hs2_debug_set_wait_budget"]
 
 
 def _ptr(t, dtype, what, nullable=False):
@@ -209,6 +212,11 @@ def hs2_block_decode(seq_len, q_full, Kc, Vc, k_scale, v_scale, o_full, lse, idx
 
 def hs2_get_device_status(stream=None) -> int:
     return int(_lib.hs2_get_device_status(_stream(stream)))
+
+
+def hs2_debug_set_wait_budget(cycles: int) -> None:
+    """Testing hook: spin budget of the kernels' bounded waits (<= 0: default)."""
+    _check(_lib.hs2_debug_set_wait_budget(int(cycles)), "hs2_debug_set_wait_budget")
 
 
 def hs2_kernel_launches() -> int:

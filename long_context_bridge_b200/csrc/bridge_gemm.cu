@@ -20,6 +20,7 @@
 namespace hs2 {
 
 HS2_STATUS_ACCESSOR(status_bridge)
+HS2_BUDGET_SETTER(budget_bridge)
 
 
 namespace {
@@ -77,6 +78,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ---------------- TMA producer ----------------
     prefetch_tmap(&tmH);
     prefetch_tmap(isV ? &tmWv : &tmWk);
+    int issued = 0;
     for (int kb = 0; kb < num_kb; ++kb) {
       const int s = kb % STAGES;
       if (kb >= STAGES && !mbar_wait(&empty[s], ((kb / STAGES) & 1) ^ 1)) break;
@@ -87,7 +89,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
       for (int c = 0; c < BN / 64; ++c)
         tma_load_2d(sB + c * (BK * 128), isV ? &tmWv : &tmWk, &full[s], nloc + c * 64, kb * BK);
+      issued = kb + 1;
     }
+    // every issued copy lands before the CTA can exit
+    for (int s = 0; s < STAGES; ++s) drain_phase(&full[s], issued > s ? (issued - 1 - s) / STAGES + 1 : 0);
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer ----------------
     bool ok = true;
@@ -108,6 +113,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mma_commit(&empty[s]);
     }
     mma_commit(accbar);
+    mbar_wait_budget(accbar, 0, kDrainBudgetCycles);  // no MMA outlives the TMEM
   } else if (warp >= 2) {
     // ---------------- epilogue ----------------
     const int sub = warp & 3;  // TMEM lanes 32*sub .. 32*sub+31
@@ -206,9 +212,11 @@ __global__ void __launch_bounds__(THREADS, 2)
     prefetch_tmap(&tmH);
     prefetch_tmap(&tmWk);
     prefetch_tmap(&tmWv);
+    int issued = 0;
     for (int kb = 0; kb < num_kb; ++kb) {
       const int s = kb % F_STAGES;
       if (kb >= F_STAGES && !mbar_wait(&empty[s], ((kb / F_STAGES) & 1) ^ 1)) break;
+      issued = kb + 1;
       uint8_t* sA = smem + s * F_STAGE_BYTES;
       uint8_t* sBk = sA + F_A_BYTES;
       uint8_t* sBv = sBk + F_B_BYTES;
@@ -220,6 +228,8 @@ __global__ void __launch_bounds__(THREADS, 2)
         tma_load_2d(sBv + c * (BK * 128), &tmWv, &full[s], g * 128 + c * 64, kb * BK);
       }
     }
+    for (int s = 0; s < F_STAGES; ++s)
+      drain_phase(&full[s], issued > s ? (issued - 1 - s) / F_STAGES + 1 : 0);
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer ----------------
     bool ok = true;
@@ -240,6 +250,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       mma_commit(&empty[s]);
     }
     mma_commit(accbar);
+    mbar_wait_budget(accbar, 0, kDrainBudgetCycles);  // no MMA outlives the TMEM
   } else if (warp >= 2) {
     // ---------------- epilogue: one thread per token ----------------
     const int sub = warp & 3;  // TMEM lanes 32*sub .. 32*sub+31

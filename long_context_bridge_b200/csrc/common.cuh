@@ -34,8 +34,20 @@ __device__ __forceinline__ void set_dev_status(unsigned code) {
   atomicOr(&g_dev_status, code);
 }
 
-// Spin budget for one wait: ~2^31 cycles (about a second at 1.9 GHz).
+// Spin budget for one wait: ~2^31 cycles (about a second at 1.9 GHz) unless a
+// test shortens it through hs2_debug_set_wait_budget (each translation unit
+// has its own copy, set through HS2_BUDGET_SETTER).
 constexpr long long kWaitBudgetCycles = 1ll << 31;
+static __device__ long long g_wait_budget = kWaitBudgetCycles;
+
+#define HS2_BUDGET_SETTER(fn)                                                         \
+  cudaError_t fn(long long cycles) {                                                 \
+    return cudaMemcpyToSymbol(g_wait_budget, &cycles, sizeof(cycles));               \
+  }
+
+// Budget of the waits that drain a kernel's own copies and MMAs before it
+// exits after a timeout: those complete on their own, so this one is fixed.
+constexpr long long kDrainBudgetCycles = 1ll << 31;
 
 // ---------------------------------------------------------------------------
 // shared memory addresses
@@ -83,16 +95,30 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Wait for phase `parity` of `bar` to complete.  Returns false (and records
 // DEV_TIMEOUT) if it has not completed within the cycle budget.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_budget(uint64_t* bar, uint32_t parity,
+                                                 long long budget) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitBudgetCycles) {
+    if (clock64() - t0 > budget) {
       set_dev_status(DEV_TIMEOUT);
       return false;
     }
   }
   return true;
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_budget(bar, parity, *const_cast<volatile long long*>(&g_wait_budget));
+}
+
+// Before a kernel that may have timed out exits: wait until the last phase
+// a producer armed on `bar` (its n-th use, n >= 1) has completed, i.e. its
+// asynchronous copies have landed.  Use n of a barrier is only armed after
+// use n-1 completed, so only the last one can be pending.
+__device__ __forceinline__ void drain_phase(uint64_t* bar, uint32_t n) {
+  if (n > 0) mbar_wait_budget(bar, (n - 1) & 1, kDrainBudgetCycles);
 }
 
 // ---------------------------------------------------------------------------
@@ -172,6 +198,14 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
           smem_u32(bar))
       : "memory");
+}
+
+// The MMA issuer's last act: wait (fixed budget) until every tcgen05 op it
+// issued has completed, so that TMEM is never released under a running MMA.
+// `bar` is a barrier of count 1 used for nothing else.
+__device__ __forceinline__ void mma_drain(uint64_t* bar) {
+  mma_commit(bar);
+  mbar_wait_budget(bar, 0, kDrainBudgetCycles);
 }
 
 // Instruction descriptor for kind::f16: bf16 A/B, fp32 D, dense.

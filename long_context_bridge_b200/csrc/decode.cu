@@ -42,6 +42,7 @@
 namespace hs2 {
 
 HS2_STATUS_ACCESSOR(status_decode)
+HS2_BUDGET_SETTER(budget_decode)
 
 namespace {
 
@@ -152,11 +153,13 @@ __global__ void __launch_bounds__((DP_WARPS + 1) * 32, 3)
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
     }
+    int issued = 0;
     for (int si = 0; si < n_st; ++si) {
       const int slot = si % DSTAGES;
       bool go = true;
       if (lane == 0 && si >= DSTAGES) go = mbar_wait(&empty[slot], ((si / DSTAGES) & 1) ^ 1);
       if (!__shfl_sync(0xffffffffu, go, 0)) break;
+      issued = si + 1;
       const int64_t kbase = c_lo + int64_t(si) * DSTAGE_KEYS;
 #pragma unroll
       for (int u = 0; u < DSTAGE_KEYS / 32; ++u) {
@@ -175,6 +178,12 @@ __global__ void __launch_bounds__((DP_WARPS + 1) * 32, 3)
         tma_load_3d(st + DSTAGE_KEYS * 128, &tmV, &full[slot], 0, g, z);
       }
     }
+    // every issued copy (TMA tiles and every lane's scales) lands before the
+    // CTA can exit
+    if (lane == 0)
+      for (int sl = 0; sl < DSTAGES; ++sl)
+        drain_phase(&full[sl], issued > sl ? (issued - 1 - sl) / DSTAGES + 1 : 0);
+    __syncwarp();
     return;
   }
 

@@ -29,6 +29,7 @@
 namespace hs2 {
 
 HS2_STATUS_ACCESSOR(status_full_attn)
+HS2_BUDGET_SETTER(budget_full_attn)
 
 namespace {
 
@@ -53,6 +54,7 @@ struct Bars {
   uint64_t s_full[2];   // per Q tile
   uint64_t p_full[2];   // per Q tile (128 arrivals)
   uint64_t o_done[2];   // per Q tile (last PV)
+  uint64_t drain;       // the MMA issuer's final commit
   uint32_t tmem_slot;
 };
 
@@ -96,6 +98,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&bars->p_full[s], 128);
       mbar_init(&bars->o_done[s], 1);
     }
+    mbar_init(&bars->drain, 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -118,6 +121,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int c = 0; c < 2; ++c)
           tma_load_3d(smem + OFF_Q + X * TILE_BYTES + c * CHUNK, &tmQ, &bars->q_full, c * 64,
                       g * G, q0[X]);
+      int nk = 0, nv = 0;  // K and V tiles issued
       for (int j = 0; j < n_max; ++j) {
         const int s = j & 1;
         const uint32_t ph = ((j >> 1) & 1) ^ 1;
@@ -126,11 +130,19 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int c = 0; c < 2; ++c)
           tma_load_3d(smem + OFF_K + s * TILE_BYTES + c * CHUNK, &tmK, &bars->k_full[s], c * 64,
                       g, j * TILE);
+        nk = j + 1;
         if (j >= 2 && !mbar_wait(&bars->v_empty[s], ph)) break;
         mbar_arrive_expect_tx(&bars->v_full[s], TILE_BYTES);
         for (int c = 0; c < 2; ++c)
           tma_load_3d(smem + OFF_V + s * TILE_BYTES + c * CHUNK, &tmV, &bars->v_full[s], c * 64,
                       g, j * TILE);
+        nv = j + 1;
+      }
+      // every issued copy lands before the CTA can exit
+      drain_phase(&bars->q_full, 1);
+      for (int s = 0; s < 2; ++s) {
+        drain_phase(&bars->k_full[s], nk > s ? (nk - 1 - s) / 2 + 1 : 0);
+        drain_phase(&bars->v_full[s], nv > s ? (nv - 1 - s) / 2 + 1 : 0);
       }
     }
   } else if (warp == 1) {
@@ -186,6 +198,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           mma_commit(&bars->k_empty[(j + 1) & 1]);
         }
       }
+      mma_drain(&bars->drain);  // no MMA outlives the TMEM
     }
   } else {
     // -------------------------------- softmax -------------------------------

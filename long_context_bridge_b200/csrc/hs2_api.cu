@@ -154,6 +154,15 @@ hs2_status hs2_get_device_status(void* stream) {
   return HS2_OK;
 }
 
+hs2_status hs2_debug_set_wait_budget(int64_t cycles) {
+  const long long c = cycles > 0 ? static_cast<long long>(cycles) : kWaitBudgetCycles;
+  cudaError_t e = budget_bridge(c);
+  if (e == cudaSuccess) e = budget_full_attn(c);
+  if (e == cudaSuccess) e = budget_select(c);
+  if (e == cudaSuccess) e = budget_decode(c);
+  return cuda_status(e);
+}
+
 size_t hs2_workspace_size(int32_t op, const hs2_shape* s, int32_t batch, int32_t d_model) {
   (void)d_model;
   const bool sel = op == HS2_OP_SELECT || op == HS2_OP_BLOCK_PREFILL || op == HS2_OP_BLOCK_DECODE;

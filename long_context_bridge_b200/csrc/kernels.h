@@ -18,6 +18,12 @@ unsigned status_select(bool clear);
 unsigned status_sparse(bool clear);
 unsigned status_decode(bool clear);
 
+// spin budget (cycles) of the bounded waits in each kernel file (testing)
+cudaError_t budget_bridge(long long cycles);
+cudaError_t budget_full_attn(long long cycles);
+cudaError_t budget_select(long long cycles);
+cudaError_t budget_decode(long long cycles);
+
 // Tensor maps (bf16, 128-byte swizzle, zero fill out of bounds).
 // dims/strides: x fastest; strides in bytes for dims 1.. .
 bool make_tmap_2d(CUtensorMap* map, const void* base, uint64_t dim_x, uint64_t dim_y,

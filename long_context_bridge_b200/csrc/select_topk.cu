@@ -13,35 +13,48 @@
 //              N = 128 (query, head) rows) into one of four TMEM buffers
 //   warps 2-17 scorers, four per TMEM lane quarter: thread = key (TMEM lane);
 //              scorer warp 4s + r takes the s-th quarter of the item's queries
-//              (TMEM columns 32s .. 32s + 31) for keys 32r .. 32r + 31; a
-//              thread sums exp2(s*scale*log2e - lse2) over each query's G
-//              heads in registers, so a query's score needs no shuffles.
+//              (TMEM columns 32s .. 32s + 31) for keys 32r .. 32r + 31.
+// Exact pruning before any exponential: a candidate can only enter the top k
+// if its score reaches the query's floor F (below).  With y_h = log2 of head
+// h's probability over F, score / F = sum_h 2^y_h.  Each 2^y_h is bounded from
+// above by its chord between integers, 2^floor(y) (1 + frac(y)) (2^y is
+// convex), which the FMA and integer pipes evaluate from the float bits of
+// y + 96 with no exponential; the bound is at most 6.2% above 2^y.  Only
+// candidates whose summed bounds reach the floor survive; their G logits are
+// staged in shared memory and their exact scores, sum_h exp2(s*scale*log2e -
+// lse2), are computed 32 at a time by full warps.
 // Streaming exact top-k without CTA barriers in the tile loop:
-//   * every scorer warp appends the candidates of its 32 keys to its own
-//     per-query sub-buffer (ballot order = ascending position); the four
-//     warps of a query's quarter hold disjoint key sets;
+//   * every scorer warp appends the survivors of its 32 keys whose exact
+//     score reaches the floor to its own per-query sub-buffer; the four warps
+//     of a query's quarter hold disjoint key sets;
 //   * every append is also counted in a per-query histogram of score bins
 //     (eighths of a binade below the largest possible score G) in shared
 //     memory; whatever snapshot of it a warp reads, the highest bin with at
 //     least k appended entries at or above it bounds the k-th best score from
-//     below, so candidates in lower bins are dropped.  The bin floor is shared
-//     by the warps (atomicMax) and only rises;
-//   * a full sub-buffer drops its entries below the floor (stable), or, if
-//     that is not enough, keeps its own exact k best;
+//     below, so that bin's lower edge is a valid floor.  One warp owns each
+//     query's floor, which only rises;
+//   * a sub-buffer about to overflow drops its entries below the floor, or,
+//     if that is not enough, keeps its own exact k best;
 //   * at the end of the item one warp per query selects the k best of the
 //     union of the four sub-buffers on the 64-bit key
 //     (score bits << 32 | ~position), larger score first and equal scores to
-//     the smaller position: a bin histogram fixes the k-th best's bin, radix
-//     digits resolve inside that bin only, and the chosen positions are
-//     sorted ascending by a register bitonic sort.
+//     the smaller position: the append histogram gives the k-th best's bin
+//     (a counting pass rebuilds it if entries were dropped), one pass takes
+//     every entry above that bin and lists the bin's own entries, an exact
+//     radix select over that short list settles the rest (over every entry
+//     if the list is too long), and the chosen positions are sorted
+//     ascending by a bitonic sort.
 // Items whose every query has at most k candidates skip the scoring: all
 // candidates are selected.
+#include <cstddef>
+
 #include "common.cuh"
 #include "kernels.h"
 
 namespace hs2 {
 
 HS2_STATUS_ACCESSOR(status_select)
+HS2_BUDGET_SETTER(budget_select)
 
 namespace {
 
@@ -59,6 +72,11 @@ constexpr int NSB = 4;          // S^T buffers in TMEM (128 columns each)
 constexpr uint32_t IDESC = idesc_bf16(128, 128, 0, 0);
 constexpr float kLog2e = 1.4426950408889634f;
 
+constexpr int STG = 64;             // staged survivors per scorer warp
+constexpr int kRefresh = 4;         // tiles between floor refreshes (a power of two)
+constexpr int kBoundaryCap = 1024;  // boundary-bin entries per final select in scratch
+constexpr int kSortWords = 2048 + 2 * kBoundaryCap;  // per-warp sort scratch (32-bit words)
+
 template <int G>
 struct SelCfg {
   static constexpr int QT = TILE / G;                 // queries per item
@@ -71,6 +89,7 @@ struct Bars {
   uint64_t q_full, q_empty;
   uint64_t k_full[MAX_STAGES], k_empty[MAX_STAGES];
   uint64_t s_full[NSB], s_empty[NSB];
+  uint64_t drain;  // the MMA issuer's final commit
   uint32_t tmem_slot;
 };
 
@@ -78,12 +97,27 @@ template <int G>
 struct Misc {
   static constexpr int QT = SelCfg<G>::QT, NB = SelCfg<G>::NB;
   Bars bars;
-  float lse2[128];            // base-2 lse of the item's 128 (query, head) rows
+  alignas(16) float lse2[128];   // base-2 lse of the item's 128 (query, head) rows
+  alignas(16) float nbeta[128];  // 96 - lse2 - log2(floor) per row: the chord test's offset
   uint32_t floor_bits[QT];    // candidates need score bits >= floor_bits (a bin's lower edge)
+  uint32_t compacted[QT];     // a sub-buffer of the query dropped entries (hist inexact)
   uint32_t cnt[4][QT];        // entries in each sub-buffer
   uint32_t hist[QT][NB];      // appended entries per score bin
-  uint32_t dig[SCORER_WARPS][256];  // per-warp radix histograms of the final select
+  uint32_t dig[SCORER_WARPS][256];  // per-warp radix histograms
+  alignas(16) float stg_x[SCORER_WARPS][STG][G];  // staged survivors: their G logits,
+  int32_t stg_pos[SCORER_WARPS][STG]; // key position
+  uint8_t stg_q[SCORER_WARPS][STG];   // and query of the warp's set
 };
+
+// 16-byte vector accesses to the staged logits and the chord offsets
+template <int G>
+constexpr bool misc_aligned() {
+  return offsetof(Misc<G>, stg_x) % 16 == 0 && offsetof(Misc<G>, nbeta) % 16 == 0 &&
+         offsetof(Misc<G>, lse2) % 16 == 0 && sizeof(Misc<G>) % 16 == 0;
+}
+static_assert(misc_aligned<1>() && misc_aligned<2>() && misc_aligned<4>() && misc_aligned<8>() &&
+                  misc_aligned<16>(),
+              "shared-memory layout of the selection kernel");
 
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int ks) {
   return sdesc_sw128(tile + (ks >> 2) * CHUNK + (ks & 3) * 32, 16, 1024);
@@ -277,6 +311,21 @@ __device__ __forceinline__ void warp_sort1024(uint32_t (&v)[32], int lane) {
   }
 }
 
+// Chord upper bound of 2^y for t = y + 96 with y in [-32, 32): the float
+// whose exponent is floor(y) and whose mantissa is frac(y), 2^floor(y) *
+// (1 + frac(y)) >= 2^y (2^y is convex, the chord between integers lies above
+// it, at most 6.2% above).  t in [64, 128) holds y + 32 in its mantissa with
+// 17 fractional bits, so shifting its bits left by 6 and adding a constant
+// gives the bits of the chord value.  Callers clamp t to at least 64 (y >= -32).
+__device__ __forceinline__ float chord_exp2(float t) {
+  return __uint_as_float((__float_as_uint(t) << 6) + 0x8F800000u);
+}
+
+// A candidate's chord bounds must reach at least this fraction of the floor
+// for its exact score to be computed: the bound is an upper bound up to fp32
+// rounding (relative ~1e-5), far inside this margin.
+constexpr float kChordPass = 1.0f - 1.0f / 1024.0f;
+
 template <int G>
 __global__ void __launch_bounds__(THREADS, 1)
     select_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -321,6 +370,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&br->s_full[b], 1);
       mbar_init(&br->s_empty[b], SCORERS);
     }
+    mbar_init(&br->drain, 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -336,7 +386,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       // ------------------------------ producer ------------------------------
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
-      uint32_t kt = 0, qn = 0;
+      uint32_t kt = 0, qn = 0, q_issued = 0;
       bool ok = true;
       for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
         int q0, g, n_tiles;
@@ -347,6 +397,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         mbar_arrive_expect_tx(&br->q_full, TILE_BYTES);
         for (int c = 0; c < 2; ++c)
           tma_load_3d(smem + OFF_Q + c * CHUNK, &tmQ, &br->q_full, c * 64, g * G, q0);
+        ++q_issued;
         for (int t = 0; t < n_tiles; ++t, ++kt) {
           const int s = kt % kst;
           if (kt >= uint32_t(kst) && !mbar_wait(&br->k_empty[s], ((kt / kst) & 1) ^ 1)) {
@@ -360,6 +411,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         ++qn;
       }
+      // every issued copy lands before the CTA can exit (kt counts the K
+      // tiles issued: a timed-out wait leaves the loop before the increment)
+      drain_phase(&br->q_full, q_issued);
+      for (int s = 0; s < kst; ++s)
+        drain_phase(&br->k_full[s], kt > uint32_t(s) ? (kt - 1 - s) / kst + 1 : 0);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -388,6 +444,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         mma_commit(&br->q_empty);
         ++qn;
       }
+      mma_drain(&br->drain);  // no MMA outlives the TMEM
     }
   } else {
     // -------------------------------- scorers -------------------------------
@@ -398,6 +455,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t lane_addr = uint32_t(sub * 32) << 16;
     const uint32_t lt_mask = (1u << lane) - 1u;
     uint2* my_bufs = ws + (size_t(blockIdx.x) * 4 + sub) * QT * capw;  // [QT][capw]
+    float* stx = &ms->stg_x[sw][0][0];
+    int32_t* stp = ms->stg_pos[sw];
+    uint8_t* stq = ms->stg_q[sw];
+    const uint64_t c2 = f2(scale_log2, scale_log2);
     uint32_t st = 0;
     bool ok = true;
     for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
@@ -407,17 +468,88 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (tid < 128) {
         const int qrow = q0 + tid / G;
         ms->lse2[tid] = qrow < T ? lse[size_t(qrow) * Hq + g * G + tid % G] * kLog2e : INFINITY;
+        ms->nbeta[tid] = INFINITY;  // floor 0: every candidate passes the chord test
       }
       for (int i = tid; i < QT; i += SCORERS) {
         ms->floor_bits[i] = 0;
+        ms->compacted[i] = 0;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) ms->cnt[v][i] = 0;
       }
       for (int i = tid; i < QT * NB; i += SCORERS) (&ms->hist[0][0])[i] = 0;
       const int qb0 = half * QH;        // this warp's queries: qb0 .. qb0 + QH - 1
       const int qvalid = T - q0 - qb0;  // of which those below qvalid exist
-      uint32_t n[QH];                   // entries in this warp's sub-buffers
-#pragma unroll
-      for (int ql = 0; ql < QH; ++ql) n[ql] = 0;
       scorer_sync();
+
+      // ms->nbeta[c] = 96 - lse2 - log2(floor) of column c = (query, head):
+      // t = s * scale_log2 + nbeta = y + 96, y = log2(p_head / floor)
+      const float* nbw = &ms->nbeta[half * 32];
+
+      // make room in this warp's sub-buffer of query q: drop entries below
+      // the floor (stable), or, if that is not enough, keep its own exact k
+      // best (they contain its part of the top k)
+      auto make_room = [&](int q) {
+        __syncwarp();
+        uint2* buf = my_bufs + size_t(q) * capw;
+        const uint32_t fl = ms->floor_bits[q];
+        uint32_t n = warp_compact(buf, ms->cnt[sub][q], lane, [&](uint2 v) { return v.x >= fl; });
+        if (n + 32 > uint32_t(capw) / 2 + k / 2 && n > uint32_t(k)) {
+          uint2* one[4] = {buf, buf, buf, buf};
+          const uint32_t nn[4] = {n, 0, 0, 0};
+          uint64_t pf, mk;
+          radix_select<NB, BSHIFT>(one, nn, k, lo, ms->dig[sw], lane, pf, mk);
+          n = warp_compact(buf, n, lane, [&](uint2 v) { return (sel_key(v) & mk) >= pf; });
+        }
+        if (lane == 0) {
+          ms->cnt[sub][q] = n;
+          ms->compacted[q] = 1;
+        }
+        __syncwarp();
+      };
+
+      // exact scores of staged survivors base .. base + cnt - 1 (one per
+      // lane) and their appends
+      auto process = [&](int base, int cnt) {
+        const bool act = lane < cnt;
+        const int e = base + (act ? lane : 0);
+        float x[G];
+        if constexpr (G % 4 == 0) {
+#pragma unroll
+          for (int h = 0; h < G; h += 4) {
+            const float4 v = *reinterpret_cast<const float4*>(stx + e * G + h);
+            x[h] = v.x;
+            x[h + 1] = v.y;
+            x[h + 2] = v.z;
+            x[h + 3] = v.w;
+          }
+        } else {
+#pragma unroll
+          for (int h = 0; h < G; ++h) x[h] = stx[e * G + h];
+        }
+        const int ql = stq[e];
+        const int jj = stp[e];
+        const float* l2 = &ms->lse2[half * 32 + ql * G];
+        float acc = 0.f;
+#pragma unroll
+        for (int h = 0; h < G; ++h) acc += fast_exp2(fmaf(x[h], scale_log2, -l2[h]));
+        const int q = qb0 + ql;
+        const uint32_t bits = __float_as_uint(acc);
+        const bool risk = act && ms->cnt[sub][q] + 32 > uint32_t(capw);
+        uint32_t rb = __ballot_sync(0xffffffffu, risk);
+        while (rb != 0) {  // rare: a sub-buffer this batch could overflow
+          const int qr = __shfl_sync(0xffffffffu, ql, __ffs(rb) - 1);
+          make_room(qb0 + qr);
+          rb &= ~__ballot_sync(0xffffffffu, ql == qr);
+        }
+        if (act && bits >= ms->floor_bits[q]) {
+          const uint32_t pos = atomicAdd(&ms->cnt[sub][q], 1u);
+          my_bufs[size_t(q) * capw + pos] = make_uint2(bits, uint32_t(jj));
+          atomicAdd(&ms->hist[q][bin_of<NB, BSHIFT>(bits, lo)], 1u);
+        }
+        __syncwarp();
+      };
+
+      int nst = 0;  // staged survivors of this warp (the same in every lane)
       for (int t = 0; t < n_tiles; ++t, ++st) {
         const int b = st % NSB;
         ok = ok && mbar_wait(&br->s_full[b], (st / NSB) & 1);
@@ -426,82 +558,88 @@ __global__ void __launch_bounds__(THREADS, 1)
         // candidate test for query qb0 + ql: j + w <= its position, i.e.
         // dpos <= ql, and the query inside the sequence (ql < qvalid)
         const int dpos = j + w - q0 - qb0;
-        float sc[QH];
-        {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_addr + b * 128 + half * 32, r);
-          tmem_wait_ld();
-          tc_fence_before();
-          mbar_arrive(&br->s_empty[b]);
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_addr + b * 128 + half * 32, r);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&br->s_empty[b]);
+        // chord upper bound of each query's score relative to its floor
+        float qsum[QH];
 #pragma unroll
-          for (int qq = 0; qq < QH; ++qq) {
-            float acc = 0.f;
+        for (int qq = 0; qq < QH; ++qq) {
+          if constexpr (G == 1) {
+            qsum[qq] = chord_exp2(fmaxf(fmaf(__uint_as_float(r[qq]), scale_log2, nbw[qq]), 64.f));
+          } else {
+            uint64_t a2 = f2(0.f, 0.f);
 #pragma unroll
-            for (int h = 0; h < G; ++h)
-              acc += fast_exp2(fmaf(__uint_as_float(r[qq * G + h]), scale_log2,
-                                    -ms->lse2[half * 32 + qq * G + h]));
-            sc[qq] = acc;
+            for (int h = 0; h < G; h += 2) {
+              const int c = qq * G + h;
+              const float2 nb2 = *reinterpret_cast<const float2*>(nbw + c);
+              float t0, t1;
+              f2_split(f2_fma(f2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), c2,
+                              f2(nb2.x, nb2.y)),
+                       t0, t1);
+              a2 = f2_add(a2, f2(chord_exp2(fmaxf(t0, 64.f)), chord_exp2(fmaxf(t1, 64.f))));
+            }
+            float s0, s1;
+            f2_split(a2, s0, s1);
+            qsum[qq] = s0 + s1;
           }
         }
-        uint32_t bal[QH], anymask = 0;
+        // stage the survivors' logits; exact scores in full warps
 #pragma unroll
-        for (int ql = 0; ql < QH; ++ql) {
-          const bool pass = dpos <= ql && ql < qvalid &&
-                            __float_as_uint(sc[ql]) >= ms->floor_bits[qb0 + ql];
-          bal[ql] = __ballot_sync(0xffffffffu, pass);
-          anymask |= uint32_t(bal[ql] != 0) << ql;
-        }
-        if (anymask != 0) {
+        for (int qq = 0; qq < QH; ++qq) {
+          const bool p = dpos <= qq && qq < qvalid && qsum[qq] >= kChordPass;
+          const uint32_t bal = __ballot_sync(0xffffffffu, p);
+          if (bal == 0) continue;
+          if (p) {
+            const int slot = nst + __popc(bal & lt_mask);
+            float* dst = stx + slot * G;
+            if constexpr (G % 4 == 0) {
 #pragma unroll
-          for (int ql = 0; ql < QH; ++ql) {
-            if (!((anymask >> ql) & 1u) || n[ql] + 32 <= uint32_t(capw)) continue;
-            // make room: drop entries below the current floor, else keep the
-            // sub-buffer's own k best (they contain its part of the top k)
+              for (int h = 0; h < G; h += 4)
+                *reinterpret_cast<float4*>(dst + h) =
+                    make_float4(__uint_as_float(r[qq * G + h]), __uint_as_float(r[qq * G + h + 1]),
+                                __uint_as_float(r[qq * G + h + 2]),
+                                __uint_as_float(r[qq * G + h + 3]));
+            } else {
+#pragma unroll
+              for (int h = 0; h < G; ++h) dst[h] = __uint_as_float(r[qq * G + h]);
+            }
+            stp[slot] = j;
+            stq[slot] = uint8_t(qq);
+          }
+          nst += __popc(bal);
+          if (nst >= 32) {
             __syncwarp();
-            const int q = qb0 + ql;
-            uint2* buf = my_bufs + size_t(q) * capw;
-            const uint32_t fl = ms->floor_bits[q];
-            n[ql] = warp_compact(buf, n[ql], lane, [&](uint2 v) { return v.x >= fl; });
-            if (n[ql] + 32 > uint32_t(capw) / 2 + k / 2 && n[ql] > uint32_t(k)) {
-              uint2* one[4] = {buf, buf, buf, buf};
-              const uint32_t nn[4] = {n[ql], 0, 0, 0};
-              uint64_t pf, mk;
-              radix_select<NB, BSHIFT>(one, nn, k, lo, ms->dig[sw], lane, pf, mk);
-              n[ql] = warp_compact(buf, n[ql], lane,
-                                   [&](uint2 v) { return (sel_key(v) & mk) >= pf; });
-            }
-          }
-          // append in position order; count the appends per score bin
-#pragma unroll
-          for (int ql = 0; ql < QH; ++ql) {
-            if ((bal[ql] >> lane) & 1u) {
-              const int q = qb0 + ql;
-              const uint32_t bits = __float_as_uint(sc[ql]);
-              my_bufs[size_t(q) * capw + n[ql] + __popc(bal[ql] & lt_mask)] =
-                  make_uint2(bits, uint32_t(j));
-              atomicAdd(&ms->hist[q][bin_of<NB, BSHIFT>(bits, lo)], 1u);
-            }
-            n[ql] += __popc(bal[ql]);
+            process(nst - 32, 32);
+            nst -= 32;
           }
         }
         // raise the floors of this warp's queries to the highest bin with at
         // least k appended entries at or above it (any snapshot of the counts
-        // gives a valid floor)
-        if ((t & 3) == 3 || t == n_tiles - 1) {
+        // gives a valid floor), then reload the chord offsets of its columns
+        if ((t & (kRefresh - 1)) == kRefresh - 1) {
           for (int q = half * QH + sub; q < (half + 1) * QH; q += 4) {
             uint32_t above, inbin;
             const int fb = hist_cross<NB>(ms->hist[q], uint32_t(k), lane, above, inbin);
-            if (fb > 0 && lane == 0) atomicMax(&ms->floor_bits[q], (uint32_t(fb) + lo) << BSHIFT);
+            const uint32_t fbits = fb > 0 ? (uint32_t(fb) + lo) << BSHIFT : 0u;
+            if (fbits > ms->floor_bits[q]) {
+              __syncwarp();
+              if (lane == 0) ms->floor_bits[q] = fbits;
+              const float L = __log2f(__uint_as_float(fbits));
+              if (lane < G) ms->nbeta[q * G + lane] = 96.f - ms->lse2[q * G + lane] - L;
+            }
           }
+          __syncwarp();
         }
       }
-      if (lane == 0) {
-#pragma unroll
-        for (int ql = 0; ql < QH; ++ql) ms->cnt[sub][qb0 + ql] = n[ql];
-      }
+      __syncwarp();
+      if (nst > 0) process(0, nst);
       scorer_sync();
       // ---- outputs of the item: one warp per query ----
-      uint32_t* sp = wsort + (size_t(blockIdx.x) * SCORER_WARPS + sw) * 2048;  // staging
+      uint32_t* sp = wsort + (size_t(blockIdx.x) * SCORER_WARPS + sw) * kSortWords;  // positions
+      uint2* bl = reinterpret_cast<uint2*>(sp + 2048);                               // boundary bin
       for (int q = sw; q < QT; q += SCORER_WARPS) {
         const int qpos = q0 + q;
         if (qpos >= T) continue;
@@ -512,31 +650,106 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int e = lane; e < k; e += 32) out[e] = e < ncand ? e : -1;
         } else {
           uint2* sb[4];
-          uint32_t nb[4];
+          uint32_t nbv[4];
           for (int v = 0; v < 4; ++v) {
             sb[v] = ws + ((size_t(blockIdx.x) * 4 + v) * QT + q) * capw;
-            nb[v] = ms->cnt[v][q];
+            nbv[v] = ms->cnt[v][q];
           }
-          uint64_t pf = 0, mk = 0;
-          if (ok) radix_select<NB, BSHIFT>(sb, nb, k, lo, ms->dig[sw], lane, pf, mk);
-          // gather the chosen positions (each list is in position order)
-          uint32_t got = 0, mn = 0xFFFFFFFFu;
-          for (int v = 0; v < 4; ++v) {
-            for (uint32_t base = 0; base < nb[v]; base += 32) {
-              const uint32_t e = base + lane;
-              uint2 x = make_uint2(0u, 0u);
-              bool sel = false;
-              if (e < nb[v]) {
-                x = sb[v][e];
-                sel = (sel_key(x) & mk) >= pf;
+          // the bin of the k-th best: from the append histogram when every
+          // appended entry is still buffered, else from one counting pass
+          const uint32_t* hq = ms->hist[q];
+          if (ms->compacted[q]) {
+            uint32_t* hd = ms->dig[sw];
+            for (int b2 = lane; b2 < NB; b2 += 32) hd[b2] = 0;
+            __syncwarp();
+            for_each_entry(sb, nbv, lane, [&](uint2 v, bool act, int) {
+              if (act) atomicAdd(&hd[bin_of<NB, BSHIFT>(v.x, lo)], 1u);
+            });
+            __syncwarp();
+            hq = hd;
+          }
+          uint32_t above = 0, inbin = 0;
+          const int bstar = ok ? hist_cross<NB>(hq, uint32_t(k), lane, above, inbin) : -1;
+          __syncwarp();
+          uint32_t got = 0, nbl = 0, mn = 0xFFFFFFFFu;
+          if (bstar >= 0) {
+            const uint32_t need = uint32_t(k) - above;
+            const bool all_in = inbin == need;
+            // one pass: entries above the boundary bin are selected, the
+            // boundary bin's entries go to a list for an exact select
+            for (int v = 0; v < 4; ++v) {
+              for (uint32_t base = 0; base < nbv[v]; base += 32) {
+                const uint32_t e = base + lane;
+                uint2 x = make_uint2(0u, 0u);
+                int bx = -1;
+                if (e < nbv[v]) {
+                  x = sb[v][e];
+                  bx = int(bin_of<NB, BSHIFT>(x.x, lo));
+                }
+                const bool sel = bx > bstar || (all_in && bx == bstar);
+                const bool tob = !all_in && bx == bstar;
+                const uint32_t bs = __ballot_sync(0xffffffffu, sel);
+                const uint32_t bb = __ballot_sync(0xffffffffu, tob);
+                if (sel) {
+                  const uint32_t pos = got + __popc(bs & lt_mask);
+                  if (pos < uint32_t(k)) sp[pos] = x.y;
+                  mn = min(mn, x.x);
+                }
+                if (tob) {
+                  const uint32_t pos = nbl + __popc(bb & lt_mask);
+                  if (pos < uint32_t(kBoundaryCap)) bl[pos] = x;
+                }
+                got += __popc(bs);
+                nbl += __popc(bb);
               }
-              const uint32_t bb = __ballot_sync(0xffffffffu, sel);
-              const uint32_t pos = got + __popc(bb & lt_mask);
-              if (sel && pos < uint32_t(k)) {
-                sp[pos] = x.y;
-                mn = min(mn, x.x);
+            }
+            __syncwarp();
+            if (!all_in && nbl <= uint32_t(kBoundaryCap)) {
+              uint2* one[4] = {bl, bl, bl, bl};
+              const uint32_t nn[4] = {nbl, 0, 0, 0};
+              uint64_t pf, mk;
+              radix_select<NB, BSHIFT>(one, nn, need, lo, ms->dig[sw], lane, pf, mk);
+              for (uint32_t base = 0; base < nbl; base += 32) {
+                const uint32_t e = base + lane;
+                uint2 x = make_uint2(0u, 0u);
+                bool sel = false;
+                if (e < nbl) {
+                  x = bl[e];
+                  sel = (sel_key(x) & mk) >= pf;
+                }
+                const uint32_t bs = __ballot_sync(0xffffffffu, sel);
+                if (sel) {
+                  const uint32_t pos = got + __popc(bs & lt_mask);
+                  if (pos < uint32_t(k)) sp[pos] = x.y;
+                  mn = min(mn, x.x);
+                }
+                got += __popc(bs);
               }
-              got += __popc(bb);
+            }
+          }
+          if (bstar < 0 || (!(inbin == uint32_t(k) - above) && nbl > uint32_t(kBoundaryCap))) {
+            // fall-back: an exact radix select over every buffered entry
+            got = 0;
+            mn = 0xFFFFFFFFu;
+            uint64_t pf = 0, mk = 0;
+            if (ok) radix_select<NB, BSHIFT>(sb, nbv, k, lo, ms->dig[sw], lane, pf, mk);
+            for (int v = 0; v < 4; ++v) {
+              for (uint32_t base = 0; base < nbv[v]; base += 32) {
+                const uint32_t e = base + lane;
+                uint2 x = make_uint2(0u, 0u);
+                bool sel = false;
+                if (e < nbv[v]) {
+                  x = sb[v][e];
+                  sel = (sel_key(x) & mk) >= pf;
+                }
+                const uint32_t bs = __ballot_sync(0xffffffffu, sel);
+                if (sel) {
+                  const uint32_t pos = got + __popc(bs & lt_mask);
+                  if (pos < uint32_t(k)) sp[pos] = x.y;
+                  mn = min(mn, x.x);
+                }
+                got += __popc(bs);
+              }
             }
           }
           got = min(got, uint32_t(k));
@@ -660,12 +873,13 @@ cudaError_t select_scratch_address(void** out) {
 }
 
 // bytes of the file-scope scratch taken by one CTA (the documented figure:
-// 4 * (128 / G) * max(2k, 256) * 8 + 131072)
+// 4 * (128 / G) * max(2k, 256) * 8 + 262144)
 size_t noalloc_cta_bytes(int QT, int k) {
-  return size_t(4) * QT * buffer_cap(k) * sizeof(uint2) + size_t(SCORER_WARPS) * 2048 * sizeof(uint32_t);
+  return size_t(4) * QT * buffer_cap(k) * sizeof(uint2) +
+         size_t(SCORER_WARPS) * kSortWords * sizeof(uint32_t);
 }
-static_assert(size_t(SCORER_WARPS) * 2048 * sizeof(uint32_t) == 131072,
-              "the per-CTA staging term documented for hs2_select_topk_noalloc");
+static_assert(size_t(SCORER_WARPS) * kSortWords * sizeof(uint32_t) == 262144,
+              "the per-CTA sort term documented for hs2_select_topk_noalloc");
 
 template <int G>
 cudaError_t launch_noalloc_g(const SelectArgs& a, void* scratch, cudaStream_t stream) {
@@ -699,7 +913,7 @@ size_t select_workspace_bytes(int64_t T, int Hq, int Hkv, int k, int w) {
   (void)w;
   const int QT = TILE / (Hq / Hkv);
   return size_t(sm_count()) * (size_t(4) * QT * buffer_cap(k) * sizeof(uint2) +
-                               size_t(SCORER_WARPS) * 2048 * sizeof(uint32_t));
+                               size_t(SCORER_WARPS) * kSortWords * sizeof(uint32_t));
 }
 
 size_t select_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }

@@ -8,7 +8,7 @@ import numpy as np
 import pytest
 
 import synth
-from helpers import assert_close_bf16, dev, dev_bf16, host_f64
+from helpers import assert_close_bf16, check_index_lists, dev, dev_bf16, host_f64
 
 pytestmark = pytest.mark.gpu
 RNG = np.random.default_rng(31)
@@ -70,3 +70,85 @@ def test_sparse_attn_skips_out_of_range_entries(hs2, orc, Hq, Hkv):
     assert hs2.hs2_get_device_status() == hs2.ERR_BAD_INDEX
     for x in Os:
         assert_close_bf16(host_f64(x), Oo, "fused layers on lists with bad entries")
+
+
+def test_waits_that_run_out_unwind_and_report(hs2, orc):
+    """With the spin budget of every bounded wait cut to one cycle, the waits
+    of the TMA/tensor-core kernels run out.  Each kernel then waits (with its
+    own fixed budget) for the copies and MMAs it already issued, releases its
+    tensor memory and exits, and the next status read is HS2_ERR_TIMEOUT.
+    With the default budget restored, the same calls in the same process
+    return the oracle's results: the context is still usable."""
+    import torch
+    T, Hq, Hkv, k, w, dm = 1500, 8, 2, 256, 64, 256
+    # the dyadic grid makes the bridge exact in fp32, so the block's K/V equal
+    # the oracle's bit for bit and the oracle runs on its own K/V
+    H, Wk, Wv = synth.bridge_inputs_dyadic_np(
+        synth.BlockConfig("timeouts", 6, T, Hq, Hkv, d_model=dm))
+    Q, Qs = rand_bf16((T, Hq, 128)), rand_bf16((T, Hq, 128))
+    shape = hs2.Shape.make(T, Hq, Hkv, k_global=k, window=w)
+    ws = torch.empty(hs2.workspace_size(hs2.OP_BLOCK_PREFILL, shape), dtype=torch.uint8,
+                     device="cuda")
+    Hd, Wkd, Wvd, Qd, Qsd = dev_bf16(H), dev_bf16(Wk), dev_bf16(Wv), dev_bf16(Q), dev_bf16(Qs)
+
+    def block():
+        K = torch.empty(T, Hkv, 128, dtype=torch.bfloat16, device="cuda")
+        V = torch.empty_like(K)
+        O, Os = torch.empty_like(Qd), torch.empty_like(Qd)
+        lse = torch.empty(T, Hq, dtype=torch.float32, device="cuda")
+        idx = torch.empty(T, Hkv, k + w, dtype=torch.int32, device="cuda")
+        hs2.hs2_block_prefill(Hd, Wkd, Wvd, K, V, Qd, O, lse, idx, [Qsd], [Os], shape, ws)
+        return K, V, O, lse, idx, Os
+
+    def decode():
+        cap, lens = 3000, [3000, 1700]
+        Kc = torch.randint(0, 0x7E, (2, cap, Hkv, 128), dtype=torch.uint8, device="cuda")
+        Vc = torch.randint(0, 0x7E, (2, cap, Hkv, 128), dtype=torch.uint8, device="cuda")
+        S = torch.full((2, cap, Hkv), 1.0 / 256, dtype=torch.float32, device="cuda")
+        sh = hs2.Shape.make(cap, Hq, Hkv, k_global=k, window=w)
+        wsd = torch.empty(hs2.workspace_size(hs2.OP_BLOCK_DECODE, sh, 2), dtype=torch.uint8,
+                          device="cuda")
+        q = torch.randn(2, Hq, 128, device="cuda").bfloat16()
+        o = torch.empty_like(q)
+        hs2.hs2_block_decode(lens, q, Kc, Vc, S, S, o,
+                             torch.empty(2, Hq, dtype=torch.float32, device="cuda"),
+                             torch.empty(2, Hkv, k + w, dtype=torch.int32, device="cuda"), [q],
+                             [torch.empty_like(q)], sh, wsd)
+
+    assert hs2.hs2_get_device_status() == hs2.OK
+    hs2.hs2_debug_set_wait_budget(1)
+    try:
+        block()
+        st_block = hs2.hs2_get_device_status()
+        decode()
+        st_decode = hs2.hs2_get_device_status()
+        K8 = torch.empty(T, Hkv, 128, dtype=torch.uint8, device="cuda")
+        hs2.hs2_bridge_kv_fp8(Hd, Wkd, Wvd, K8, torch.empty_like(K8),
+                              torch.empty(T, Hkv, dtype=torch.float32, device="cuda"),
+                              hs2.Shape.make(T, Hkv, Hkv))
+        st_f8 = hs2.hs2_get_device_status()
+    finally:
+        hs2.hs2_debug_set_wait_budget(0)
+    assert st_block == hs2.ERR_TIMEOUT
+    assert st_decode == hs2.ERR_TIMEOUT
+    assert st_f8 == hs2.ERR_TIMEOUT
+    assert hs2.hs2_get_device_status() == hs2.OK
+    # default budget again: the same block, checked against the oracle
+    K, V, O, lse, idx, Os = block()
+    assert hs2.hs2_get_device_status() == hs2.OK
+    Ko, Vo = orc.bridge(H, Wk).reshape(T, Hkv, 128), orc.bridge(H, Wv).reshape(T, Hkv, 128)
+    assert np.array_equal(K.view(torch.int16).cpu().numpy().view(np.uint16), Ko)
+    assert np.array_equal(V.view(torch.int16).cpu().numpy().view(np.uint16), Vo)
+    kv = orc.KV(Ko, Vo)
+    rows = np.array([0, 63, 64, 319, 320, 777, 1200, T - 1])
+    ref = orc.block_rows(kv, Q[rows], [Qs[rows]], rows, 1 / math.sqrt(128), k, w)
+    assert_close_bf16(host_f64(O[rows]), ref["O"], "O_full after the timeouts")
+    assert np.max(np.abs(lse[rows].cpu().numpy() - ref["lse"])) <= 2e-4
+    gi = idx[rows].cpu().numpy()
+    check_index_lists(gi, ref["idx"], ref["kth"], rows, k, w,
+                      lambda r, g, js: orc.scores(kv, Q[rows][r], g, 1 / math.sqrt(128),
+                                                  ref["lse"][r], js))
+    same = np.all(gi == ref["idx"], axis=(1, 2))
+    assert_close_bf16(host_f64(Os[rows])[same], ref["O_sparse"][0][same], "O_sparse")
+    decode()
+    assert hs2.hs2_get_device_status() == hs2.OK
