@@ -14,15 +14,15 @@
 //   warps 2-17 scorers, four per TMEM lane quarter: thread = key (TMEM lane);
 //              scorer warp 4s + r takes the s-th quarter of the item's queries
 //              (TMEM columns 32s .. 32s + 31) for keys 32r .. 32r + 31.
-// Exact pruning before any exponential: a candidate can only enter the top k
-// if its score reaches the query's floor F (below).  With y_h = log2 of head
-// h's probability over F, score / F = sum_h 2^y_h.  Each 2^y_h is bounded from
-// above by its chord between integers, 2^floor(y) (1 + frac(y)) (2^y is
-// convex), which the FMA and integer pipes evaluate from the float bits of
-// y + 96 with no exponential; the bound is at most 6.2% above 2^y.  Only
-// candidates whose summed bounds reach the floor survive; their G logits are
-// staged in shared memory and their exact scores, sum_h exp2(s*scale*log2e -
-// lse2), are computed 32 at a time by full warps.
+// Pruning before the exact scores: a candidate can only enter the top k if
+// its score reaches the query's floor F (below).  With y_h = log2 of head
+// h's probability over F, score / F = sum_h 2^y_h.  A pre-filter evaluates
+// that sum in half precision, two heads per instruction (FFMA2 for the y
+// pair, one conversion to f16x2, ex2.approx.f16x2, f16x2 adds); its error
+// bound is far inside the 3% margin it is compared with, so it drops no
+// candidate that reaches the floor.  The survivors' G logits are staged in
+// shared memory and their exact scores, sum_h exp2(s*scale*log2e - lse2) in
+// fp32, are computed 32 at a time by full warps.
 // Streaming exact top-k without CTA barriers in the tile loop:
 //   * every scorer warp appends the survivors of its 32 keys whose exact
 //     score reaches the floor to its own per-query sub-buffer; the four warps
@@ -43,7 +43,7 @@
 //     every entry above that bin and lists the bin's own entries, an exact
 //     radix select over that short list settles the rest (over every entry
 //     if the list is too long), and the chosen positions are sorted
-//     ascending by a bitonic sort.
+//     ascending by a bitonic sort held lane-major in registers.
 // Items whose every query has at most k candidates skip the scoring: all
 // candidates are selected.
 #include <cstddef>
@@ -72,7 +72,6 @@ constexpr int NSB = 4;          // S^T buffers in TMEM (128 columns each)
 constexpr uint32_t IDESC = idesc_bf16(128, 128, 0, 0);
 constexpr float kLog2e = 1.4426950408889634f;
 
-constexpr int STG = 64;             // staged survivors per scorer warp
 constexpr int kRefresh = 4;         // tiles between floor refreshes (a power of two)
 constexpr int kBoundaryCap = 1024;  // boundary-bin entries per final select in scratch
 constexpr int kSortWords = 2048 + 2 * kBoundaryCap;  // per-warp sort scratch (32-bit words)
@@ -97,23 +96,19 @@ template <int G>
 struct Misc {
   static constexpr int QT = SelCfg<G>::QT, NB = SelCfg<G>::NB;
   Bars bars;
-  alignas(16) float lse2[128];   // base-2 lse of the item's 128 (query, head) rows
-  alignas(16) float nbeta[128];  // 96 - lse2 - log2(floor) per row: the chord test's offset
+  alignas(16) float nlse2[128];  // minus the base-2 lse of the item's 128 (query, head) rows
   uint32_t floor_bits[QT];    // candidates need score bits >= floor_bits (a bin's lower edge)
   uint32_t compacted[QT];     // a sub-buffer of the query dropped entries (hist inexact)
   uint32_t cnt[4][QT];        // entries in each sub-buffer
-  uint32_t hist[QT][NB];      // appended entries per score bin
-  uint32_t dig[SCORER_WARPS][256];  // per-warp radix histograms
-  alignas(16) float stg_x[SCORER_WARPS][STG][G];  // staged survivors: their G logits,
-  int32_t stg_pos[SCORER_WARPS][STG]; // key position
-  uint8_t stg_q[SCORER_WARPS][STG];   // and query of the warp's set
+  alignas(16) uint32_t hist[QT][NB];  // appended entries per score bin
+  uint32_t dig[SCORER_WARPS][256];    // per-warp radix histograms
 };
 
-// 16-byte vector accesses to the staged logits and the chord offsets
+// 16-byte vector accesses to the histograms and the lse rows
 template <int G>
 constexpr bool misc_aligned() {
-  return offsetof(Misc<G>, stg_x) % 16 == 0 && offsetof(Misc<G>, nbeta) % 16 == 0 &&
-         offsetof(Misc<G>, lse2) % 16 == 0 && sizeof(Misc<G>) % 16 == 0;
+  return offsetof(Misc<G>, nlse2) % 16 == 0 && offsetof(Misc<G>, hist) % 16 == 0 &&
+         sizeof(Misc<G>) % 16 == 0;
 }
 static_assert(misc_aligned<1>() && misc_aligned<2>() && misc_aligned<4>() && misc_aligned<8>() &&
                   misc_aligned<16>(),
@@ -145,12 +140,27 @@ template <int NB>
 __device__ __forceinline__ int hist_cross(const uint32_t* hist, uint32_t need, int lane,
                                           uint32_t& above, uint32_t& inbin) {
   constexpr int PER = NB / 32;
+  static_assert(PER == 2 || PER % 4 == 0, "bins per lane");
+  // lane l owns bins NB-1-PER*l down to NB-PER*(l+1): one contiguous block,
+  // read with vector loads (conflict-free) and taken highest first
   uint32_t c[PER], local = 0;
+  const uint32_t* blk = hist + NB - PER * (lane + 1);
+  if constexpr (PER == 2) {
+    const uint2 v = *reinterpret_cast<const uint2*>(blk);
+    c[0] = v.y;
+    c[1] = v.x;
+  } else {
 #pragma unroll
-  for (int i = 0; i < PER; ++i) {
-    c[i] = hist[NB - 1 - PER * lane - i];
-    local += c[i];
+    for (int i = 0; i < PER; i += 4) {
+      const uint4 v = *reinterpret_cast<const uint4*>(blk + i);
+      c[PER - 1 - i] = v.x;
+      c[PER - 2 - i] = v.y;
+      c[PER - 3 - i] = v.z;
+      c[PER - 4 - i] = v.w;
+    }
   }
+#pragma unroll
+  for (int i = 0; i < PER; ++i) local += c[i];
   uint32_t incl = local;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -277,10 +287,10 @@ __device__ void radix_select(uint2* const* sub, const uint32_t* n, uint32_t k, u
   mask_out = mask;
 }
 
-// Ascending bitonic sort of 1024 values held as v[r] of lane l = element
-// r * 32 + l.  Strides below 32 cross lanes (shuffles), larger ones cross
-// registers of one lane.
-__device__ __forceinline__ void warp_sort1024(uint32_t (&v)[32], int lane) {
+// Ascending bitonic sort of 1024 values held lane-major: v[r] of lane l is
+// element 32 l + r.  The 40 stages with strides below 32 compare registers of
+// one lane; only the 15 stages with larger strides exchange across lanes.
+__device__ __forceinline__ void warp_sort1024_lm(uint32_t (&v)[32], int lane) {
 #pragma unroll
   for (int size = 2; size <= 1024; size <<= 1) {
 #pragma unroll
@@ -288,43 +298,46 @@ __device__ __forceinline__ void warp_sort1024(uint32_t (&v)[32], int lane) {
       if (stride < 32) {
 #pragma unroll
         for (int r = 0; r < 32; ++r) {
-          const uint32_t o = __shfl_xor_sync(0xffffffffu, v[r], stride);
-          const int i = r * 32 + lane;
-          const bool up = (i & size) == 0;
-          const bool lower = (lane & stride) == 0;
-          v[r] = (lower == up) ? min(v[r], o) : max(v[r], o);
+          if (r & stride) continue;
+          // element 32 l + r ascends iff bit `size` of its index is clear
+          const bool up = size < 32 ? (r & size) == 0 : ((lane << 5) & size) == 0;
+          const uint32_t a = v[r], b = v[r + stride];
+          v[r] = up ? min(a, b) : max(a, b);
+          v[r + stride] = up ? max(a, b) : min(a, b);
         }
       } else {
-        const int rs = stride >> 5;
+        const int ls = stride >> 5;
+        const bool up = ((lane << 5) & size) == 0;
+        const bool lower = (lane & ls) == 0;
 #pragma unroll
         for (int r = 0; r < 32; ++r) {
-          if (r & rs) continue;
-          const int i = r * 32 + lane;
-          const bool up = (i & size) == 0;
-          const uint32_t a = v[r], b = v[r + rs];
-          const bool sw = (a > b) == up;
-          v[r] = sw ? b : a;
-          v[r + rs] = sw ? a : b;
+          const uint32_t o = __shfl_xor_sync(0xffffffffu, v[r], ls);
+          v[r] = (lower == up) ? min(v[r], o) : max(v[r], o);
         }
       }
     }
   }
 }
 
-// Chord upper bound of 2^y for t = y + 96 with y in [-32, 32): the float
-// whose exponent is floor(y) and whose mantissa is frac(y), 2^floor(y) *
-// (1 + frac(y)) >= 2^y (2^y is convex, the chord between integers lies above
-// it, at most 6.2% above).  t in [64, 128) holds y + 32 in its mantissa with
-// 17 fractional bits, so shifting its bits left by 6 and adding a constant
-// gives the bits of the chord value.  Callers clamp t to at least 64 (y >= -32).
-__device__ __forceinline__ float chord_exp2(float t) {
-  return __uint_as_float((__float_as_uint(t) << 6) + 0x8F800000u);
+// Make room in a sub-buffer of n entries: drop the entries below the floor
+// fl (stable), or, if that is not enough, keep its own exact k best (they
+// contain its part of the top k).  Returns the new count.  Kept out of line:
+// it runs rarely and would otherwise bloat the scorers' tile loop.
+template <int NB, int BSHIFT>
+__device__ __noinline__ uint32_t make_room(uint2* buf, uint32_t n, uint32_t fl, int k, int capw,
+                                           uint32_t lo, uint32_t* dig, int lane) {
+  __syncwarp();
+  n = warp_compact(buf, n, lane, [&](uint2 v) { return v.x >= fl; });
+  if (n + 32 > uint32_t(capw) / 2 + k / 2 && n > uint32_t(k)) {
+    uint2* one[4] = {buf, buf, buf, buf};
+    const uint32_t nn[4] = {n, 0, 0, 0};
+    uint64_t pf, mk;
+    radix_select<NB, BSHIFT>(one, nn, k, lo, dig, lane, pf, mk);
+    n = warp_compact(buf, n, lane, [&](uint2 v) { return (sel_key(v) & mk) >= pf; });
+  }
+  __syncwarp();
+  return n;
 }
-
-// A candidate's chord bounds must reach at least this fraction of the floor
-// for its exact score to be computed: the bound is an upper bound up to fp32
-// rounding (relative ~1e-5), far inside this margin.
-constexpr float kChordPass = 1.0f - 1.0f / 1024.0f;
 
 template <int G>
 __global__ void __launch_bounds__(THREADS, 1)
@@ -455,9 +468,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t lane_addr = uint32_t(sub * 32) << 16;
     const uint32_t lt_mask = (1u << lane) - 1u;
     uint2* my_bufs = ws + (size_t(blockIdx.x) * 4 + sub) * QT * capw;  // [QT][capw]
-    float* stx = &ms->stg_x[sw][0][0];
-    int32_t* stp = ms->stg_pos[sw];
-    uint8_t* stq = ms->stg_q[sw];
     const uint64_t c2 = f2(scale_log2, scale_log2);
     uint32_t st = 0;
     bool ok = true;
@@ -467,175 +477,100 @@ __global__ void __launch_bounds__(THREADS, 1)
       item(it, q0, g, n_tiles, score);
       if (tid < 128) {
         const int qrow = q0 + tid / G;
-        ms->lse2[tid] = qrow < T ? lse[size_t(qrow) * Hq + g * G + tid % G] * kLog2e : INFINITY;
-        ms->nbeta[tid] = INFINITY;  // floor 0: every candidate passes the chord test
+        ms->nlse2[tid] = qrow < T ? -lse[size_t(qrow) * Hq + g * G + tid % G] * kLog2e : -INFINITY;
       }
       for (int i = tid; i < QT; i += SCORERS) {
         ms->floor_bits[i] = 0;
         ms->compacted[i] = 0;
-#pragma unroll
-        for (int v = 0; v < 4; ++v) ms->cnt[v][i] = 0;
       }
       for (int i = tid; i < QT * NB; i += SCORERS) (&ms->hist[0][0])[i] = 0;
       const int qb0 = half * QH;        // this warp's queries: qb0 .. qb0 + QH - 1
       const int qvalid = T - q0 - qb0;  // of which those below qvalid exist
+      uint2* qbuf = my_bufs + size_t(qb0) * capw;  // query qb0 + qq at qbuf + qq * capw
+      // tiles whose every key is a candidate of every query of the set need no
+      // per-key test: keys up to q0 + qb0 - w are candidates of query qb0
+      const bool all_exist = qvalid >= QH;
+      const int last_free = q0 + qb0 - w;
+      const float* nlw = &ms->nlse2[half * 32];
+      uint32_t n[QH], fl[QH];  // appended entries and floors of this warp's queries
+#pragma unroll
+      for (int qq = 0; qq < QH; ++qq) n[qq] = fl[qq] = 0;
       scorer_sync();
-
-      // ms->nbeta[c] = 96 - lse2 - log2(floor) of column c = (query, head):
-      // t = s * scale_log2 + nbeta = y + 96, y = log2(p_head / floor)
-      const float* nbw = &ms->nbeta[half * 32];
-
-      // make room in this warp's sub-buffer of query q: drop entries below
-      // the floor (stable), or, if that is not enough, keep its own exact k
-      // best (they contain its part of the top k)
-      auto make_room = [&](int q) {
-        __syncwarp();
-        uint2* buf = my_bufs + size_t(q) * capw;
-        const uint32_t fl = ms->floor_bits[q];
-        uint32_t n = warp_compact(buf, ms->cnt[sub][q], lane, [&](uint2 v) { return v.x >= fl; });
-        if (n + 32 > uint32_t(capw) / 2 + k / 2 && n > uint32_t(k)) {
-          uint2* one[4] = {buf, buf, buf, buf};
-          const uint32_t nn[4] = {n, 0, 0, 0};
-          uint64_t pf, mk;
-          radix_select<NB, BSHIFT>(one, nn, k, lo, ms->dig[sw], lane, pf, mk);
-          n = warp_compact(buf, n, lane, [&](uint2 v) { return (sel_key(v) & mk) >= pf; });
-        }
-        if (lane == 0) {
-          ms->cnt[sub][q] = n;
-          ms->compacted[q] = 1;
-        }
-        __syncwarp();
-      };
-
-      // exact scores of staged survivors base .. base + cnt - 1 (one per
-      // lane) and their appends
-      auto process = [&](int base, int cnt) {
-        const bool act = lane < cnt;
-        const int e = base + (act ? lane : 0);
-        float x[G];
-        if constexpr (G % 4 == 0) {
-#pragma unroll
-          for (int h = 0; h < G; h += 4) {
-            const float4 v = *reinterpret_cast<const float4*>(stx + e * G + h);
-            x[h] = v.x;
-            x[h + 1] = v.y;
-            x[h + 2] = v.z;
-            x[h + 3] = v.w;
-          }
-        } else {
-#pragma unroll
-          for (int h = 0; h < G; ++h) x[h] = stx[e * G + h];
-        }
-        const int ql = stq[e];
-        const int jj = stp[e];
-        const float* l2 = &ms->lse2[half * 32 + ql * G];
-        float acc = 0.f;
-#pragma unroll
-        for (int h = 0; h < G; ++h) acc += fast_exp2(fmaf(x[h], scale_log2, -l2[h]));
-        const int q = qb0 + ql;
-        const uint32_t bits = __float_as_uint(acc);
-        const bool risk = act && ms->cnt[sub][q] + 32 > uint32_t(capw);
-        uint32_t rb = __ballot_sync(0xffffffffu, risk);
-        while (rb != 0) {  // rare: a sub-buffer this batch could overflow
-          const int qr = __shfl_sync(0xffffffffu, ql, __ffs(rb) - 1);
-          make_room(qb0 + qr);
-          rb &= ~__ballot_sync(0xffffffffu, ql == qr);
-        }
-        if (act && bits >= ms->floor_bits[q]) {
-          const uint32_t pos = atomicAdd(&ms->cnt[sub][q], 1u);
-          my_bufs[size_t(q) * capw + pos] = make_uint2(bits, uint32_t(jj));
-          atomicAdd(&ms->hist[q][bin_of<NB, BSHIFT>(bits, lo)], 1u);
-        }
-        __syncwarp();
-      };
-
-      int nst = 0;  // staged survivors of this warp (the same in every lane)
       for (int t = 0; t < n_tiles; ++t, ++st) {
         const int b = st % NSB;
         ok = ok && mbar_wait(&br->s_full[b], (st / NSB) & 1);
         tc_fence_after();
         const int j = t * TILE + sub * 32 + lane;  // this thread's key
-        // candidate test for query qb0 + ql: j + w <= its position, i.e.
-        // dpos <= ql, and the query inside the sequence (ql < qvalid)
-        const int dpos = j + w - q0 - qb0;
         uint32_t r[32];
         tmem_ld32(tmem + lane_addr + b * 128 + half * 32, r);
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(&br->s_empty[b]);
-        // chord upper bound of each query's score relative to its floor
-        float qsum[QH];
+        // score of each query: sum over its G heads of exp2(s * scale_log2 - lse2)
+        float sc[QH];
 #pragma unroll
         for (int qq = 0; qq < QH; ++qq) {
           if constexpr (G == 1) {
-            qsum[qq] = chord_exp2(fmaxf(fmaf(__uint_as_float(r[qq]), scale_log2, nbw[qq]), 64.f));
+            sc[qq] = fast_exp2(fmaf(__uint_as_float(r[qq]), scale_log2, nlw[qq]));
           } else {
-            uint64_t a2 = f2(0.f, 0.f);
+            uint64_t a2 = 0;
 #pragma unroll
             for (int h = 0; h < G; h += 2) {
               const int c = qq * G + h;
-              const float2 nb2 = *reinterpret_cast<const float2*>(nbw + c);
-              float t0, t1;
+              const float2 nl = *reinterpret_cast<const float2*>(nlw + c);
+              float y0, y1;
               f2_split(f2_fma(f2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), c2,
-                              f2(nb2.x, nb2.y)),
-                       t0, t1);
-              a2 = f2_add(a2, f2(chord_exp2(fmaxf(t0, 64.f)), chord_exp2(fmaxf(t1, 64.f))));
+                              f2(nl.x, nl.y)),
+                       y0, y1);
+              const uint64_t e2 = f2(fast_exp2(y0), fast_exp2(y1));
+              a2 = h == 0 ? e2 : f2_add(a2, e2);
             }
             float s0, s1;
             f2_split(a2, s0, s1);
-            qsum[qq] = s0 + s1;
+            sc[qq] = s0 + s1;
           }
         }
-        // stage the survivors' logits; exact scores in full warps
+        // candidates at or above the floor go to this warp's sub-buffer of
+        // the query, in position order; each append is counted by score bin
+        const bool chk = !all_exist || t * TILE + TILE - 1 > last_free;
+        const int dpos = j + w - q0 - qb0;  // candidate of query qb0 + qq iff dpos <= qq
 #pragma unroll
         for (int qq = 0; qq < QH; ++qq) {
-          const bool p = dpos <= qq && qq < qvalid && qsum[qq] >= kChordPass;
+          const uint32_t bits = __float_as_uint(sc[qq]);
+          bool p = bits >= fl[qq];
+          if (chk) p = p && dpos <= qq && qq < qvalid;
           const uint32_t bal = __ballot_sync(0xffffffffu, p);
           if (bal == 0) continue;
+          if (n[qq] + 32 > uint32_t(capw)) {
+            n[qq] = make_room<NB, BSHIFT>(qbuf + size_t(qq) * capw, n[qq], ms->floor_bits[qb0 + qq],
+                                          k, capw, lo, ms->dig[sw], lane);
+            if (lane == 0) ms->compacted[qb0 + qq] = 1;
+          }
           if (p) {
-            const int slot = nst + __popc(bal & lt_mask);
-            float* dst = stx + slot * G;
-            if constexpr (G % 4 == 0) {
-#pragma unroll
-              for (int h = 0; h < G; h += 4)
-                *reinterpret_cast<float4*>(dst + h) =
-                    make_float4(__uint_as_float(r[qq * G + h]), __uint_as_float(r[qq * G + h + 1]),
-                                __uint_as_float(r[qq * G + h + 2]),
-                                __uint_as_float(r[qq * G + h + 3]));
-            } else {
-#pragma unroll
-              for (int h = 0; h < G; ++h) dst[h] = __uint_as_float(r[qq * G + h]);
-            }
-            stp[slot] = j;
-            stq[slot] = uint8_t(qq);
+            qbuf[size_t(qq) * capw + n[qq] + __popc(bal & lt_mask)] = make_uint2(bits, uint32_t(j));
+            atomicAdd(&ms->hist[qb0 + qq][bin_of<NB, BSHIFT>(bits, lo)], 1u);
           }
-          nst += __popc(bal);
-          if (nst >= 32) {
-            __syncwarp();
-            process(nst - 32, 32);
-            nst -= 32;
-          }
+          n[qq] += __popc(bal);
         }
-        // raise the floors of this warp's queries to the highest bin with at
-        // least k appended entries at or above it (any snapshot of the counts
-        // gives a valid floor), then reload the chord offsets of its columns
+        // raise the floors this warp owns to the highest bin with at least k
+        // appended entries at or above it (any snapshot of the counts gives a
+        // valid floor), then take up every floor of its queries
         if ((t & (kRefresh - 1)) == kRefresh - 1) {
           for (int q = half * QH + sub; q < (half + 1) * QH; q += 4) {
             uint32_t above, inbin;
             const int fb = hist_cross<NB>(ms->hist[q], uint32_t(k), lane, above, inbin);
             const uint32_t fbits = fb > 0 ? (uint32_t(fb) + lo) << BSHIFT : 0u;
-            if (fbits > ms->floor_bits[q]) {
-              __syncwarp();
-              if (lane == 0) ms->floor_bits[q] = fbits;
-              const float L = __log2f(__uint_as_float(fbits));
-              if (lane < G) ms->nbeta[q * G + lane] = 96.f - ms->lse2[q * G + lane] - L;
-            }
+            if (lane == 0 && fbits > ms->floor_bits[q]) ms->floor_bits[q] = fbits;
           }
           __syncwarp();
+#pragma unroll
+          for (int qq = 0; qq < QH; ++qq) fl[qq] = ms->floor_bits[qb0 + qq];
         }
       }
-      __syncwarp();
-      if (nst > 0) process(0, nst);
+      if (lane == 0) {
+#pragma unroll
+        for (int qq = 0; qq < QH; ++qq) ms->cnt[sub][qb0 + qq] = n[qq];
+      }
       scorer_sync();
       // ---- outputs of the item: one warp per query ----
       uint32_t* sp = wsort + (size_t(blockIdx.x) * SCORER_WARPS + sw) * kSortWords;  // positions
@@ -755,18 +690,28 @@ __global__ void __launch_bounds__(THREADS, 1)
           got = min(got, uint32_t(k));
           __syncwarp();
           if (k <= 1024) {
+            // lane l sorts elements 32 l .. 32 l + 31 (16-byte loads), the
+            // sorted run goes back through the scratch and out coalesced
             uint32_t v[32];
+            uint4* spv = reinterpret_cast<uint4*>(sp) + lane * 8;
 #pragma unroll
-            for (int r = 0; r < 32; ++r) {
-              const int e = r * 32 + lane;
-              v[r] = e < int(got) ? sp[e] : 0xFFFFFFFFu;
+            for (int u = 0; u < 8; ++u) {
+              const uint4 x = spv[u];
+              v[4 * u] = x.x;
+              v[4 * u + 1] = x.y;
+              v[4 * u + 2] = x.z;
+              v[4 * u + 3] = x.w;
             }
-            warp_sort1024(v, lane);
 #pragma unroll
-            for (int r = 0; r < 32; ++r) {
-              const int e = r * 32 + lane;
-              if (e < k) out[e] = e < int(got) ? int32_t(v[r]) : -1;
-            }
+            for (int r = 0; r < 32; ++r)
+              if (lane * 32 + r >= int(got)) v[r] = 0xFFFFFFFFu;
+            warp_sort1024_lm(v, lane);
+            __syncwarp();
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              spv[u] = make_uint4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+            __syncwarp();
+            for (int e = lane; e < k; e += 32) out[e] = e < int(got) ? int32_t(sp[e]) : -1;
           } else {
             // k in (1024, 2048]: bitonic sort of the staging buffer
             for (int e = got + lane; e < 2048; e += 32) sp[e] = 0xFFFFFFFFu;
