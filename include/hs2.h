@@ -250,6 +250,73 @@ hs2_status hs2_block_decode(int32_t batch, const int64_t* seq_len, const hs2_bf1
                             const hs2_shape* shape, void* workspace, size_t workspace_bytes,
                             void* stream);
 
+/*
+ * One decode step of the block with each sequence's context split over R
+ * ranks (devices), in four calls with an all-gather of small records between
+ * consecutive calls.  Not on the pages, which serve the 1M-token FP8 cache
+ * from one device (zgeo.com.cn comparison table); this is the split that
+ * lets that cache span several GPUs.  Every rank makes the same four calls;
+ * the outputs of hs2_decode_cp_select, _sparse and _finish are identical on
+ * every rank and equal to hs2_block_decode's up to fp32 rounding order (the
+ * index lists are exact).
+ *
+ * Rank r holds, for each sequence b, the slice [slice_lo[b], slice_hi[b])
+ * of its positions (HOST arrays [batch]; 0 <= lo <= hi <= seq_len[b]; the
+ * ranks' slices tile [0, seq_len[b])).  Its cache stores that slice only:
+ * position p at row p - slice_lo[b] of sequence b, Kc/Vc [batch, shape->T,
+ * n_kv_heads, 128] e4m3 and k_scale/v_scale [batch, shape->T, n_kv_heads]
+ * with shape->T >= hi - lo (the local capacity).  seq_len (HOST [batch]) is
+ * the whole sequence length; the new token is position seq_len[b] - 1.
+ * Records (all DEVICE memory, 16-byte aligned):
+ *   attention / sparse record: 130 floats per (b, query head): the softmax
+ *     state m (base-2 max logit), l (sum of 2^(x - m)), o[128] (unnormalised
+ *     sum of 2^(x - m) v) over the rank's keys;
+ *   selection record: 2 x uint32 per entry (score bits, position), k entries
+ *     per (b, KV head): the rank's own exact top k (padded with
+ *     (0, 0xFFFFFFFF) when it has fewer candidates).
+ * "Gathered" inputs are the R ranks' records concatenated in rank order
+ * (what an all-gather into one buffer writes).  n_ranks * k_global <= 8192.
+ *
+ * 1. hs2_decode_cp_attn: attention of the new token over the rank's slice ->
+ *    attn_rec [batch][n_q_heads][130].  Workspace as hs2_block_decode
+ *    (hs2_workspace_size(HS2_OP_BLOCK_DECODE, shape, batch, 0) with the
+ *    local capacity); keep it for step 2, which reads this step's logits.
+ * 2. hs2_decode_cp_select: merges the gathered attn_recs [R][batch][Hq][130]
+ *    into o_full [batch, Hq, 128] bf16 and lse [batch, Hq] (natural log),
+ *    scores the rank's candidates and writes its top k as sel_rec
+ *    [batch][n_kv_heads][k][2].
+ * 3. hs2_decode_cp_sparse: merges the gathered sel_recs [R][batch][Hkv][k][2]
+ *    into idx [batch, Hkv, k + w] (the exact top k of the whole context,
+ *    ascending, then the window) and runs the n_sparse sparse layers over the
+ *    listed positions in the rank's slice -> sparse_rec
+ *    [n_sparse][batch][Hq][130].  q_sparse: HOST array of n_sparse DEVICE
+ *    pointers [batch, Hq, 128].  No workspace.
+ * 4. hs2_decode_cp_finish: merges the gathered sparse_recs
+ *    [R][n_sparse][batch][Hq][130] into o_sparse (HOST array of n_sparse
+ *    DEVICE pointers [batch, Hq, 128] bf16).  No workspace.
+ * Errors as hs2_block_decode; HS2_ERR_UNSUPPORTED if n_ranks * k > 8192.
+ */
+hs2_status hs2_decode_cp_attn(int32_t batch, const int64_t* seq_len, const int64_t* slice_lo,
+                              const int64_t* slice_hi, const hs2_bf16* q_full,
+                              const hs2_fp8e4m3* Kc, const hs2_fp8e4m3* Vc, const float* k_scale,
+                              const float* v_scale, float* attn_rec, const hs2_shape* shape,
+                              void* workspace, size_t workspace_bytes, void* stream);
+hs2_status hs2_decode_cp_select(int32_t batch, const int64_t* seq_len, const int64_t* slice_lo,
+                                const int64_t* slice_hi, int32_t n_ranks, const float* attn_recs,
+                                hs2_bf16* o_full, float* lse, uint32_t* sel_rec,
+                                const hs2_shape* shape, void* workspace, size_t workspace_bytes,
+                                void* stream);
+hs2_status hs2_decode_cp_sparse(int32_t batch, const int64_t* seq_len, const int64_t* slice_lo,
+                                const int64_t* slice_hi, int32_t n_ranks,
+                                const uint32_t* sel_recs, int32_t* idx, const hs2_fp8e4m3* Kc,
+                                const hs2_fp8e4m3* Vc, const float* k_scale,
+                                const float* v_scale, int32_t n_sparse,
+                                const hs2_bf16* const* q_sparse, float* sparse_rec,
+                                const hs2_shape* shape, void* stream);
+hs2_status hs2_decode_cp_finish(int32_t batch, int32_t n_ranks, int32_t n_sparse,
+                                const float* sparse_recs, hs2_bf16* const* o_sparse,
+                                const hs2_shape* shape, void* stream);
+
 /* Workspace bytes needed by `op` (an HS2_OP_* code) for these sizes; 0 when
  * the op needs none.  Returns (size_t)-1 for invalid arguments. */
 size_t hs2_workspace_size(int32_t op, const hs2_shape* shape, int32_t batch, int32_t d_model);

@@ -58,6 +58,13 @@ def _load(path: str = LIB_PATH):
         "hs2_block_prefill": [P, I32, P, P, P, P, P, P, P, P, I32, PP, PP, SP, P, SZ, P],
         "hs2_block_decode": [I32, C.POINTER(C.c_int64), P, P, P, P, P, P, P, P, I32, PP, PP, SP,
                              P, SZ, P],
+        "hs2_decode_cp_attn": [I32, C.POINTER(C.c_int64), C.POINTER(C.c_int64),
+                               C.POINTER(C.c_int64), P, P, P, P, P, P, SP, P, SZ, P],
+        "hs2_decode_cp_select": [I32, C.POINTER(C.c_int64), C.POINTER(C.c_int64),
+                                 C.POINTER(C.c_int64), I32, P, P, P, P, SP, P, SZ, P],
+        "hs2_decode_cp_sparse": [I32, C.POINTER(C.c_int64), C.POINTER(C.c_int64),
+                                 C.POINTER(C.c_int64), I32, P, P, P, P, P, P, I32, PP, P, SP, P],
+        "hs2_decode_cp_finish": [I32, I32, I32, P, PP, SP, P],
     }
     for name, args in sigs.items():
         fn = getattr(L, name)
@@ -81,7 +88,8 @@ EXPORTED = ["hs2_bridge_kv", "hs2_bridge_kv_fp8", "hs2_full_attn_lse", "hs2_sele
             "hs2_sparse_attn", "hs2_sparse_attn_layers",
             "hs2_block_prefill", "hs2_block_decode", "hs2_workspace_size",
             "hs2_get_device_status", "hs2_status_string", "hs2_kernel_launches",
-            "hs2_debug_set_wait_budget"]
+            "hs2_debug_set_wait_budget", "hs2_decode_cp_attn", "hs2_decode_cp_select",
+            "hs2_decode_cp_sparse", "hs2_decode_cp_finish"]
 
 
 def _ptr(t, dtype, what, nullable=False):
@@ -208,6 +216,53 @@ def hs2_block_decode(seq_len, q_full, Kc, Vc, k_scale, v_scale, o_full, lse, idx
         _ptr(lse, F32, "lse"), _ptr(idx, I32T, "idx"), len(q_sparse), qs, os_, C.byref(shape),
         _ptr(workspace, U8, "workspace", True), nbytes, _stream(stream)), "hs2_block_decode")
 
+
+
+def _i64s(xs):
+    return (C.c_int64 * len(xs))(*[int(x) for x in xs])
+
+
+DECODE_REC_FLOATS = 130   # softmax-state record: m, l, o[128]
+
+
+def hs2_decode_cp_attn(seq_len, slice_lo, slice_hi, q_full, Kc, Vc, k_scale, v_scale, attn_rec,
+                       shape: Shape, workspace, stream=None):
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.hs2_decode_cp_attn(
+        len(seq_len), _i64s(seq_len), _i64s(slice_lo), _i64s(slice_hi),
+        _ptr(q_full, BF16, "q_full"), _ptr(Kc, U8, "Kc"), _ptr(Vc, U8, "Vc"),
+        _ptr(k_scale, F32, "k_scale"), _ptr(v_scale, F32, "v_scale"),
+        _ptr(attn_rec, F32, "attn_rec"), C.byref(shape), _ptr(workspace, U8, "workspace", True),
+        nbytes, _stream(stream)), "hs2_decode_cp_attn")
+
+
+def hs2_decode_cp_select(seq_len, slice_lo, slice_hi, n_ranks, attn_recs, o_full, lse, sel_rec,
+                         shape: Shape, workspace, stream=None):
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.hs2_decode_cp_select(
+        len(seq_len), _i64s(seq_len), _i64s(slice_lo), _i64s(slice_hi), int(n_ranks),
+        _ptr(attn_recs, F32, "attn_recs"), _ptr(o_full, BF16, "o_full"), _ptr(lse, F32, "lse"),
+        _ptr(sel_rec, I32T, "sel_rec"), C.byref(shape), _ptr(workspace, U8, "workspace", True),
+        nbytes, _stream(stream)), "hs2_decode_cp_select")
+
+
+def hs2_decode_cp_sparse(seq_len, slice_lo, slice_hi, n_ranks, sel_recs, idx, Kc, Vc, k_scale,
+                         v_scale, q_sparse, sparse_rec, shape: Shape, stream=None):
+    qs, _keep_q = _ptr_array(q_sparse, BF16, "q_sparse")
+    _check(_lib.hs2_decode_cp_sparse(
+        len(seq_len), _i64s(seq_len), _i64s(slice_lo), _i64s(slice_hi), int(n_ranks),
+        _ptr(sel_recs, I32T, "sel_recs"), _ptr(idx, I32T, "idx"), _ptr(Kc, U8, "Kc"),
+        _ptr(Vc, U8, "Vc"), _ptr(k_scale, F32, "k_scale"), _ptr(v_scale, F32, "v_scale"),
+        len(q_sparse), qs, _ptr(sparse_rec, F32, "sparse_rec", True), C.byref(shape),
+        _stream(stream)), "hs2_decode_cp_sparse")
+
+
+def hs2_decode_cp_finish(n_ranks, sparse_recs, o_sparse, shape: Shape, stream=None):
+    os_, _keep_o = _ptr_array(o_sparse, BF16, "o_sparse")
+    batch = o_sparse[0].shape[0]
+    _check(_lib.hs2_decode_cp_finish(batch, int(n_ranks), len(o_sparse),
+                                     _ptr(sparse_recs, F32, "sparse_recs"), os_, C.byref(shape),
+                                     _stream(stream)), "hs2_decode_cp_finish")
 
 
 def hs2_get_device_status(stream=None) -> int:

@@ -49,7 +49,7 @@ namespace {
 constexpr int CH = 8192;            // keys per decode_partial CTA
 constexpr int DP_WARPS = 4;         // each warp: CH / 4 keys, 16 per step
 constexpr int NBUCKET = 2048;       // score buckets (bits >> 20 of fp32 < 2^8)
-constexpr int CAPC = 8192;          // candidate list capacity per (b, g)
+constexpr int CAPC = kDecodeMergeCap;  // candidate list capacity per (b, g)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -60,8 +60,10 @@ struct Partial {  // per (b, h, chunk)
   float m, l;
 };
 
-struct SeqLens {  // sequence lengths, passed by value
-  int n[MAX_B];
+struct SeqLens {  // per sequence, passed by value: its length n (the new token
+  int n[MAX_B];     // is n - 1) and the slice [lo, hi) of its cache this call
+  int lo[MAX_B];    // covers (the whole cache, [0, n), unless the context is
+  int hi[MAX_B];    // split over ranks)
 };
 
 // both e4m3 pairs of a 32-bit word -> two f16x2 (low pair, high pair)
@@ -130,12 +132,15 @@ __global__ void __launch_bounds__((DP_WARPS + 1) * 32, 3)
   const int g = blockIdx.x, c = blockIdx.y, b = blockIdx.z;
   const int warp = warp_id(), lane = lane_id();
   const int gid = lane >> 2, t = lane & 3;
-  const int N = seq_len.n[b];
   const int Hq = Hkv * G;
-  const int64_t c_lo = int64_t(c) * CH;
-  const int64_t c_hi = min(c_lo + CH, int64_t(N));
+  // chunk c covers positions lo + c * CH .. (local rows c * CH ..) of the slice
+  const int64_t c_lo = int64_t(seq_len.lo[b]) + int64_t(c) * CH;
+  const int64_t c_hi = min(c_lo + CH, int64_t(seq_len.hi[b]));
   const int n_st = c_hi > c_lo ? int((c_hi - c_lo + DSTAGE_KEYS - 1) / DSTAGE_KEYS) : 0;
-  const size_t rowbase = size_t(b) * cap;  // first cache row of sequence b
+  // cache row of position p of sequence b: the cache holds its slice
+  // [lo, hi), position lo at row b * cap
+  const int64_t lo = seq_len.lo[b];
+  const int64_t rowpos = int64_t(b) * cap - lo;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < DSTAGES; ++i) {
@@ -165,14 +170,14 @@ __global__ void __launch_bounds__((DP_WARPS + 1) * 32, 3)
       for (int u = 0; u < DSTAGE_KEYS / 32; ++u) {
         const int64_t key = kbase + lane + 32 * u;
         const bool in = key < c_hi;
-        const size_t off = (rowbase + size_t(in ? key : c_lo)) * Hkv + g;
+        const size_t off = size_t(rowpos + (in ? key : c_lo)) * Hkv + g;
         cp_async4(&sScale[slot][0][lane + 32 * u], ks + off, in ? 4 : 0);
         cp_async4(&sScale[slot][1][lane + 32 * u], vs + off, in ? 4 : 0);
       }
       cp_async_arrive(&full[slot]);
       if (lane == 0) {
         uint8_t* st = ring + slot * DSTAGE_BYTES;
-        const int z = int(rowbase + c_lo) + si * DSTAGE_KEYS;
+        const int z = int(rowpos + c_lo) + si * DSTAGE_KEYS;
         mbar_arrive_expect_tx(&full[slot], DSTAGE_BYTES);
         tma_load_3d(st, &tmK, &full[slot], 0, g, z);
         tma_load_3d(st + DSTAGE_KEYS * 128, &tmV, &full[slot], 0, g, z);
@@ -273,11 +278,11 @@ __global__ void __launch_bounds__((DP_WARPS + 1) * 32, 3)
         if (h0 >= GH + nt * 8) sv[q2][0][0] = sv[q2][1][0] = -INFINITY;  // padded heads
         if (h0 + 1 >= GH + nt * 8) sv[q2][0][1] = sv[q2][1][1] = -INFINITY;
         if (h0 + 1 < G) {
-          if (v0) *reinterpret_cast<float2*>(lg + r0 * G + h0) = make_float2(sv[q2][0][0], sv[q2][0][1]);
-          if (v1) *reinterpret_cast<float2*>(lg + r1 * G + h0) = make_float2(sv[q2][1][0], sv[q2][1][1]);
+          if (v0) *reinterpret_cast<float2*>(lg + (r0 - lo) * G + h0) = make_float2(sv[q2][0][0], sv[q2][0][1]);
+          if (v1) *reinterpret_cast<float2*>(lg + (r1 - lo) * G + h0) = make_float2(sv[q2][1][0], sv[q2][1][1]);
         } else if (h0 < G) {
-          if (v0) lg[r0 * G + h0] = sv[q2][0][0];
-          if (v1) lg[r1 * G + h0] = sv[q2][1][0];
+          if (v0) lg[(r0 - lo) * G + h0] = sv[q2][0][0];
+          if (v1) lg[(r1 - lo) * G + h0] = sv[q2][1][0];
         }
       }
       // online softmax over the warp's 32 keys of the stage for heads h0, h0+1
@@ -420,16 +425,21 @@ __global__ void __launch_bounds__((DP_WARPS + 1) * 32, 3)
 // decode_merge: grid (Hq, B), 128 threads
 // ---------------------------------------------------------------------------
 constexpr int MERGE_GROUPS = 4;  // groups of 128 threads, each over every 4th chunk
+constexpr int REC = kDecodeRecFloats;  // a softmax-state record: m, l, o[128] (floats)
 
+// Merges the chunk partials of each (b, h) over the chunks covering its
+// slice.  rec == nullptr: the result o (bf16), lse (natural log) and lse2;
+// otherwise the merged state itself as one record (m, l, o unnormalised),
+// [B][Hq][REC], for a merge across ranks.
 __global__ void __launch_bounds__(128 * MERGE_GROUPS)
     decode_merge(const Partial* __restrict__ part, const float* __restrict__ part_o,
                  SeqLens seq_len, int Hq, int nch, __nv_bfloat16* __restrict__ o,
-                 float* __restrict__ lse, float* __restrict__ lse2_out) {
+                 float* __restrict__ lse, float* __restrict__ lse2_out, float* __restrict__ rec) {
   __shared__ float s_red[MERGE_GROUPS][129];
   __shared__ float s_max[128 * MERGE_GROUPS / 32];
   const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int d = tid & 127, grp = tid >> 7;
-  const int nc = (seq_len.n[b] + CH - 1) / CH;
+  const int nc = (seq_len.hi[b] - seq_len.lo[b] + CH - 1) / CH;  // chunks of the slice
   const size_t base = (size_t(b) * Hq + h) * nch;
   // the largest chunk maximum
   float M = -INFINITY;
@@ -456,12 +466,47 @@ __global__ void __launch_bounds__(128 * MERGE_GROUPS)
     for (int q = 1; q < MERGE_GROUPS; ++q) acc += s_red[q][d];
     L = 0.f;
     for (int q = 0; q < MERGE_GROUPS; ++q) L += s_red[q][128];
+    if (rec != nullptr) {
+      float* r = rec + (size_t(b) * Hq + h) * REC;
+      r[2 + d] = acc;
+      if (d == 0) {
+        r[0] = M;
+        r[1] = L;
+      }
+      return;
+    }
     o[(size_t(b) * Hq + h) * 128 + d] = __float2bfloat16_rn(acc / L);
     if (d == 0) {
       const float l2 = M + __log2f(L);
       lse[size_t(b) * Hq + h] = l2 * kLn2;
       lse2_out[size_t(b) * Hq + h] = l2;
     }
+  }
+}
+
+// Merges the records of R ranks for (b, h): record r at
+// recs + r * rank_stride + (b * Hq + h) * REC.  Writes o (bf16), and lse /
+// lse2 where those pointers are not null.
+__global__ void __launch_bounds__(128)
+    decode_merge_ranks(const float* __restrict__ recs, int R, int64_t rank_stride, int Hq,
+                       __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
+                       float* __restrict__ lse2_out) {
+  const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
+  const size_t off = (size_t(b) * Hq + h) * REC;
+  float M = -INFINITY;
+  for (int r = 0; r < R; ++r) M = fmaxf(M, recs[r * rank_stride + off]);
+  float L = 0.f, acc = 0.f;
+  for (int r = 0; r < R; ++r) {
+    const float* rr = recs + r * rank_stride + off;
+    const float f = rr[0] == -INFINITY ? 0.f : fast_exp2(rr[0] - M);
+    L += rr[1] * f;
+    acc += rr[2 + d] * f;
+  }
+  o[(size_t(b) * Hq + h) * 128 + d] = __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
+  if (d == 0) {
+    const float l2 = L > 0.f ? M + __log2f(L) : -INFINITY;
+    if (lse != nullptr) lse[size_t(b) * Hq + h] = l2 * kLn2;
+    if (lse2_out != nullptr) lse2_out[size_t(b) * Hq + h] = l2;
   }
 }
 
@@ -480,20 +525,22 @@ __global__ void __launch_bounds__(256)
   __shared__ float sl[G];
   const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int N = seq_len.n[b];
-  const int64_t ncand = int64_t(N) - w;  // candidates j < ncand (j <= i - w)
+  // candidates j <= i - w, i.e. j < N - w, inside the slice [lo, hi)
+  const int64_t j_end = min(int64_t(N) - w, int64_t(seq_len.hi[b]));
   for (int i = threadIdx.x; i < NBUCKET; i += 256) sh[i] = 0;
   if (threadIdx.x < G) sl[threadIdx.x] = lse2[size_t(b) * Hkv * G + g * G + threadIdx.x];
   __syncthreads();
+  const int64_t lo = seq_len.lo[b];  // logits and scores are indexed by j - lo
   const float* lg = logits + (size_t(b) * Hkv + g) * cap * G;
   float* sc = score + (size_t(b) * Hkv + g) * cap;
-  const int64_t j_hi = min(int64_t(c + 1) * CH, ncand);
-  for (int64_t j = int64_t(c) * CH + threadIdx.x; j < j_hi; j += 256) {
+  const int64_t j_hi = min(lo + int64_t(c + 1) * CH, j_end);
+  for (int64_t j = lo + int64_t(c) * CH + threadIdx.x; j < j_hi; j += 256) {
     // the G logits of key j: 16-byte loads where G allows
     float x[G];
     if constexpr (G % 4 == 0) {
 #pragma unroll
       for (int h = 0; h < G; h += 4) {
-        const float4 v = *reinterpret_cast<const float4*>(lg + j * G + h);
+        const float4 v = *reinterpret_cast<const float4*>(lg + (j - lo) * G + h);
         x[h] = v.x;
         x[h + 1] = v.y;
         x[h + 2] = v.z;
@@ -501,12 +548,12 @@ __global__ void __launch_bounds__(256)
       }
     } else {
 #pragma unroll
-      for (int h = 0; h < G; ++h) x[h] = lg[j * G + h];
+      for (int h = 0; h < G; ++h) x[h] = lg[(j - lo) * G + h];
     }
     float acc = 0.f;
 #pragma unroll
     for (int h = 0; h < G; ++h) acc += fast_exp2(x[h] - sl[h]);
-    sc[j] = acc;
+    sc[j - lo] = acc;
     atomicAdd(&sh[__float_as_uint(acc) >> 20], 1u);
   }
   __syncthreads();
@@ -575,39 +622,44 @@ __global__ void __launch_bounds__(256)
                    uint2* __restrict__ cand, uint32_t* __restrict__ ccount) {
   const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int N = seq_len.n[b];
-  const int64_t ncand = int64_t(N) - w;
-  if (ncand <= k) return;  // everything is selected; decode_final writes it
-  const int64_t j_lo = int64_t(c) * CH;
-  if (j_lo >= ncand) return;
+  const int64_t s_lo = seq_len.lo[b];
+  const int64_t s_hi = min(int64_t(N) - w, int64_t(seq_len.hi[b]));  // slice candidates [s_lo, s_hi)
+  if (s_hi - s_lo <= k) return;  // every candidate is selected; decode_final writes them
+  const int64_t j_lo = s_lo + int64_t(c) * CH;
+  const int64_t j_hi = min(j_lo + CH, s_hi);
+  if (j_lo >= j_hi) return;
   const size_t bg = size_t(b) * Hkv + g;
   const int kb = kth_bucket[bg];
   const uint32_t thr = kb < 0 ? 0u : uint32_t(kb);
-  const float* sc = score + bg * cap;
-  const int64_t j_hi = min(j_lo + CH, ncand);
+  const float* sc = score + bg * cap;  // score of key j at sc[j - s_lo]
   const int lane = lane_id();
   const bool vec = (cap & 3) == 0;  // rows of scores start 16-byte aligned
-  // rounds of 2048 keys: thread owns keys j0 .. j0+3 and j0+1024 .. j0+1027;
-  // all eight loads are issued before any is used
-  for (int64_t base = j_lo; base < j_hi; base += 2048) {
+  // in local indices x = j - s_lo: rounds of 2048 keys from a multiple of 4
+  // at or below x_lo; thread owns keys x0 .. x0+3 and x0+1024 .. x0+1027
+  // (16-byte aligned when cap is a multiple of 4); all eight loads are
+  // issued before any is used
+  const int64_t x_lo = j_lo - s_lo, x_hi = j_hi - s_lo;
+  for (int64_t base = x_lo & ~int64_t(3); base < x_hi; base += 2048) {
     float v[8];
 #pragma unroll
     for (int hlf = 0; hlf < 2; ++hlf) {
-      const int64_t j0 = base + 1024 * hlf + 4 * threadIdx.x;
-      if (vec && j0 + 3 < j_hi) {
-        const float4 x = __ldcs(reinterpret_cast<const float4*>(sc + j0));
+      const int64_t x0 = base + 1024 * hlf + 4 * threadIdx.x;
+      if (vec && x0 + 3 < x_hi) {
+        const float4 x = __ldcs(reinterpret_cast<const float4*>(sc + x0));
         v[4 * hlf] = x.x;
         v[4 * hlf + 1] = x.y;
         v[4 * hlf + 2] = x.z;
         v[4 * hlf + 3] = x.w;
       } else {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) v[4 * hlf + u] = j0 + u < j_hi ? sc[j0 + u] : 0.f;
+        for (int u = 0; u < 4; ++u) v[4 * hlf + u] = x0 + u < x_hi ? sc[x0 + u] : 0.f;
       }
     }
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      const int64_t j = base + 1024 * (e >> 2) + 4 * threadIdx.x + (e & 3);
-      const bool take = j < j_hi && (__float_as_uint(v[e]) >> 20) >= thr;
+      const int64_t xl = base + 1024 * (e >> 2) + 4 * threadIdx.x + (e & 3);
+      const int64_t j = xl + s_lo;
+      const bool take = xl >= x_lo && xl < x_hi && (__float_as_uint(v[e]) >> 20) >= thr;
       const uint32_t bal = __ballot_sync(0xffffffffu, take);
       if (bal) {
         uint32_t pos = 0;
@@ -640,10 +692,33 @@ __device__ void block_bitonic_u64(uint64_t* s, int np, bool descending) {
     }
 }
 
+// What decode_final reads and writes.
+//   FINAL_FULL   the whole block on one device: the top k of the candidate
+//                list (or, when it overflowed, of every candidate's score),
+//                positions ascending, then the window, into idx.
+//   FINAL_LOCAL  one rank of a context split over ranks: the top k of the
+//                candidates in its slice as records (score bits, position),
+//                [B][Hkv][k], padded with (0, 0xFFFFFFFF) (below every real
+//                candidate) when the slice has fewer.
+//   FINAL_MERGE  the top k of the ranks' gathered records, positions
+//                ascending, then the window, into idx.  Record e of (b, g)
+//                is recs[(e / k) * rank_stride + (b * Hkv + g) * k + e % k].
+enum { FINAL_FULL = 0, FINAL_LOCAL = 1, FINAL_MERGE = 2 };
+
+struct FinalIO {
+  const uint2* cand;        // decode_collect's lists [B][Hkv][CAPC]
+  const uint32_t* ccount;   // and their lengths
+  const uint2* recs;        // FINAL_MERGE: gathered records
+  int n_ranks;
+  int64_t rank_stride;      // in records
+  uint2* rec_out;           // FINAL_LOCAL: this rank's records
+  int32_t* idx;             // FINAL_FULL / FINAL_MERGE: [B][Hkv][k + w]
+};
+
+template <int MODE>
 __global__ void __launch_bounds__(512)
-    decode_final(const uint2* __restrict__ cand, const uint32_t* __restrict__ ccount,
-                 const float* __restrict__ score, SeqLens seq_len, int64_t cap,
-                 int Hkv, int k, int w, int32_t* __restrict__ idx) {
+    decode_final(FinalIO io, const float* __restrict__ score, SeqLens seq_len, int64_t cap,
+                 int Hkv, int k, int w) {
   extern __shared__ uint64_t sk[];  // CAPC keys
   __shared__ uint32_t s_hist[256];
   __shared__ uint32_t s_misc[4];
@@ -652,22 +727,40 @@ __global__ void __launch_bounds__(512)
   const int64_t i = N - 1;
   const int64_t ncand = max(int64_t(0), i - w + 1);
   const size_t bg = size_t(b) * Hkv + g;
-  int32_t* out = idx + bg * (k + w);
-  for (int t2 = tid; t2 < w; t2 += blockDim.x) {
-    const int64_t p = i - w + 1 + t2;
-    out[k + t2] = p >= 0 ? int32_t(p) : -1;
+  int32_t* out = MODE == FINAL_LOCAL ? nullptr : io.idx + bg * (k + w);
+  uint2* rec = MODE == FINAL_LOCAL ? io.rec_out + bg * k : nullptr;
+  // candidates of this call: all of [0, ncand), or those of the slice
+  const int64_t c_lo = MODE == FINAL_LOCAL ? min(int64_t(seq_len.lo[b]), ncand) : 0;
+  const int64_t c_hi = MODE == FINAL_LOCAL ? min(int64_t(seq_len.hi[b]), ncand) : ncand;
+  const int64_t nc = max(int64_t(0), c_hi - c_lo);
+  // score of candidate j at sc[j - lo] (the cache holds the slice from lo)
+  const int64_t lo = seq_len.lo[b];
+  const float* sc = score + bg * cap;
+  if (MODE != FINAL_LOCAL) {
+    for (int t2 = tid; t2 < w; t2 += blockDim.x) {
+      const int64_t p = i - w + 1 + t2;
+      out[k + t2] = p >= 0 ? int32_t(p) : -1;
+    }
   }
-  if (ncand <= k) {
-    for (int e = tid; e < k; e += blockDim.x) out[e] = e < ncand ? e : -1;
+  if (nc <= k) {
+    if (MODE == FINAL_LOCAL) {
+      for (int e = tid; e < k; e += blockDim.x)
+        rec[e] = e < nc ? make_uint2(__float_as_uint(sc[c_lo + e - lo]), uint32_t(c_lo + e))
+                        : make_uint2(0u, 0xFFFFFFFFu);
+    } else {
+      for (int e = tid; e < k; e += blockDim.x) out[e] = e < nc ? e : -1;
+    }
     return;
   }
-  const uint32_t n = ccount[bg];
+  const uint32_t n = MODE == FINAL_MERGE ? uint32_t(io.n_ranks) * uint32_t(k) : io.ccount[bg];
   if (n <= uint32_t(CAPC)) {
     int np = 1;
     while (np < int(n)) np <<= 1;
     for (int e = tid; e < np; e += blockDim.x) {
       if (e < int(n)) {
-        const uint2 v = cand[bg * CAPC + e];
+        const uint2 v = MODE == FINAL_MERGE
+                            ? io.recs[(e / k) * io.rank_stride + int64_t(bg) * k + e % k]
+                            : io.cand[bg * CAPC + e];
         sk[e] = (uint64_t(v.x) << 32) | uint64_t(~v.y);
       } else {
         sk[e] = 0;  // below every real key
@@ -675,6 +768,11 @@ __global__ void __launch_bounds__(512)
     }
     __syncthreads();
     block_bitonic_u64(sk, np, true);  // best first
+    if (MODE == FINAL_LOCAL) {
+      for (int e = tid; e < k; e += blockDim.x)
+        rec[e] = make_uint2(uint32_t(sk[e] >> 32), ~uint32_t(sk[e]));
+      return;
+    }
     // the k best positions, ascending
     int kp = 1;
     while (kp < k) kp <<= 1;
@@ -686,16 +784,15 @@ __global__ void __launch_bounds__(512)
     for (int e = tid; e < k; e += blockDim.x) out[e] = int32_t(sk[e]);
     return;
   }
-  // overflow: exact radix select over every candidate's score, then the
-  // selected positions in ascending order by a block-wide ordered scan
-  const float* sc = score + bg * cap;
+  // overflow (FULL / LOCAL): exact radix select over every candidate's score,
+  // then the selected positions in ascending order by a block-wide ordered scan
   uint64_t prefix = 0, mask = 0;
   uint32_t remaining = k;
   for (int shift = 56; shift >= 0; shift -= 8) {
     for (int e = tid; e < 256; e += blockDim.x) s_hist[e] = 0;
     __syncthreads();
-    for (int64_t j = tid; j < ncand; j += blockDim.x) {
-      const uint64_t key = (uint64_t(__float_as_uint(sc[j])) << 32) | uint64_t(~uint32_t(j));
+    for (int64_t j = c_lo + tid; j < c_hi; j += blockDim.x) {
+      const uint64_t key = (uint64_t(__float_as_uint(sc[j - lo])) << 32) | uint64_t(~uint32_t(j));
       if ((key & mask) == prefix) atomicAdd(&s_hist[(key >> shift) & 255], 1u);
     }
     __syncthreads();
@@ -720,11 +817,13 @@ __global__ void __launch_bounds__(512)
   }
   __shared__ uint32_t s_warp[16];
   uint32_t written = 0;
-  for (int64_t base = 0; base < ncand; base += blockDim.x) {
+  for (int64_t base = c_lo; base < c_hi; base += blockDim.x) {
     const int64_t j = base + tid;
     bool sel = false;
-    if (j < ncand) {
-      const uint64_t key = (uint64_t(__float_as_uint(sc[j])) << 32) | uint64_t(~uint32_t(j));
+    float v = 0.f;
+    if (j < c_hi) {
+      v = sc[j - lo];
+      const uint64_t key = (uint64_t(__float_as_uint(v)) << 32) | uint64_t(~uint32_t(j));
       sel = (key & mask) >= prefix;
     }
     const uint32_t bal = __ballot_sync(0xffffffffu, sel);
@@ -736,7 +835,12 @@ __global__ void __launch_bounds__(512)
     for (int w2 = 0; w2 < int(blockDim.x / 32); ++w2) tot += s_warp[w2];
     if (sel) {
       const uint32_t p = before + __popc(bal & ((1u << lane_id()) - 1u));
-      if (p < uint32_t(k)) out[p] = int32_t(j);
+      if (p < uint32_t(k)) {
+        if (MODE == FINAL_LOCAL)
+          rec[p] = make_uint2(__float_as_uint(v), uint32_t(j));
+        else
+          out[p] = int32_t(j);
+      }
     }
     written += tot;
     __syncthreads();
@@ -748,8 +852,10 @@ cudaError_t launch_dec_g(const DecodeArgs& a, const SeqLens& d_seq, int max_len,
                          uint8_t* w8) {
   const int Hq = a.Hq, Hkv = a.Hkv, B = a.B;
   const int nch = int((a.cap + CH - 1) / CH);
-  const int nch_used = (max_len + CH - 1) / CH;
-  // workspace layout (see decode_workspace_bytes)
+  const int nch_used = (max_len + CH - 1) / CH;  // chunks of the longest slice (<= nch)
+  const bool full = a.step == DEC_FULL;
+  // workspace layout (see decode_workspace_bytes); DEC_CP_ATTN leaves the
+  // logits there for DEC_CP_SELECT
   size_t off = 0;
   auto take = [&](size_t bytes) {
     uint8_t* p = w8 + off;
@@ -767,56 +873,126 @@ cudaError_t launch_dec_g(const DecodeArgs& a, const SeqLens& d_seq, int max_len,
   uint32_t* done = ccount + size_t(B) * Hkv;
   int* kth_bucket = reinterpret_cast<int*>(done + size_t(B) * Hkv);
   uint2* cand = reinterpret_cast<uint2*>(take(size_t(B) * Hkv * CAPC * 8));
-
-  cudaError_t e = cudaMemsetAsync(hist, 0, size_t(B) * Hkv * NBUCKET * 4, st);
-  if (e != cudaSuccess) return e;
-  e = cudaMemsetAsync(ccount, 0, size_t(B) * Hkv * 8, st);  // counts and tickets
-  if (e != cudaSuccess) return e;
   const float sl2 = a.scale * kLog2e;
-  // K, V codes viewed as [B*cap tokens][Hkv][64 two-byte units]: 64-row boxes
-  CUtensorMap tmK, tmV;
-  const uint64_t rows = uint64_t(B) * a.cap;
-  if (!make_tmap_3d(&tmK, a.Kc, 64, Hkv, rows, 128, uint64_t(Hkv) * 128, 64, 1, DSTAGE_KEYS) ||
-      !make_tmap_3d(&tmV, a.Vc, 64, Hkv, rows, 128, uint64_t(Hkv) * 128, 64, 1, DSTAGE_KEYS))
-    return cudaErrorInvalidValue;
-  const int psmem = DSTAGES * DSTAGE_BYTES + 1024;
-  e = ensure_smem_attr(reinterpret_cast<const void*>(decode_partial<G>), psmem);
-  if (e != cudaSuccess) return e;
-  decode_partial<G><<<dim3(Hkv, nch_used, B), (DP_WARPS + 1) * 32, psmem, st>>>(
-      tmK, tmV, reinterpret_cast<const __nv_bfloat16*>(a.q), a.ks, a.vs, d_seq, a.cap, Hkv, nch,
-      sl2, logits, part, part_o);
-  decode_merge<<<dim3(Hq, B), 128 * MERGE_GROUPS, 0, st>>>(part, part_o, d_seq, Hq, nch,
-                                            reinterpret_cast<__nv_bfloat16*>(a.o), a.lse, lse2);
-  decode_score<G><<<dim3(nch_used, Hkv, B), 256, 0, st>>>(logits, lse2, d_seq, a.cap, Hkv, a.k,
-                                                          a.w, score, hist, done, kth_bucket);
-  decode_collect<<<dim3(nch_used, Hkv, B), 256, 0, st>>>(score, kth_bucket, d_seq, a.cap, Hkv,
-                                                         a.k, a.w, cand, ccount);
-  const int fsmem = CAPC * 8;
-  e = ensure_smem_attr(reinterpret_cast<const void*>(decode_final), fsmem);
-  if (e != cudaSuccess) return e;
-  decode_final<<<dim3(Hkv, B), 512, fsmem, st>>>(cand, ccount, score, d_seq, a.cap, Hkv, a.k, a.w,
-                                                 a.idx);
-  count_launch(5);
+  cudaError_t e = cudaSuccess;
+  unsigned launches = 0;
+
+  if (full || a.step == DEC_CP_ATTN) {
+    // K, V codes viewed as [B*cap tokens][Hkv][64 two-byte units]: 64-row boxes
+    CUtensorMap tmK, tmV;
+    const uint64_t rows = uint64_t(B) * a.cap;
+    if (!make_tmap_3d(&tmK, a.Kc, 64, Hkv, rows, 128, uint64_t(Hkv) * 128, 64, 1, DSTAGE_KEYS) ||
+        !make_tmap_3d(&tmV, a.Vc, 64, Hkv, rows, 128, uint64_t(Hkv) * 128, 64, 1, DSTAGE_KEYS))
+      return cudaErrorInvalidValue;
+    const int psmem = DSTAGES * DSTAGE_BYTES + 1024;
+    e = ensure_smem_attr(reinterpret_cast<const void*>(decode_partial<G>), psmem);
+    if (e != cudaSuccess) return e;
+    if (nch_used > 0)
+      decode_partial<G><<<dim3(Hkv, nch_used, B), (DP_WARPS + 1) * 32, psmem, st>>>(
+          tmK, tmV, reinterpret_cast<const __nv_bfloat16*>(a.q), a.ks, a.vs, d_seq, a.cap, Hkv,
+          nch, sl2, logits, part, part_o);
+    decode_merge<<<dim3(Hq, B), 128 * MERGE_GROUPS, 0, st>>>(
+        part, part_o, d_seq, Hq, nch, reinterpret_cast<__nv_bfloat16*>(a.o), a.lse, lse2,
+        full ? nullptr : a.attn_rec);
+    launches += 2;
+    if (!full) {
+      count_launch(launches);
+      return cudaGetLastError();
+    }
+  }
+  if (a.step == DEC_CP_SELECT) {
+    decode_merge_ranks<<<dim3(Hq, B), 128, 0, st>>>(
+        a.attn_recs, a.n_ranks, int64_t(B) * Hq * REC, Hq, reinterpret_cast<__nv_bfloat16*>(a.o),
+        a.lse, lse2);
+    ++launches;
+  }
+  if (full || a.step == DEC_CP_SELECT) {
+    e = cudaMemsetAsync(hist, 0, size_t(B) * Hkv * NBUCKET * 4, st);
+    if (e != cudaSuccess) return e;
+    e = cudaMemsetAsync(ccount, 0, size_t(B) * Hkv * 8, st);  // counts and tickets
+    if (e != cudaSuccess) return e;
+    if (nch_used > 0) {
+      decode_score<G><<<dim3(nch_used, Hkv, B), 256, 0, st>>>(logits, lse2, d_seq, a.cap, Hkv,
+                                                              a.k, a.w, score, hist, done,
+                                                              kth_bucket);
+      decode_collect<<<dim3(nch_used, Hkv, B), 256, 0, st>>>(score, kth_bucket, d_seq, a.cap,
+                                                             Hkv, a.k, a.w, cand, ccount);
+      launches += 2;
+    }
+    const int fsmem = CAPC * 8;
+    FinalIO io{};
+    io.cand = cand;
+    io.ccount = ccount;
+    if (full) {
+      io.idx = a.idx;
+      e = ensure_smem_attr(reinterpret_cast<const void*>(decode_final<FINAL_FULL>), fsmem);
+      if (e != cudaSuccess) return e;
+      decode_final<FINAL_FULL><<<dim3(Hkv, B), 512, fsmem, st>>>(io, score, d_seq, a.cap, Hkv,
+                                                                 a.k, a.w);
+    } else {
+      io.rec_out = a.sel_rec;
+      e = ensure_smem_attr(reinterpret_cast<const void*>(decode_final<FINAL_LOCAL>), fsmem);
+      if (e != cudaSuccess) return e;
+      decode_final<FINAL_LOCAL><<<dim3(Hkv, B), 512, fsmem, st>>>(io, score, d_seq, a.cap, Hkv,
+                                                                  a.k, a.w);
+    }
+    ++launches;
+    if (!full) {
+      count_launch(launches);
+      return cudaGetLastError();
+    }
+  }
+  if (a.step == DEC_CP_SPARSE) {
+    const int fsmem = CAPC * 8;
+    FinalIO io{};
+    io.recs = a.sel_recs;
+    io.n_ranks = a.n_ranks;
+    io.rank_stride = int64_t(B) * Hkv * a.k;
+    io.idx = a.idx;
+    e = ensure_smem_attr(reinterpret_cast<const void*>(decode_final<FINAL_MERGE>), fsmem);
+    if (e != cudaSuccess) return e;
+    decode_final<FINAL_MERGE><<<dim3(Hkv, B), 512, fsmem, st>>>(io, score, d_seq, a.cap, Hkv,
+                                                                a.k, a.w);
+    ++launches;
+  }
+  count_launch(launches);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  for (int l = 0; l < a.n_sparse; ++l) {
-    SparseArgs s{};
-    s.Q = a.qs[l];
-    s.idx = a.idx;
-    s.O = a.os[l];
-    s.lse = nullptr;
-    s.T = B;
-    s.Hq = Hq;
-    s.Hkv = Hkv;
-    s.scale = a.scale;
-    s.kw = a.k + a.w;
-    s.Kc = a.Kc;
-    s.Vc = a.Vc;
-    s.ks = a.ks;
-    s.vs = a.vs;
-    s.cache_T = a.cap;
-    e = launch_sparse(s, st);
-    if (e != cudaSuccess) return e;
+  if (full || a.step == DEC_CP_SPARSE) {
+    for (int l = 0; l < a.n_sparse; ++l) {
+      SparseArgs s{};
+      s.Q = a.qs[l];
+      s.idx = a.idx;
+      s.O = full ? a.os[l] : nullptr;
+      s.lse = nullptr;
+      s.T = B;
+      s.Hq = Hq;
+      s.Hkv = Hkv;
+      s.scale = a.scale;
+      s.kw = a.k + a.w;
+      s.Kc = a.Kc;
+      s.Vc = a.Vc;
+      s.ks = a.ks;
+      s.vs = a.vs;
+      s.cache_T = a.cap;
+      for (int b = 0; b < B; ++b) {
+        s.spans.lo[b] = d_seq.lo[b];
+        s.spans.hi[b] = full ? int(a.cap) : d_seq.hi[b];
+      }
+      s.rec = full ? nullptr : a.sparse_rec + size_t(l) * B * Hq * REC;
+      e = launch_sparse(s, st);
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+  }
+  if (a.step == DEC_CP_FINISH) {
+    for (int l = 0; l < a.n_sparse; ++l) {
+      decode_merge_ranks<<<dim3(Hq, B), 128, 0, st>>>(
+          a.sparse_recs + size_t(l) * B * Hq * REC, a.n_ranks, int64_t(a.n_sparse) * B * Hq * REC,
+          Hq, reinterpret_cast<__nv_bfloat16*>(a.os[l]), nullptr, nullptr);
+    }
+    count_launch(a.n_sparse);
+    return cudaGetLastError();
   }
   return cudaSuccess;
 }
@@ -841,11 +1017,14 @@ size_t decode_workspace_bytes(int B, int64_t cap, int Hq, int Hkv, int k, int w)
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
   if (a.B > MAX_B || a.k > CAPC / 2 || int64_t(a.B) * a.cap > INT32_MAX) return cudaErrorNotSupported;
+  if (a.step != DEC_FULL && int64_t(a.n_ranks) * a.k > CAPC) return cudaErrorNotSupported;
   SeqLens d_seq{};
-  int max_len = 0;
+  int max_len = 0;  // the longest slice
   for (int b = 0; b < a.B; ++b) {
     d_seq.n[b] = int(a.seq_len_host[b]);
-    max_len = d_seq.n[b] > max_len ? d_seq.n[b] : max_len;
+    d_seq.lo[b] = a.lo_host != nullptr ? int(a.lo_host[b]) : 0;
+    d_seq.hi[b] = a.hi_host != nullptr ? int(a.hi_host[b]) : d_seq.n[b];
+    max_len = d_seq.hi[b] - d_seq.lo[b] > max_len ? d_seq.hi[b] - d_seq.lo[b] : max_len;
   }
   uint8_t* w8 = reinterpret_cast<uint8_t*>(a.ws);
   switch (a.Hq / a.Hkv) {

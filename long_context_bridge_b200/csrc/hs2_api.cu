@@ -373,4 +373,163 @@ hs2_status hs2_block_decode(int32_t batch, const int64_t* seq_len, const hs2_bf1
   return cuda_status(launch_decode(a, static_cast<cudaStream_t>(stream)));
 }
 
+// ---------------------------------------------------------------------------
+// decode with each sequence's cache split over ranks
+// ---------------------------------------------------------------------------
+}  // extern "C"
+
+namespace {
+
+// checks shared by the context-parallel decode steps: shape, batch, lengths
+// and each sequence's slice [lo, hi) of its cache on this rank
+hs2_status check_cp(int32_t batch, const int64_t* seq_len, const int64_t* lo, const int64_t* hi,
+                    const hs2_shape* s) {
+  HS2_TRY(check_shape(s, true));
+  HS2_NEED(batch > 0 && seq_len);
+  if (batch > kDecodeMaxBatch || int64_t(batch) * s->T > INT32_MAX) return HS2_ERR_UNSUPPORTED;
+  for (int b = 0; b < batch; ++b) {
+    HS2_NEED(seq_len[b] >= 1 && seq_len[b] <= INT32_MAX);
+    if (lo != nullptr || hi != nullptr) {
+      HS2_NEED(lo && hi && lo[b] >= 0 && lo[b] <= hi[b] && hi[b] <= seq_len[b]);
+      HS2_NEED(hi[b] - lo[b] <= s->T);
+    }
+  }
+  return HS2_OK;
+}
+
+hs2_status check_ranks(int32_t n_ranks, const hs2_shape* s) {
+  HS2_NEED(n_ranks >= 1);
+  if (int64_t(n_ranks) * s->k_global > kDecodeMergeCap) return HS2_ERR_UNSUPPORTED;
+  return HS2_OK;
+}
+
+DecodeArgs cp_args(int step, int32_t batch, const int64_t* seq_len, const int64_t* lo,
+                   const int64_t* hi, const hs2_shape* s) {
+  DecodeArgs a{};
+  a.step = step;
+  a.B = batch;
+  a.seq_len_host = seq_len;
+  a.lo_host = lo;
+  a.hi_host = hi;
+  a.cap = s->T;
+  a.Hq = s->n_q_heads;
+  a.Hkv = s->n_kv_heads;
+  a.scale = s->scale;
+  a.k = s->k_global;
+  a.w = s->window;
+  return a;
+}
+
+bool aligned8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+hs2_status hs2_decode_cp_attn(int32_t batch, const int64_t* seq_len, const int64_t* slice_lo,
+                              const int64_t* slice_hi, const hs2_bf16* q_full,
+                              const hs2_fp8e4m3* Kc, const hs2_fp8e4m3* Vc, const float* k_scale,
+                              const float* v_scale, float* attn_rec, const hs2_shape* s,
+                              void* ws, size_t ws_bytes, void* stream) {
+  HS2_NEED(slice_lo && slice_hi);
+  HS2_TRY(check_cp(batch, seq_len, slice_lo, slice_hi, s));
+  HS2_NEED(q_full && Kc && Vc && k_scale && v_scale && attn_rec);
+  HS2_NEED(aligned16(q_full) && aligned16(Kc) && aligned16(Vc) && aligned16(attn_rec));
+  HS2_NEED((reinterpret_cast<uintptr_t>(k_scale) & 3) == 0 &&
+           (reinterpret_cast<uintptr_t>(v_scale) & 3) == 0);
+  const size_t need = decode_workspace_bytes(batch, s->T, s->n_q_heads, s->n_kv_heads,
+                                             s->k_global, s->window);
+  if (ws == nullptr || ws_bytes < need || !aligned16(ws)) return HS2_ERR_WORKSPACE;
+  DecodeArgs a = cp_args(DEC_CP_ATTN, batch, seq_len, slice_lo, slice_hi, s);
+  a.q = q_full;
+  a.Kc = Kc;
+  a.Vc = Vc;
+  a.ks = k_scale;
+  a.vs = v_scale;
+  a.attn_rec = attn_rec;
+  a.ws = ws;
+  a.ws_bytes = ws_bytes;
+  return cuda_status(launch_decode(a, static_cast<cudaStream_t>(stream)));
+}
+
+hs2_status hs2_decode_cp_select(int32_t batch, const int64_t* seq_len, const int64_t* slice_lo,
+                                const int64_t* slice_hi, int32_t n_ranks, const float* attn_recs,
+                                hs2_bf16* o_full, float* lse, uint32_t* sel_rec,
+                                const hs2_shape* s, void* ws, size_t ws_bytes, void* stream) {
+  HS2_NEED(slice_lo && slice_hi);
+  HS2_TRY(check_cp(batch, seq_len, slice_lo, slice_hi, s));
+  HS2_TRY(check_ranks(n_ranks, s));
+  HS2_NEED(attn_recs && o_full && lse && sel_rec);
+  HS2_NEED(aligned16(attn_recs) && aligned16(o_full) && aligned16(lse) && aligned16(sel_rec));
+  const size_t need = decode_workspace_bytes(batch, s->T, s->n_q_heads, s->n_kv_heads,
+                                             s->k_global, s->window);
+  if (ws == nullptr || ws_bytes < need || !aligned16(ws)) return HS2_ERR_WORKSPACE;
+  DecodeArgs a = cp_args(DEC_CP_SELECT, batch, seq_len, slice_lo, slice_hi, s);
+  a.n_ranks = n_ranks;
+  a.attn_recs = attn_recs;
+  a.o = o_full;
+  a.lse = lse;
+  a.sel_rec = reinterpret_cast<uint2*>(sel_rec);
+  a.ws = ws;
+  a.ws_bytes = ws_bytes;
+  return cuda_status(launch_decode(a, static_cast<cudaStream_t>(stream)));
+}
+
+hs2_status hs2_decode_cp_sparse(int32_t batch, const int64_t* seq_len, const int64_t* slice_lo,
+                                const int64_t* slice_hi, int32_t n_ranks,
+                                const uint32_t* sel_recs, int32_t* idx, const hs2_fp8e4m3* Kc,
+                                const hs2_fp8e4m3* Vc, const float* k_scale,
+                                const float* v_scale, int32_t n_sparse,
+                                const hs2_bf16* const* q_sparse, float* sparse_rec,
+                                const hs2_shape* s, void* stream) {
+  HS2_NEED(slice_lo && slice_hi);
+  HS2_TRY(check_cp(batch, seq_len, slice_lo, slice_hi, s));
+  HS2_TRY(check_ranks(n_ranks, s));
+  HS2_NEED(sel_recs && idx && Kc && Vc && k_scale && v_scale);
+  HS2_NEED(aligned8(sel_recs) && aligned16(idx) && aligned16(Kc) && aligned16(Vc));
+  HS2_NEED((reinterpret_cast<uintptr_t>(k_scale) & 3) == 0 &&
+           (reinterpret_cast<uintptr_t>(v_scale) & 3) == 0);
+  HS2_NEED(n_sparse >= 0 && (n_sparse == 0 || (q_sparse && sparse_rec && aligned16(sparse_rec))));
+  for (int l = 0; l < n_sparse; ++l) HS2_NEED(q_sparse[l] && aligned16(q_sparse[l]));
+  DecodeArgs a = cp_args(DEC_CP_SPARSE, batch, seq_len, slice_lo, slice_hi, s);
+  a.n_ranks = n_ranks;
+  a.sel_recs = reinterpret_cast<const uint2*>(sel_recs);
+  a.idx = idx;
+  a.Kc = Kc;
+  a.Vc = Vc;
+  a.ks = k_scale;
+  a.vs = v_scale;
+  a.n_sparse = n_sparse;
+  a.qs = reinterpret_cast<const void* const*>(q_sparse);
+  a.sparse_rec = sparse_rec;
+  return cuda_status(launch_decode(a, static_cast<cudaStream_t>(stream)));
+}
+
+hs2_status hs2_decode_cp_finish(int32_t batch, int32_t n_ranks, int32_t n_sparse,
+                                const float* sparse_recs, hs2_bf16* const* o_sparse,
+                                const hs2_shape* s, void* stream) {
+  HS2_TRY(check_shape(s, true));
+  HS2_NEED(batch > 0);
+  if (batch > kDecodeMaxBatch) return HS2_ERR_UNSUPPORTED;
+  HS2_TRY(check_ranks(n_ranks, s));
+  HS2_NEED(n_sparse >= 1 && sparse_recs && o_sparse && aligned16(sparse_recs));
+  for (int l = 0; l < n_sparse; ++l) HS2_NEED(o_sparse[l] && aligned16(o_sparse[l]));
+  DecodeArgs a{};
+  a.step = DEC_CP_FINISH;
+  a.B = batch;
+  a.Hq = s->n_q_heads;
+  a.Hkv = s->n_kv_heads;
+  a.k = s->k_global;
+  a.cap = s->T;
+  a.n_ranks = n_ranks;
+  a.n_sparse = n_sparse;
+  a.sparse_recs = sparse_recs;
+  a.os = reinterpret_cast<void* const*>(o_sparse);
+  static const int64_t one = 1;
+  int64_t lens[kDecodeMaxBatch];
+  for (int b = 0; b < batch; ++b) lens[b] = one;
+  a.seq_len_host = lens;
+  return cuda_status(launch_decode(a, static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

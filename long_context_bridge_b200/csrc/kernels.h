@@ -91,6 +91,14 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);
 size_t select_noalloc_scratch_bytes();
 cudaError_t launch_select_noalloc(const SelectArgs& a, cudaStream_t stream);
 
+// Decode with the context split over ranks: per sequence (row) the slice
+// [lo, hi) of its cache that this rank holds.
+constexpr int kMaxSpanRows = 64;
+struct RowSpans {
+  int lo[kMaxSpanRows];
+  int hi[kMaxSpanRows];
+};
+
 struct SparseArgs {
   const void* Q;
   const void* K;
@@ -108,6 +116,8 @@ struct SparseArgs {
   const float* ks;
   const float* vs;
   int64_t cache_T;  // decode: tokens per sequence in the cache
+  RowSpans spans;   // decode: the slice of each sequence's cache to use
+  float* rec;       // decode, nullable: write softmax-state records instead of O
 };
 cudaError_t launch_sparse(const SparseArgs& a, cudaStream_t stream);
 
@@ -123,7 +133,30 @@ int max_fused_layers(int G);
 cudaError_t launch_sparse_fused(const SparseArgs& a, const SparseLayers& lp, int L,
                                 cudaStream_t stream);
 
+// One decode step of the block (DEC_FULL), or one part of it when each
+// sequence's cache is split over ranks (the DEC_CP_* steps, in this order,
+// with an all-gather of the records between consecutive steps).
+enum DecodeStep {
+  DEC_FULL = 0,
+  DEC_CP_ATTN = 1,    // partial attention over the slice -> attn_rec
+  DEC_CP_SELECT = 2,  // merge attn_recs -> o, lse; local top k of the slice -> sel_rec
+  DEC_CP_SPARSE = 3,  // merge sel_recs -> idx; partial sparse layers -> sparse_rec
+  DEC_CP_FINISH = 4   // merge sparse_recs -> o_sparse
+};
+constexpr int kDecodeRecFloats = 130;  // a softmax-state record: m, l, o[128]
+constexpr int kDecodeMergeCap = 8192;  // n_ranks * k records merged per (sequence, KV head)
+
 struct DecodeArgs {
+  int step;
+  const int64_t* lo_host;  // DEC_CP_*: this rank's slice [lo, hi) of each sequence
+  const int64_t* hi_host;
+  int n_ranks;
+  float* attn_rec;           // [B][Hq][130]
+  const float* attn_recs;    // [R][B][Hq][130]
+  uint2* sel_rec;            // [B][Hkv][k]
+  const uint2* sel_recs;     // [R][B][Hkv][k]
+  float* sparse_rec;         // [n_sparse][B][Hq][130]
+  const float* sparse_recs;  // [R][n_sparse][B][Hq][130]
   int B;
   const int64_t* seq_len_host;
   const void* q;

@@ -126,7 +126,8 @@ __global__ void __launch_bounds__(128)
                       const float* __restrict__ vs, const int32_t* __restrict__ idx,
                       __nv_bfloat16* __restrict__ O, float* __restrict__ lse, int64_t rows,
                       int Hkv, int kw, float scale_log2, int64_t cache_T,
-                      const __grid_constant__ SparseLayers lp) {
+                      const __grid_constant__ SparseLayers lp,
+                      const __grid_constant__ RowSpans spans, float* __restrict__ rec) {
   constexpr int HE = NL * G;                      // heads of a pair
   constexpr int NT = (HE + 7) / 8;                // 8-head n-tiles
   static_assert(NL == 1 || (WPR == 1 && !FP8), "layers are fused on the prefill path only");
@@ -152,12 +153,15 @@ __global__ void __launch_bounds__(128)
   const int64_t r = active ? pair % rows : 0;
   const int g = active ? int(pair / rows) : 0;
   const int Hq = Hkv * G;
-  const int64_t tok0 = FP8 ? r * cache_T : 0;  // decode: sequence r's cache rows
+  const int64_t tok0 = FP8 ? r * cache_T : 0;  // decode: sequence r's cache rows,
+  const int jlo = FP8 ? spans.lo[r] : 0;         // holding its positions from jlo
   const int32_t* list = idx + (r * Hkv + g) * kw;
   const int per = (kw + WPR * CS - 1) / (WPR * CS);
   const int e_lo = part * per, e_hi = min(kw, e_lo + per);
-  // valid positions: rows of K/V (prefill) or of a sequence's cache (decode)
-  const int jbound = int(FP8 ? cache_T : rows);
+  // valid positions: rows of K/V (prefill); in decode the list holds absolute
+  // positions and the slice test below keeps every read inside the cache
+  // (its slice [lo, hi) spans at most cache_T rows)
+  const int jbound = FP8 ? INT32_MAX : int(rows);
 
   // query fragments: head nt*8+gid; step s uses the dims that lane t's K
   // loads hold: bf16 dims 64(s/4) + 16t + 4(s%4) + {0..3}, FP8 dims 32t + 4s + {0..3}
@@ -202,7 +206,9 @@ __global__ void __launch_bounds__(128)
   // one step ahead so that a step's gathers do not wait for its list load
   int jl_next = (active && e_lo + (lane & 15) < e_hi) ? __ldg(list + e_lo + (lane & 15)) : -1;
   for (int e0 = e_lo; e0 < e_hi && active; e0 += 16) {
-    const int jl = checked_entry(jl_next, jbound);
+    int jl = checked_entry(jl_next, jbound);
+    // decode with the context split over ranks: only this rank's slice
+    if (FP8 && (jl < spans.lo[r] || jl >= spans.hi[r])) jl = -1;
     const int en = e0 + 16 + (lane & 15);
     jl_next = en < e_hi ? __ldg(list + en) : -1;
     const int jA = __shfl_sync(0xffffffffu, jl, gid), jB = __shfl_sync(0xffffffffu, jl, gid + 8);
@@ -210,8 +216,8 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
     for (int u = 0; u < 4; ++u) jP[u] = __shfl_sync(0xffffffffu, jl, 4 * t + u);
     const bool vA = jA >= 0, vB = jB >= 0;
-    const int64_t rowA = (tok0 + (vA ? jA : 0)) * Hkv + g;
-    const int64_t rowB = (tok0 + (vB ? jB : 0)) * Hkv + g;
+    const int64_t rowA = (tok0 + (vA ? jA - jlo : 0)) * Hkv + g;
+    const int64_t rowB = (tok0 + (vB ? jB - jlo : 0)) * Hkv + g;
 
     // ---- gathers: K rows (this lane's 32 dims), V rows 4t+u (16 dims)
     uint32_t ka[16], kb[16];  // bf16: words; FP8: first 8 hold 32 codes
@@ -236,7 +242,7 @@ __global__ void __launch_bounds__(128)
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int64_t rv = (tok0 + (jP[u] >= 0 ? jP[u] : 0)) * Hkv + g;
+        const int64_t rv = (tok0 + (jP[u] >= 0 ? jP[u] - jlo : 0)) * Hkv + g;
         // lanes gid = 0..7 read a whole 256-byte row, 32 bytes each: dims
         // 16*gid .. +15
         ldg256(reinterpret_cast<const __nv_bfloat16*>(Vp) + rv * 128 + 16 * gid, vw[u]);
@@ -257,7 +263,7 @@ __global__ void __launch_bounds__(128)
       ksB = vB ? __ldg(ks + rowB) : 0.f;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int64_t rv = (tok0 + (jP[u] >= 0 ? jP[u] : 0)) * Hkv + g;
+        const int64_t rv = (tok0 + (jP[u] >= 0 ? jP[u] - jlo : 0)) * Hkv + g;
         const uint4 x = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(Vp) +
                                                              rv * 128 + 16 * gid));
         vw[u][0] = x.x; vw[u][1] = x.y; vw[u][2] = x.z; vw[u][3] = x.w;
@@ -453,13 +459,22 @@ __global__ void __launch_bounds__(128)
             L += *cluster.map_shared_rank(&cL[h], q) * Mr[q];
           }
           const float inv = L > 0.f ? oscale / L : 0.f;
+          // rec: this rank's softmax state over its slice (m, l, o unnormalised)
+          float* rr = rec != nullptr ? rec + (r * Hq + g * G + h) * 130 : nullptr;
           for (int d = lane; d < 128; d += 32) {
             float acc = 0.f;
 #pragma unroll
             for (int q = 0; q < CS; ++q) acc += *cluster.map_shared_rank(&cO[h][d], q) * Mr[q];
-            O[(r * Hq + g * G + h) * 128 + d] = __float2bfloat16_rn(acc * inv);
+            if (rr != nullptr)
+              rr[2 + d] = acc * oscale;
+            else
+              O[(r * Hq + g * G + h) * 128 + d] = __float2bfloat16_rn(acc * inv);
           }
-          if (lse != nullptr && lane == 0)
+          if (rr != nullptr && lane == 0) {
+            rr[0] = M;
+            rr[1] = L;
+          }
+          if (rr == nullptr && lse != nullptr && lane == 0)
             lse[r * Hq + g * G + h] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
         }
       }
@@ -512,12 +527,13 @@ cudaError_t launch_g(const SparseArgs& a, cudaStream_t stream) {
         static_cast<const void*>(a.Vc), static_cast<const float*>(a.ks),
         static_cast<const float*>(a.vs), static_cast<const int32_t*>(a.idx),
         reinterpret_cast<__nv_bfloat16*>(a.O), a.lse, int64_t(a.T), a.Hkv, a.kw, sl2,
-        int64_t(a.cache_T), SparseLayers{});
+        int64_t(a.cache_T), SparseLayers{}, a.spans, a.rec);
     if (e != cudaSuccess) return e;
   } else {
     sparse_mma_kernel<G, false, 1><<<unsigned((pairs + 3) / 4), 128, 0, stream>>>(
         reinterpret_cast<const __nv_bfloat16*>(a.Q), a.K, a.V, nullptr, nullptr, a.idx,
-        reinterpret_cast<__nv_bfloat16*>(a.O), a.lse, a.T, a.Hkv, a.kw, sl2, 0, SparseLayers{});
+        reinterpret_cast<__nv_bfloat16*>(a.O), a.lse, a.T, a.Hkv, a.kw, sl2, 0, SparseLayers{},
+        RowSpans{}, nullptr);
   }
   count_launch();
   return cudaGetLastError();
@@ -529,7 +545,7 @@ cudaError_t launch_fused(const SparseArgs& a, const SparseLayers& lp, cudaStream
   const int64_t pairs = a.T * a.Hkv;
   sparse_mma_kernel<G, false, 1, 1, L><<<unsigned((pairs + 3) / 4), 128, 0, stream>>>(
       nullptr, a.K, a.V, nullptr, nullptr, a.idx, nullptr, nullptr, a.T, a.Hkv, a.kw,
-      a.scale * kLog2e, 0, lp);
+      a.scale * kLog2e, 0, lp, RowSpans{}, nullptr);
   count_launch();
   return cudaGetLastError();
 }

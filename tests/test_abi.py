@@ -107,6 +107,20 @@ def test_host_side_errors(hs2):
                               None) == hs2.ERR_UNSUPPORTED
     with pytest.raises(hs2.HS2Error):
         hs2.workspace_size(hs2.OP_BLOCK_DECODE, sd, 65)
+    # context-parallel decode: a slice past the sequence, a slice longer than
+    # the local cache, too many ranks for the merge of their top-k records
+    i64 = lambda *v: (C.c_int64 * len(v))(*v)
+    sh = hs2.Shape.make(4096, 8, 2)
+    assert L.hs2_decode_cp_attn(1, i64(5000), i64(4000), i64(5001), ok_ptr, ok_ptr, ok_ptr, ok_ptr,
+                                ok_ptr, ok_ptr, C.byref(sh), ok_ptr, 1 << 40,
+                                None) == hs2.ERR_INVALID_ARG
+    assert L.hs2_decode_cp_attn(1, i64(9000), i64(0), i64(4097), ok_ptr, ok_ptr, ok_ptr, ok_ptr,
+                                ok_ptr, ok_ptr, C.byref(sh), ok_ptr, 1 << 40,
+                                None) == hs2.ERR_INVALID_ARG
+    assert L.hs2_decode_cp_select(1, i64(9000), i64(0), i64(4096), 9, ok_ptr, ok_ptr, ok_ptr,
+                                  ok_ptr, C.byref(sh), ok_ptr, 1 << 40, None) == hs2.ERR_UNSUPPORTED
+    assert L.hs2_decode_cp_finish(1, 0, 1, ok_ptr, C.cast(arr, C.POINTER(C.c_void_p)),
+                                  C.byref(sh), None) == hs2.ERR_INVALID_ARG
     assert hs2.hs2_status_string(hs2.ERR_TIMEOUT) == "device-side wait timed out"
     assert hs2.hs2_status_string(hs2.ERR_BAD_INDEX) == "index list entry out of range (skipped)"
 
