@@ -226,6 +226,24 @@ hs2_status hs2_block_prefill(const hs2_bf16* H, int32_t d_model, const hs2_bf16*
                              void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * The block at prefill for a range of query rows, given the K/V of the whole
+ * causal prefix: rows of Q_full, O_full, lse, idx, Q_sparse and O_sparse are
+ * positions q_begin .. q_begin + shape->T - 1; K and V [q_begin + shape->T,
+ * n_kv_heads, 128] hold positions 0 .. q_begin + shape->T - 1.  Every row
+ * is computed exactly as hs2_block_prefill computes it for the whole prompt
+ * (full attention, selection, n_sparse sparse layers), so a prompt can be
+ * split into row ranges over calls or over ranks (each rank with the
+ * all-gathered K/V).  No counterpart on the pages.  q_begin must be a
+ * multiple of 128 (HS2_ERR_UNSUPPORTED otherwise).  No bridge: K/V are
+ * inputs.  Workspace: hs2_workspace_size(HS2_OP_BLOCK_PREFILL, shape, ...).
+ */
+hs2_status hs2_block_prefill_rows(int64_t q_begin, const hs2_bf16* K, const hs2_bf16* V,
+                                  const hs2_bf16* Q_full, hs2_bf16* O_full, float* lse,
+                                  int32_t* idx, int32_t n_sparse, const hs2_bf16* const* Q_sparse,
+                                  hs2_bf16* const* O_sparse, const hs2_shape* shape,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * One decode step of the block over an FP8 KV cache (step S5).  The FP8 KV
  * cache of the zgeo.com.cn comparison table and of the javabetter.cn
  * explainer's 1M-token figures; the cross-decoder runs only while generating.

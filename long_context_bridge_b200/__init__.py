@@ -58,6 +58,7 @@ def _load(path: str = LIB_PATH):
         "hs2_block_prefill": [P, I32, P, P, P, P, P, P, P, P, I32, PP, PP, SP, P, SZ, P],
         "hs2_block_decode": [I32, C.POINTER(C.c_int64), P, P, P, P, P, P, P, P, I32, PP, PP, SP,
                              P, SZ, P],
+        "hs2_block_prefill_rows": [I64, P, P, P, P, P, P, I32, PP, PP, SP, P, SZ, P],
         "hs2_decode_cp_attn": [I32, C.POINTER(C.c_int64), C.POINTER(C.c_int64),
                                C.POINTER(C.c_int64), P, P, P, P, P, P, SP, P, SZ, P],
         "hs2_decode_cp_select": [I32, C.POINTER(C.c_int64), C.POINTER(C.c_int64),
@@ -88,7 +89,8 @@ EXPORTED = ["hs2_bridge_kv", "hs2_bridge_kv_fp8", "hs2_full_attn_lse", "hs2_sele
             "hs2_sparse_attn", "hs2_sparse_attn_layers",
             "hs2_block_prefill", "hs2_block_decode", "hs2_workspace_size",
             "hs2_get_device_status", "hs2_status_string", "hs2_kernel_launches",
-            "hs2_debug_set_wait_budget", "hs2_decode_cp_attn", "hs2_decode_cp_select",
+            "hs2_debug_set_wait_budget", "hs2_block_prefill_rows", "hs2_decode_cp_attn",
+            "hs2_decode_cp_select",
             "hs2_decode_cp_sparse", "hs2_decode_cp_finish"]
 
 
@@ -201,6 +203,18 @@ def hs2_block_prefill(H, W_k, W_v, K, V, Q_full, O_full, lse, idx, Q_sparse, O_s
         _ptr(Q_full, BF16, "Q_full"), _ptr(O_full, BF16, "O_full"), _ptr(lse, F32, "lse"),
         _ptr(idx, I32T, "idx"), len(Q_sparse), qs, os_, C.byref(shape),
         _ptr(workspace, U8, "workspace", True), nbytes, _stream(stream)), "hs2_block_prefill")
+
+
+def hs2_block_prefill_rows(q_begin, K, V, Q_full, O_full, lse, idx, Q_sparse, O_sparse,
+                           shape: Shape, workspace, stream=None):
+    qs, _keep_q = _ptr_array(Q_sparse, BF16, "Q_sparse")
+    os_, _keep_o = _ptr_array(O_sparse, BF16, "O_sparse")
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.hs2_block_prefill_rows(
+        int(q_begin), _ptr(K, BF16, "K"), _ptr(V, BF16, "V"), _ptr(Q_full, BF16, "Q_full"),
+        _ptr(O_full, BF16, "O_full"), _ptr(lse, F32, "lse"), _ptr(idx, I32T, "idx"),
+        len(Q_sparse), qs, os_, C.byref(shape), _ptr(workspace, U8, "workspace", True), nbytes,
+        _stream(stream)), "hs2_block_prefill_rows")
 
 
 def hs2_block_decode(seq_len, q_full, Kc, Vc, k_scale, v_scale, o_full, lse, idx, q_sparse,

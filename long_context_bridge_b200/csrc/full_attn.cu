@@ -68,7 +68,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     full_attn_kernel(const __grid_constant__ CUtensorMap tmQ,
                      const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ O,
-                     float* __restrict__ lse, int T, int Hkv, float scale_log2) {
+                     float* __restrict__ lse, int T, int Hkv, float scale_log2, int q_begin) {
   constexpr int QT = TILE / G;  // queries per Q tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -82,8 +82,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   int q0[2], n_t[2];
 #pragma unroll
   for (int X = 0; X < 2; ++X) {
+    // rows of Q/O/lse are positions q_begin + row (q_begin a multiple of
+    // TILE), so a Q tile's queries share one diagonal K tile
     q0[X] = (2 * pr + X) * QT;
-    n_t[X] = q0[X] < T ? (min(q0[X] + QT, T) - 1) / TILE + 1 : 0;
+    n_t[X] = q0[X] < T ? (q_begin + min(q0[X] + QT, T) - 1) / TILE + 1 : 0;
   }
   const int n_max = max(n_t[0], n_t[1]);
 
@@ -206,7 +208,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int sub = warp & 3;
     const int row = sub * 32 + lane;            // TMEM lane == tile row
     const int q0X = X ? q0[1] : q0[0];
-    const int qi = q0X + row / G;               // this row's query position
+    const int qi = q0X + row / G;               // this row of Q/O/lse
+    const int qpos = q_begin + qi;              // and its position
     const int h = g * G + row % G;              // and head
     const uint32_t lane_addr = uint32_t(sub * 32) << 16;
     const uint32_t tS = tmem + lane_addr + X * 256, tO = tS + 128;
@@ -227,7 +230,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(r[e]);
       }
       if (j == n - 1) {  // causal mask on the diagonal tile
-        const int lim = qi - j * TILE;  // keys with column > lim are masked
+        const int lim = qpos - j * TILE;  // keys with column > lim are masked
 #pragma unroll
         for (int e = 0; e < 128; ++e)
           if (e > lim) x[e] = -INFINITY;
@@ -327,10 +330,11 @@ cudaError_t launch_g(const AttnArgs& a, cudaStream_t stream) {
   // Q [T, Hq, 128]: box 64 dims x G heads x QT tokens -> 128 rows of 128 B
   if (!make_tmap_3d(&tmQ, a.Q, 128, a.Hq, a.T, 256, uint64_t(a.Hq) * 256, 64, G, QT))
     return cudaErrorInvalidValue;
-  // K, V [T, Hkv, 128]: box 64 dims x 1 head x 128 tokens
-  if (!make_tmap_3d(&tmK, a.K, 128, a.Hkv, a.T, 256, uint64_t(a.Hkv) * 256, 64, 1, TILE))
+  // K, V [q_begin + T, Hkv, 128]: box 64 dims x 1 head x 128 tokens
+  const uint64_t kv_rows = uint64_t(a.q_begin + a.T);
+  if (!make_tmap_3d(&tmK, a.K, 128, a.Hkv, kv_rows, 256, uint64_t(a.Hkv) * 256, 64, 1, TILE))
     return cudaErrorInvalidValue;
-  if (!make_tmap_3d(&tmV, a.V, 128, a.Hkv, a.T, 256, uint64_t(a.Hkv) * 256, 64, 1, TILE))
+  if (!make_tmap_3d(&tmV, a.V, 128, a.Hkv, kv_rows, 256, uint64_t(a.Hkv) * 256, 64, 1, TILE))
     return cudaErrorInvalidValue;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(full_attn_kernel<G>), SMEM);
   if (e != cudaSuccess) return e;
@@ -338,7 +342,7 @@ cudaError_t launch_g(const AttnArgs& a, cudaStream_t stream) {
   const dim3 grid(unsigned((nqb + 1) / 2), unsigned(a.Hkv));
   full_attn_kernel<G><<<grid, THREADS, SMEM, stream>>>(
       tmQ, tmK, tmV, reinterpret_cast<__nv_bfloat16*>(a.O), a.lse, int(a.T), a.Hkv,
-      a.scale * kLog2e);
+      a.scale * kLog2e, int(a.q_begin));
   count_launch();
   return cudaGetLastError();
 }

@@ -327,6 +327,47 @@ hs2_status hs2_block_prefill(const hs2_bf16* H, int32_t d_model, const hs2_bf16*
   return HS2_OK;
 }
 
+hs2_status hs2_block_prefill_rows(int64_t q_begin, const hs2_bf16* K, const hs2_bf16* V,
+                                  const hs2_bf16* Q_full, hs2_bf16* O_full, float* lse,
+                                  int32_t* idx, int32_t n_sparse, const hs2_bf16* const* Q_sparse,
+                                  hs2_bf16* const* O_sparse, const hs2_shape* s, void* ws,
+                                  size_t ws_bytes, void* stream) {
+  HS2_TRY(check_shape(s, true));
+  HS2_NEED(q_begin >= 0);
+  if (q_begin % 128 != 0 || q_begin + s->T > INT32_MAX) return HS2_ERR_UNSUPPORTED;
+  HS2_NEED(K && V && Q_full && O_full && lse && idx);
+  HS2_NEED(aligned16(K) && aligned16(V) && aligned16(Q_full) && aligned16(O_full) &&
+           aligned16(lse) && aligned16(idx));
+  HS2_NEED(n_sparse >= 0 && (n_sparse == 0 || (Q_sparse && O_sparse)));
+  for (int l = 0; l < n_sparse; ++l)
+    HS2_NEED(Q_sparse[l] && O_sparse[l] && aligned16(Q_sparse[l]) && aligned16(O_sparse[l]));
+  const size_t need =
+      select_workspace_bytes(s->T, s->n_q_heads, s->n_kv_heads, s->k_global, s->window);
+  if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws))) return HS2_ERR_WORKSPACE;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  AttnArgs fa{Q_full, K, V, O_full, lse, s->T, s->n_q_heads, s->n_kv_heads, s->scale, q_begin};
+  HS2_TRY(cuda_status(launch_full_attn(fa, st)));
+  SelectArgs sa{Q_full, K, lse, idx, nullptr, s->T, s->n_q_heads, s->n_kv_heads, s->scale,
+                s->k_global, s->window, ws, ws_bytes, q_begin};
+  HS2_TRY(cuda_status(launch_select(sa, st)));
+  for (int l = 0; l < n_sparse; ++l) {
+    SparseArgs a{};
+    a.Q = Q_sparse[l];
+    a.K = K;
+    a.V = V;
+    a.idx = idx;
+    a.O = O_sparse[l];
+    a.T = s->T;
+    a.Hq = s->n_q_heads;
+    a.Hkv = s->n_kv_heads;
+    a.scale = s->scale;
+    a.kw = s->k_global + s->window;
+    a.kv_rows = q_begin + s->T;
+    HS2_TRY(cuda_status(launch_sparse(a, st)));
+  }
+  return HS2_OK;
+}
+
 hs2_status hs2_block_decode(int32_t batch, const int64_t* seq_len, const hs2_bf16* q_full,
                             const hs2_fp8e4m3* Kc, const hs2_fp8e4m3* Vc, const float* k_scale,
                             const float* v_scale, hs2_bf16* o_full, float* lse, int32_t* idx,

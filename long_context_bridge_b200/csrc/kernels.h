@@ -66,9 +66,10 @@ struct AttnArgs {
   const void* V;
   void* O;
   float* lse;
-  int64_t T;
+  int64_t T;        // rows of Q/O/lse
   int Hq, Hkv;
   float scale;
+  int64_t q_begin;  // position of row 0 (a multiple of 128); K/V hold q_begin + T rows
 };
 cudaError_t launch_full_attn(const AttnArgs& a, cudaStream_t stream);
 
@@ -78,12 +79,13 @@ struct SelectArgs {
   const float* lse;
   int32_t* idx;
   float* kth;
-  int64_t T;
+  int64_t T;        // rows of Q/lse/idx/kth
   int Hq, Hkv;
   float scale;
   int k, w;
   void* ws;
   size_t ws_bytes;
+  int64_t q_begin;  // position of row 0 (a multiple of 128); K holds q_begin + T rows
 };
 size_t select_workspace_bytes(int64_t T, int Hq, int Hkv, int k, int w);
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);
@@ -110,6 +112,7 @@ struct SparseArgs {
   int Hq, Hkv;
   float scale;
   int kw;     // entries per list (k + w)
+  int64_t kv_rows;  // prefill: rows of K/V (list entries must lie below it)
   // FP8 source (decode): codes + per-(token, head) scales; K/V above unused
   const uint8_t* Kc;
   const uint8_t* Vc;

@@ -344,7 +344,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     select_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const float* __restrict__ lse, int32_t* __restrict__ idx,
                   float* __restrict__ kth, uint2* __restrict__ ws, uint32_t* __restrict__ wsort,
-                  int T, int Hkv, int k, int w, int capw, int kst, float scale_log2) {
+                  int T, int Hkv, int k, int w, int capw, int kst, float scale_log2, int q_begin) {
   using Cfg = SelCfg<G>;
   constexpr int QT = Cfg::QT, QH = Cfg::QH, NB = Cfg::NB, BSHIFT = Cfg::BSHIFT;
   extern __shared__ uint8_t smem_raw[];
@@ -361,13 +361,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t top = __float_as_uint(float(G)) >> BSHIFT;
   const uint32_t lo = top - (NB - 1);
 
+  // rows of Q/lse/idx are positions q_begin + row (q_begin a multiple of TILE)
   auto item = [&](int it, int& q0, int& g, int& n_tiles, bool& score) {
     // KV-head-major, heaviest query blocks first within a head, so that the
     // CTAs running at one time stream the same head's K through L2
     const int qb = nqb - 1 - it % nqb;
     g = it / nqb;
     q0 = qb * QT;
-    const int q_last = min(q0 + QT, T) - 1;
+    const int q_last = q_begin + min(q0 + QT, T) - 1;  // position of the item's last query
     score = k > 0 && (q_last - w + 1) > k;
     n_tiles = score ? (q_last - w) / TILE + 1 : 0;
   };
@@ -490,7 +491,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       // tiles whose every key is a candidate of every query of the set need no
       // per-key test: keys up to q0 + qb0 - w are candidates of query qb0
       const bool all_exist = qvalid >= QH;
-      const int last_free = q0 + qb0 - w;
+      const int last_free = q_begin + q0 + qb0 - w;
       const float* nlw = &ms->nlse2[half * 32];
       uint32_t n[QH], fl[QH];  // appended entries and floors of this warp's queries
 #pragma unroll
@@ -533,7 +534,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         // candidates at or above the floor go to this warp's sub-buffer of
         // the query, in position order; each append is counted by score bin
         const bool chk = !all_exist || t * TILE + TILE - 1 > last_free;
-        const int dpos = j + w - q0 - qb0;  // candidate of query qb0 + qq iff dpos <= qq
+        const int dpos = j + w - q_begin - q0 - qb0;  // candidate of query qb0 + qq iff dpos <= qq
 #pragma unroll
         for (int qq = 0; qq < QH; ++qq) {
           const uint32_t bits = __float_as_uint(sc[qq]);
@@ -576,10 +577,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t* sp = wsort + (size_t(blockIdx.x) * SCORER_WARPS + sw) * kSortWords;  // positions
       uint2* bl = reinterpret_cast<uint2*>(sp + 2048);                               // boundary bin
       for (int q = sw; q < QT; q += SCORER_WARPS) {
-        const int qpos = q0 + q;
-        if (qpos >= T) continue;
+        const int qrow = q0 + q;
+        if (qrow >= T) continue;
+        const int qpos = q_begin + qrow;  // its position
         const int ncand = max(0, qpos - w + 1);
-        int32_t* out = idx + (size_t(qpos) * Hkv + g) * (k + w);
+        int32_t* out = idx + (size_t(qrow) * Hkv + g) * (k + w);
         float kv = -1.f;
         if (!score || ncand <= k) {
           for (int e = lane; e < k; e += 32) out[e] = e < ncand ? e : -1;
@@ -740,7 +742,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           const int p = qpos - w + 1 + t2;
           out[k + t2] = p >= 0 ? p : -1;
         }
-        if (kth != nullptr && lane == 0) kth[size_t(qpos) * Hkv + g] = kv;
+        if (kth != nullptr && lane == 0) kth[size_t(qrow) * Hkv + g] = kv;
       }
       scorer_sync();
     }
@@ -775,7 +777,8 @@ cudaError_t launch_g(const SelectArgs& a, cudaStream_t stream) {
   CUtensorMap tmQ, tmK;
   if (!make_tmap_3d(&tmQ, a.Q, 128, a.Hq, a.T, 256, uint64_t(a.Hq) * 256, 64, G, QT))
     return cudaErrorInvalidValue;
-  if (!make_tmap_3d(&tmK, a.K, 128, a.Hkv, a.T, 256, uint64_t(a.Hkv) * 256, 64, 1, TILE))
+  if (!make_tmap_3d(&tmK, a.K, 128, a.Hkv, uint64_t(a.q_begin + a.T), 256,
+                    uint64_t(a.Hkv) * 256, 64, 1, TILE))
     return cudaErrorInvalidValue;
   const int kst = stages_for<G>();
   const int smem = OFF_K + kst * TILE_BYTES + int(sizeof(Misc<G>)) + 1024;
@@ -787,7 +790,7 @@ cudaError_t launch_g(const SelectArgs& a, cudaStream_t stream) {
   uint32_t* wsort = reinterpret_cast<uint32_t*>(ws + size_t(sm_count()) * 4 * QT * buffer_cap(a.k));
   select_kernel<G><<<grid, THREADS, smem, stream>>>(tmQ, tmK, a.lse, a.idx, a.kth, ws, wsort,
                                                     int(a.T), a.Hkv, a.k, a.w, buffer_cap(a.k),
-                                                    kst, a.scale * kLog2e);
+                                                    kst, a.scale * kLog2e, int(a.q_begin));
   count_launch();
   return cudaGetLastError();
 }
@@ -834,7 +837,8 @@ cudaError_t launch_noalloc_g(const SelectArgs& a, void* scratch, cudaStream_t st
   CUtensorMap tmQ, tmK;
   if (!make_tmap_3d(&tmQ, a.Q, 128, a.Hq, a.T, 256, uint64_t(a.Hq) * 256, 64, G, QT))
     return cudaErrorInvalidValue;
-  if (!make_tmap_3d(&tmK, a.K, 128, a.Hkv, a.T, 256, uint64_t(a.Hkv) * 256, 64, 1, TILE))
+  if (!make_tmap_3d(&tmK, a.K, 128, a.Hkv, uint64_t(a.q_begin + a.T), 256,
+                    uint64_t(a.Hkv) * 256, 64, 1, TILE))
     return cudaErrorInvalidValue;
   const int kst = stages_for<G>();
   const int smem = OFF_K + kst * TILE_BYTES + int(sizeof(Misc<G>)) + 1024;
@@ -846,7 +850,7 @@ cudaError_t launch_noalloc_g(const SelectArgs& a, void* scratch, cudaStream_t st
   uint32_t* wsort = reinterpret_cast<uint32_t*>(ws + size_t(grid) * 4 * QT * buffer_cap(a.k));
   select_kernel<G><<<grid, THREADS, smem, stream>>>(tmQ, tmK, a.lse, a.idx, a.kth, ws, wsort,
                                                     int(a.T), a.Hkv, a.k, a.w, buffer_cap(a.k),
-                                                    kst, a.scale * kLog2e);
+                                                    kst, a.scale * kLog2e, int(a.q_begin));
   count_launch();
   return cudaGetLastError();
 }

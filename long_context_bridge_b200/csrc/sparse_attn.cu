@@ -158,10 +158,10 @@ __global__ void __launch_bounds__(128)
   const int32_t* list = idx + (r * Hkv + g) * kw;
   const int per = (kw + WPR * CS - 1) / (WPR * CS);
   const int e_lo = part * per, e_hi = min(kw, e_lo + per);
-  // valid positions: rows of K/V (prefill); in decode the list holds absolute
-  // positions and the slice test below keeps every read inside the cache
-  // (its slice [lo, hi) spans at most cache_T rows)
-  const int jbound = FP8 ? INT32_MAX : int(rows);
+  // valid positions: rows of K/V (prefill: cache_T holds their count); in
+  // decode the list holds absolute positions and the slice test below keeps
+  // every read inside the cache (its slice [lo, hi) spans at most cache_T rows)
+  const int jbound = FP8 ? INT32_MAX : int(cache_T);
 
   // query fragments: head nt*8+gid; step s uses the dims that lane t's K
   // loads hold: bf16 dims 64(s/4) + 16t + 4(s%4) + {0..3}, FP8 dims 32t + 4s + {0..3}
@@ -532,8 +532,8 @@ cudaError_t launch_g(const SparseArgs& a, cudaStream_t stream) {
   } else {
     sparse_mma_kernel<G, false, 1><<<unsigned((pairs + 3) / 4), 128, 0, stream>>>(
         reinterpret_cast<const __nv_bfloat16*>(a.Q), a.K, a.V, nullptr, nullptr, a.idx,
-        reinterpret_cast<__nv_bfloat16*>(a.O), a.lse, a.T, a.Hkv, a.kw, sl2, 0, SparseLayers{},
-        RowSpans{}, nullptr);
+        reinterpret_cast<__nv_bfloat16*>(a.O), a.lse, a.T, a.Hkv, a.kw, sl2,
+        a.kv_rows > 0 ? a.kv_rows : a.T, SparseLayers{}, RowSpans{}, nullptr);
   }
   count_launch();
   return cudaGetLastError();
@@ -545,7 +545,7 @@ cudaError_t launch_fused(const SparseArgs& a, const SparseLayers& lp, cudaStream
   const int64_t pairs = a.T * a.Hkv;
   sparse_mma_kernel<G, false, 1, 1, L><<<unsigned((pairs + 3) / 4), 128, 0, stream>>>(
       nullptr, a.K, a.V, nullptr, nullptr, a.idx, nullptr, nullptr, a.T, a.Hkv, a.kw,
-      a.scale * kLog2e, 0, lp, RowSpans{}, nullptr);
+      a.scale * kLog2e, a.kv_rows > 0 ? a.kv_rows : a.T, lp, RowSpans{}, nullptr);
   count_launch();
   return cudaGetLastError();
 }

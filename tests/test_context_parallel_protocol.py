@@ -155,3 +155,56 @@ def test_context_parallel_decode_protocol_on_two_gloo_ranks():
         assert o["n_diff"] == 0
     # every rank ends with the same outputs
     assert outs[0]["checksum"] == outs[1]["checksum"] and outs[0]["idx_sum"] == outs[1]["idx_sum"]
+
+
+PREFILL_WORKER = r"""
+import json, os, sys
+sys.path.insert(0, {root!r})
+import numpy as np, torch
+import torch.distributed as dist
+from long_context_bridge_b200 import Shape
+from long_context_bridge_b200 import context_parallel as cp
+rank, world = int(os.environ["RANK"]), int(os.environ["WORLD_SIZE"])
+dist.init_process_group("gloo")
+T = 4 * world * 128
+K = torch.from_numpy(np.random.default_rng(3).standard_normal((T, 2, 128)).astype(np.float32))
+x = cp.PrefillRows(Shape.make(T, 8, 2), world, rank, "cpu")
+rows = x.rows()
+got = x.assemble(cp.dist_all_gather()(K[rows].contiguous()))  # this rank's rows only, exchanged
+print(json.dumps({{"rank": rank, "chunks": x.chunks, "same": bool(torch.equal(got, K)),
+                   "work": int((rows + 1).sum())}}), flush=True)
+dist.barrier()
+dist.destroy_process_group()
+"""
+
+
+def test_prefill_rows_exchange_on_gloo_ranks():
+    """Row-sharded prefill: with R ranks owning zig-zag chunks r and 2R-1-r,
+    exchanging each rank's own rows of K/V and reassembling them gives the
+    whole prompt's K/V on every rank, and every rank's causal work (the sum
+    over its rows of the keys each row attends to) is the same."""
+    for world in (2, 3):
+        port = _free_port()
+        code = PREFILL_WORKER.format(root=ROOT)
+        procs = []
+        for r in range(world):
+            env = dict(os.environ)
+            env.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(r),
+                       WORLD_SIZE=str(world), LOCAL_RANK=str(r))
+            procs.append(subprocess.Popen([sys.executable, "-c", code], env=env, cwd=ROOT,
+                                          stdout=subprocess.PIPE, stderr=subprocess.PIPE,
+                                          text=True))
+        outs = []
+        for p in procs:
+            try:
+                out, err = p.communicate(timeout=300)
+            except subprocess.TimeoutExpired:
+                for q in procs:
+                    q.kill()
+                raise
+            assert p.returncode == 0, err
+            outs.append(json.loads(out.strip().splitlines()[-1]))
+        assert all(o["same"] for o in outs)
+        assert len({o["work"] for o in outs}) == 1
+        spans = sorted(tuple(c) for o in outs for c in o["chunks"])
+        assert spans[0][0] == 0 and all(a[1] == b[0] for a, b in zip(spans, spans[1:]))

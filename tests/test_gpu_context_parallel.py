@@ -109,3 +109,50 @@ def test_decode_context_parallel_virtual_ranks(hs2, orc, R, lens):
                 kvs[b], qs[l][b:b + 1], gi[b:b + 1], sc)[0][0]
             assert_close_bf16(host_f64(got["os"][l])[b], want, f"o_sparse[{l}][{b}]")
     assert n_diff <= 1
+
+
+@pytest.mark.parametrize("R,T,Hq,Hkv", [(2, 8192, 16, 2), (4, 8192, 8, 1), (2, 4096, 32, 4)])
+def test_prefill_rows_split_over_virtual_ranks(hs2, R, T, Hq, Hkv):
+    """Row-sharded prefill on one GPU: R virtual ranks each bridge their
+    zig-zag chunks' rows, their K/V are stacked as an all-gather would and
+    reassembled, and each rank runs hs2_block_prefill_rows on its chunks.
+    Every row must equal, bit for bit, what the single-device
+    hs2_block_prefill (bridge inside) computes for the whole prompt: the rows
+    of a chunk see the same K/V tiles in the same order."""
+    import torch
+    from long_context_bridge_b200 import context_parallel as cp
+    cfg = synth.BlockConfig("row-sharded prefill", 8, T, Hq, Hkv, d_model=2048, q_mix=True)
+    H, Wk, Wv = synth.bridge_inputs_torch(cfg)
+    Q = synth.q_rows_torch(cfg, synth.TID_Q)
+    Qs = [synth.q_rows_torch(cfg, synth.TID_QS0 + l) for l in range(2)]
+    shape = hs2.Shape.make(T, Hq, Hkv)
+    # one device, the whole prompt
+    K1 = torch.empty(T, Hkv, 128, dtype=torch.bfloat16, device="cuda")
+    V1 = torch.empty_like(K1)
+    O1, Os1 = torch.empty_like(Q), [torch.empty_like(Q) for _ in Qs]
+    lse1 = torch.empty(T, Hq, dtype=torch.float32, device="cuda")
+    idx1 = torch.empty(T, Hkv, 1152, dtype=torch.int32, device="cuda")
+    ws = torch.empty(hs2.workspace_size(hs2.OP_BLOCK_PREFILL, shape), dtype=torch.uint8,
+                     device="cuda")
+    hs2.hs2_block_prefill(H, Wk, Wv, K1, V1, Q, O1, lse1, idx1, Qs, Os1, shape, ws)
+    # R virtual ranks
+    ranks = [cp.PrefillRows(shape, R, r, "cuda") for r in range(R)]
+    own = [x.bridge(H[x.rows().cuda()].contiguous(), Wk, Wv) for x in ranks]
+    Kg = torch.stack([k for k, _ in own])
+    Vg = torch.stack([v for _, v in own])
+    for x in ranks:
+        K, V = x.assemble(Kg), x.assemble(Vg)
+        assert torch.equal(K, K1) and torch.equal(V, V1)
+        rows = x.rows().cuda()
+        n = rows.numel()
+        O, Os = torch.empty(n, Hq, 128, dtype=torch.bfloat16, device="cuda"), None
+        Os = [torch.empty_like(O) for _ in Qs]
+        lse = torch.empty(n, Hq, dtype=torch.float32, device="cuda")
+        idx = torch.empty(n, Hkv, 1152, dtype=torch.int32, device="cuda")
+        x.block(K, V, Q[rows].contiguous(), O, lse, idx, [q[rows].contiguous() for q in Qs], Os)
+        assert hs2.hs2_get_device_status() == hs2.OK
+        assert torch.equal(O, O1[rows]), f"rank {x.rank}: O_full"
+        assert torch.equal(lse, lse1[rows]), f"rank {x.rank}: lse"
+        assert torch.equal(idx, idx1[rows]), f"rank {x.rank}: idx"
+        for l in range(len(Qs)):
+            assert torch.equal(Os[l], Os1[l][rows]), f"rank {x.rank}: O_sparse[{l}]"
