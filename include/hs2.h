@@ -355,6 +355,15 @@ hs2_status hs2_get_device_status(void* stream);
  * while library kernels run. */
 hs2_status hs2_debug_set_wait_budget(int64_t cycles);
 
+/* Measurement hook, not part of the block: `reps` passes of 16-byte loads
+ * through L2 over the DEVICE buffer buf (16-byte aligned, bytes a multiple
+ * of 16) by a grid of 4 CTAs per SM, for the read-bandwidth denominator of a
+ * roofline (a buffer that fits in L2 measures L2, a larger one HBM).  sink:
+ * one DEVICE uint32, written only in the rare event that all loaded words
+ * fold to one constant. */
+hs2_status hs2_debug_read_probe(const void* buf, size_t bytes, int32_t reps, uint32_t* sink,
+                                void* stream);
+
 /* Static English text for a status code. */
 const char* hs2_status_string(hs2_status status);
 

@@ -59,6 +59,7 @@ def _load(path: str = LIB_PATH):
         "hs2_block_decode": [I32, C.POINTER(C.c_int64), P, P, P, P, P, P, P, P, I32, PP, PP, SP,
                              P, SZ, P],
         "hs2_block_prefill_rows": [I64, P, P, P, P, P, P, I32, PP, PP, SP, P, SZ, P],
+        "hs2_debug_read_probe": [P, SZ, I32, P, P],
         "hs2_decode_cp_attn": [I32, C.POINTER(C.c_int64), C.POINTER(C.c_int64),
                                C.POINTER(C.c_int64), P, P, P, P, P, P, SP, P, SZ, P],
         "hs2_decode_cp_select": [I32, C.POINTER(C.c_int64), C.POINTER(C.c_int64),
@@ -89,7 +90,8 @@ EXPORTED = ["hs2_bridge_kv", "hs2_bridge_kv_fp8", "hs2_full_attn_lse", "hs2_sele
             "hs2_sparse_attn", "hs2_sparse_attn_layers",
             "hs2_block_prefill", "hs2_block_decode", "hs2_workspace_size",
             "hs2_get_device_status", "hs2_status_string", "hs2_kernel_launches",
-            "hs2_debug_set_wait_budget", "hs2_block_prefill_rows", "hs2_decode_cp_attn",
+            "hs2_debug_set_wait_budget", "hs2_debug_read_probe", "hs2_block_prefill_rows",
+            "hs2_decode_cp_attn",
             "hs2_decode_cp_select",
             "hs2_decode_cp_sparse", "hs2_decode_cp_finish"]
 
@@ -286,6 +288,13 @@ def hs2_get_device_status(stream=None) -> int:
 def hs2_debug_set_wait_budget(cycles: int) -> None:
     """Testing hook: spin budget of the kernels' bounded waits (<= 0: default)."""
     _check(_lib.hs2_debug_set_wait_budget(int(cycles)), "hs2_debug_set_wait_budget")
+
+
+def hs2_debug_read_probe(buf, reps: int, sink, stream=None) -> None:
+    """Measurement hook: `reps` passes of 16-byte loads over the uint8 buffer."""
+    _check(_lib.hs2_debug_read_probe(_ptr(buf, U8, "buf"), buf.numel(), int(reps),
+                                     _ptr(sink, I32T, "sink"), _stream(stream)),
+           "hs2_debug_read_probe")
 
 
 def hs2_kernel_launches() -> int:

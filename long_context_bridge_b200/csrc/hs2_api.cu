@@ -154,6 +154,12 @@ hs2_status hs2_get_device_status(void* stream) {
   return HS2_OK;
 }
 
+hs2_status hs2_debug_read_probe(const void* buf, size_t bytes, int32_t reps, uint32_t* sink,
+                                void* stream) {
+  HS2_NEED(buf && sink && aligned16(buf) && bytes >= 16 && bytes % 16 == 0 && reps >= 1);
+  return cuda_status(launch_read_probe(buf, bytes, reps, sink, static_cast<cudaStream_t>(stream)));
+}
+
 hs2_status hs2_debug_set_wait_budget(int64_t cycles) {
   const long long c = cycles > 0 ? static_cast<long long>(cycles) : kWaitBudgetCycles;
   cudaError_t e = budget_bridge(c);

@@ -185,4 +185,8 @@ constexpr int kDecodeMaxBatch = 64;
 size_t decode_workspace_bytes(int B, int64_t cap, int Hq, int Hkv, int k, int w);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 
+// read-bandwidth probe (measurement only): `reps` passes of 16-byte loads
+cudaError_t launch_read_probe(const void* buf, size_t bytes, int reps, uint32_t* sink,
+                              cudaStream_t stream);
+
 }  // namespace hs2
