@@ -355,6 +355,16 @@ hs2_status hs2_get_device_status(void* stream);
  * while library kernels run. */
 hs2_status hs2_debug_set_wait_budget(int64_t cycles);
 
+/* Testing hook, not part of the block: hs2_select_topk (and the block calls
+ * that select) start each work item's score floor at `factor` times the
+ * smallest k-th best score of the same CTA's previous item of that KV head
+ * (default 0.9; <= 0 turns this off).  A floor above an item's true k-th best
+ * is detected (a query ends with fewer than k buffered candidates) and the
+ * item is recomputed without it by a second launch, so results never depend
+ * on the factor; a factor of 1e30 forces every such item through that
+ * recomputation.  Process-wide host state; not thread-safe. */
+hs2_status hs2_debug_set_select_speculation(float factor);
+
 /* Measurement hook, not part of the block: `reps` passes of 16-byte loads
  * through L2 over the DEVICE buffer buf (16-byte aligned, bytes a multiple
  * of 16) by a grid of 4 CTAs per SM, for the read-bandwidth denominator of a

@@ -60,6 +60,7 @@ def _load(path: str = LIB_PATH):
                              P, SZ, P],
         "hs2_block_prefill_rows": [I64, P, P, P, P, P, P, I32, PP, PP, SP, P, SZ, P],
         "hs2_debug_read_probe": [P, SZ, I32, P, P],
+        "hs2_debug_set_select_speculation": [C.c_float],
         "hs2_decode_cp_attn": [I32, C.POINTER(C.c_int64), C.POINTER(C.c_int64),
                                C.POINTER(C.c_int64), P, P, P, P, P, P, SP, P, SZ, P],
         "hs2_decode_cp_select": [I32, C.POINTER(C.c_int64), C.POINTER(C.c_int64),
@@ -91,6 +92,7 @@ EXPORTED = ["hs2_bridge_kv", "hs2_bridge_kv_fp8", "hs2_full_attn_lse", "hs2_sele
             "hs2_block_prefill", "hs2_block_decode", "hs2_workspace_size",
             "hs2_get_device_status", "hs2_status_string", "hs2_kernel_launches",
             "hs2_debug_set_wait_budget", "hs2_debug_read_probe", "hs2_block_prefill_rows",
+            "hs2_debug_set_select_speculation",
             "hs2_decode_cp_attn",
             "hs2_decode_cp_select",
             "hs2_decode_cp_sparse", "hs2_decode_cp_finish"]
@@ -295,6 +297,12 @@ def hs2_debug_read_probe(buf, reps: int, sink, stream=None) -> None:
     _check(_lib.hs2_debug_read_probe(_ptr(buf, U8, "buf"), buf.numel(), int(reps),
                                      _ptr(sink, I32T, "sink"), _stream(stream)),
            "hs2_debug_read_probe")
+
+
+def hs2_debug_set_select_speculation(factor: float) -> None:
+    """Testing hook: starting fraction of the selection's speculative floor."""
+    _check(_lib.hs2_debug_set_select_speculation(float(factor)),
+           "hs2_debug_set_select_speculation")
 
 
 def hs2_kernel_launches() -> int:

@@ -160,6 +160,12 @@ hs2_status hs2_debug_read_probe(const void* buf, size_t bytes, int32_t reps, uin
   return cuda_status(launch_read_probe(buf, bytes, reps, sink, static_cast<cudaStream_t>(stream)));
 }
 
+hs2_status hs2_debug_set_select_speculation(float factor) {
+  if (factor != factor) return HS2_ERR_INVALID_ARG;
+  select_set_speculation(factor);
+  return HS2_OK;
+}
+
 hs2_status hs2_debug_set_wait_budget(int64_t cycles) {
   const long long c = cycles > 0 ? static_cast<long long>(cycles) : kWaitBudgetCycles;
   cudaError_t e = budget_bridge(c);

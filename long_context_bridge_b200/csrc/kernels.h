@@ -91,6 +91,9 @@ size_t select_workspace_bytes(int64_t T, int Hq, int Hkv, int k, int w);
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);
 // same kernel on the library's own file-scope scratch (no workspace argument)
 size_t select_noalloc_scratch_bytes();
+// fraction of the previous item's smallest k-th score that starts an item's
+// floor in hs2_select_topk (<= 0: no speculation); testing hook
+void select_set_speculation(float factor);
 cudaError_t launch_select_noalloc(const SelectArgs& a, cudaStream_t stream);
 
 // Decode with the context split over ranks: per sequence (row) the slice

@@ -102,6 +102,10 @@ struct Misc {
   uint32_t cnt[4][QT];        // entries in each sub-buffer
   alignas(16) uint32_t hist[QT][NB];  // appended entries per score bin
   uint32_t dig[SCORER_WARPS][256];    // per-warp radix histograms
+  uint32_t spec_bits;   // speculative floor for the CTA's next item of head spec_g (0: none)
+  int32_t spec_g;
+  uint32_t spec_min;    // smallest k-th best score (bits) among the item's queries
+  uint32_t item_fail;   // a query of the item ended with fewer than k buffered entries
 };
 
 // 16-byte vector accesses to the histograms and the lse rows
@@ -344,7 +348,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     select_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const float* __restrict__ lse, int32_t* __restrict__ idx,
                   float* __restrict__ kth, uint2* __restrict__ ws, uint32_t* __restrict__ wsort,
-                  int T, int Hkv, int k, int w, int capw, int kst, float scale_log2, int q_begin) {
+                  int T, int Hkv, int k, int w, int capw, int kst, float scale_log2, int q_begin,
+                  float spec_factor, const int32_t* __restrict__ item_list,
+                  uint32_t* __restrict__ fail_count, int32_t* __restrict__ fail_list) {
   using Cfg = SelCfg<G>;
   constexpr int QT = Cfg::QT, QH = Cfg::QH, NB = Cfg::NB, BSHIFT = Cfg::BSHIFT;
   extern __shared__ uint8_t smem_raw[];
@@ -355,7 +361,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int warp = warp_id(), lane = lane_id();
   const int Hq = Hkv * G;
   const int nqb = (T + QT - 1) / QT;
-  const int n_items = nqb * Hkv;
+  // all items, or (recomputing items whose speculative floor failed) the
+  // listed ones, without speculation
+  const int n_items = item_list == nullptr
+                          ? nqb * Hkv
+                          : int(min(*const_cast<volatile uint32_t*>(fail_count), uint32_t(nqb * Hkv)));
+  const bool speculate = spec_factor > 0.f && item_list == nullptr;
   // score bins: bucket (bits >> BSHIFT) relative to lo; the top bin holds the
   // largest possible score G, bin 0 everything NB-1 bins and more below it
   const uint32_t top = __float_as_uint(float(G)) >> BSHIFT;
@@ -365,6 +376,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   auto item = [&](int it, int& q0, int& g, int& n_tiles, bool& score) {
     // KV-head-major, heaviest query blocks first within a head, so that the
     // CTAs running at one time stream the same head's K through L2
+    if (item_list != nullptr) it = item_list[it];
     const int qb = nqb - 1 - it % nqb;
     g = it / nqb;
     q0 = qb * QT;
@@ -385,6 +397,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&br->s_empty[b], SCORERS);
     }
     mbar_init(&br->drain, 1);
+    ms->spec_bits = 0;
+    ms->spec_g = -1;
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -480,8 +494,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int qrow = q0 + tid / G;
         ms->nlse2[tid] = qrow < T ? -lse[size_t(qrow) * Hq + g * G + tid % G] * kLog2e : -INFINITY;
       }
+      // speculative floor: a fraction of the smallest k-th best score of the
+      // CTA's previous item of this head (earlier-processed items lie at
+      // later positions, whose k-th best scores are not larger)
+      const uint32_t spec = speculate && ms->spec_g == g ? ms->spec_bits : 0u;
       for (int i = tid; i < QT; i += SCORERS) {
-        ms->floor_bits[i] = 0;
+        ms->floor_bits[i] = spec;
         ms->compacted[i] = 0;
       }
       for (int i = tid; i < QT * NB; i += SCORERS) (&ms->hist[0][0])[i] = 0;
@@ -495,8 +513,15 @@ __global__ void __launch_bounds__(THREADS, 1)
       const float* nlw = &ms->nlse2[half * 32];
       uint32_t n[QH], fl[QH];  // appended entries and floors of this warp's queries
 #pragma unroll
-      for (int qq = 0; qq < QH; ++qq) n[qq] = fl[qq] = 0;
+      for (int qq = 0; qq < QH; ++qq) {
+        n[qq] = 0;
+        fl[qq] = spec;
+      }
       scorer_sync();
+      if (tid == 0) {
+        ms->spec_min = 0xFFFFFFFFu;
+        ms->item_fail = 0;
+      }
       for (int t = 0; t < n_tiles; ++t, ++st) {
         const int b = st % NSB;
         ok = ok && mbar_wait(&br->s_full[b], (st / NSB) & 1);
@@ -588,10 +613,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         } else {
           uint2* sb[4];
           uint32_t nbv[4];
+          uint32_t total = 0;
           for (int v = 0; v < 4; ++v) {
             sb[v] = ws + ((size_t(blockIdx.x) * 4 + v) * QT + q) * capw;
             nbv[v] = ms->cnt[v][q];
+            total += nbv[v];
           }
+          // every candidate at or above the floor is buffered, so fewer than k
+          // entries means the speculative floor was above the k-th best: the
+          // item is recomputed without speculation
+          if (total < uint32_t(k) && lane == 0) ms->item_fail = 1;
           // the bin of the k-th best: from the append histogram when every
           // appended entry is still buffered, else from one counting pass
           const uint32_t* hq = ms->hist[q];
@@ -736,6 +767,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
           kv = __uint_as_float(mn);
+          if (lane == 0 && total >= uint32_t(k)) atomicMin(&ms->spec_min, mn);
           __syncwarp();
         }
         for (int t2 = lane; t2 < w; t2 += 32) {
@@ -743,6 +775,17 @@ __global__ void __launch_bounds__(THREADS, 1)
           out[k + t2] = p >= 0 ? p : -1;
         }
         if (kth != nullptr && lane == 0) kth[size_t(qrow) * Hkv + g] = kv;
+      }
+      scorer_sync();
+      if (tid == 0 && score && speculate) {
+        // only speculative items can fail; each is listed at most once
+        if (ms->item_fail) {
+          fail_list[atomicAdd(fail_count, 1u)] = it;
+          ms->spec_bits = 0;
+        } else if (ms->spec_min != 0xFFFFFFFFu) {
+          ms->spec_bits = __float_as_uint(__uint_as_float(ms->spec_min) * spec_factor);
+          ms->spec_g = g;
+        }
       }
       scorer_sync();
     }
@@ -771,6 +814,10 @@ int stages_for() {
   return min(MAX_STAGES, (227 * 1024 - fixed) / TILE_BYTES);
 }
 
+// Fraction of the previous item's smallest k-th best score that starts an
+// item's floor (<= 0: no speculation).  Set through a testing hook.
+float g_spec_factor = 0.9f;
+
 template <int G>
 cudaError_t launch_g(const SelectArgs& a, cudaStream_t stream) {
   constexpr int QT = TILE / G;
@@ -788,11 +835,23 @@ cudaError_t launch_g(const SelectArgs& a, cudaStream_t stream) {
   const int grid = min(sm_count(), n_items);
   uint2* ws = reinterpret_cast<uint2*>(a.ws);
   uint32_t* wsort = reinterpret_cast<uint32_t*>(ws + size_t(sm_count()) * 4 * QT * buffer_cap(a.k));
-  select_kernel<G><<<grid, THREADS, smem, stream>>>(tmQ, tmK, a.lse, a.idx, a.kth, ws, wsort,
-                                                    int(a.T), a.Hkv, a.k, a.w, buffer_cap(a.k),
-                                                    kst, a.scale * kLog2e, int(a.q_begin));
-  count_launch();
-  return cudaGetLastError();
+  // items whose speculative floor failed: a count, then their indices
+  uint32_t* fail_count = wsort + size_t(sm_count()) * SCORER_WARPS * kSortWords;
+  int32_t* fail_list = reinterpret_cast<int32_t*>(fail_count + 4);
+  e = cudaMemsetAsync(fail_count, 0, sizeof(uint32_t), stream);
+  if (e != cudaSuccess) return e;
+  // every item, speculating; then the failed ones again without speculation
+  // (a CTA of the second launch exits at once when the list is empty)
+  for (int pass = 0; pass < 2; ++pass) {
+    select_kernel<G><<<grid, THREADS, smem, stream>>>(
+        tmQ, tmK, a.lse, a.idx, a.kth, ws, wsort, int(a.T), a.Hkv, a.k, a.w, buffer_cap(a.k), kst,
+        a.scale * kLog2e, int(a.q_begin), pass == 0 ? g_spec_factor : 0.f,
+        pass == 0 ? nullptr : fail_list, fail_count, fail_list);
+    count_launch();
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 // ---------------------------------------------------------------------------
@@ -850,7 +909,8 @@ cudaError_t launch_noalloc_g(const SelectArgs& a, void* scratch, cudaStream_t st
   uint32_t* wsort = reinterpret_cast<uint32_t*>(ws + size_t(grid) * 4 * QT * buffer_cap(a.k));
   select_kernel<G><<<grid, THREADS, smem, stream>>>(tmQ, tmK, a.lse, a.idx, a.kth, ws, wsort,
                                                     int(a.T), a.Hkv, a.k, a.w, buffer_cap(a.k),
-                                                    kst, a.scale * kLog2e, int(a.q_begin));
+                                                    kst, a.scale * kLog2e, int(a.q_begin), 0.f,
+                                                    nullptr, nullptr, nullptr);
   count_launch();
   return cudaGetLastError();
 }
@@ -858,14 +918,17 @@ cudaError_t launch_noalloc_g(const SelectArgs& a, void* scratch, cudaStream_t st
 }  // namespace
 
 size_t select_workspace_bytes(int64_t T, int Hq, int Hkv, int k, int w) {
-  (void)T;
   (void)w;
   const int QT = TILE / (Hq / Hkv);
+  const size_t n_items = size_t((T + QT - 1) / QT) * Hkv;
   return size_t(sm_count()) * (size_t(4) * QT * buffer_cap(k) * sizeof(uint2) +
-                               size_t(SCORER_WARPS) * kSortWords * sizeof(uint32_t));
+                               size_t(SCORER_WARPS) * kSortWords * sizeof(uint32_t)) +
+         16 + n_items * sizeof(int32_t);
 }
 
 size_t select_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+void select_set_speculation(float factor) { g_spec_factor = factor; }
 
 cudaError_t launch_select_noalloc(const SelectArgs& a, cudaStream_t stream) {
   void* scratch = nullptr;

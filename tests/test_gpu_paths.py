@@ -250,3 +250,36 @@ def test_decode_separate_k_and_v_scales(hs2, orc):
         rel = np.linalg.norm(got["o"][b] - o_sw[0]) / np.linalg.norm(o_sw[0])
         assert rel > 0.1, "swapped scales give the same output"
     assert n_diff <= 1
+
+
+@pytest.mark.parametrize("T,Hq,Hkv,k,w", [(6000, 8, 2, 1024, 128), (9000, 32, 4, 256, 64),
+                                          (5000, 4, 1, 64, 16)])
+def test_select_speculative_floor_never_changes_results(hs2, orc, T, Hq, Hkv, k, w):
+    """The selection starts each work item's floor at a fraction of the
+    smallest k-th best score its CTA found in its previous item of the same KV
+    head.  A floor above an item's true k-th best is detected and that item is
+    recomputed without it, so the lists and k-th scores must be bit for bit
+    the same with the default fraction, with speculation off, and with a
+    fraction so large that every speculative item fails and is recomputed;
+    and they must match the oracle.  T is large enough that CTAs take several
+    items of one head."""
+    import torch
+    Q, K, V = rand_bf16((T, Hq, 128)), rand_bf16((T, Hkv, 128)), rand_bf16((T, Hkv, 128))
+    kv, sc = orc.KV(K, V), 1 / math.sqrt(128)
+    rows = np.arange(T)
+    _, lse = orc.full_attn(kv, Q, rows, sc)
+    shape = hs2.Shape.make(T, Hq, Hkv, k_global=k, window=w)
+    got = {}
+    try:
+        for name, f in (("default", 0.9), ("off", 0.0), ("forced", 1e30)):
+            hs2.hs2_debug_set_select_speculation(f)
+            got[name] = _select_on_device(hs2, Q, K, lse, shape, T, Hkv, k, w)
+    finally:
+        hs2.hs2_debug_set_select_speculation(0.9)
+    for name in ("off", "forced"):
+        assert np.array_equal(got[name][0], got["default"][0]), f"{name}: index lists differ"
+        assert np.array_equal(got[name][1], got["default"][1]), f"{name}: k-th scores differ"
+    idx_o, kth_o = orc.select(kv, Q, rows, sc, lse, k, w)
+    n_diff = check_index_lists(got["default"][0], idx_o, kth_o, rows, k, w,
+                               lambda r, g, js: orc.scores(kv, Q[r], g, sc, lse[r], js))
+    assert n_diff <= 0.01 * T * Hkv
