@@ -338,6 +338,36 @@ def bench_decode(hs2, dev, steps, warmup):
 # ---------------------------------------------------------------------------
 # one launch of each hot kernel at a moderate size (for profiler captures)
 # ---------------------------------------------------------------------------
+def select_once(dev, T, Hq, Hkv):
+    """Full attention and one selection launch on the 128K workload's recipe
+    (bridge from H, needles planted, queries mixed with the needle direction)
+    with fewer heads, so that the same key-stream lengths fit a profiler's
+    multi-pass capture (about 1.3 GB on the device at T = 131072, 8/1 heads)."""
+    import long_context_bridge_b200 as hs2
+    base = synth.CONFIGS["C3"]
+    cfg = synth.BlockConfig(f"select T={T} {Hq}q/{Hkv}kv", base.number, T, Hq, Hkv,
+                            d_model=base.d_model, n_needles=base.n_needles, q_mix=True)
+    H, Wk, Wv = synth.bridge_inputs_torch(cfg, device=dev)
+    sh = hs2.Shape.make(T, Hq, Hkv)
+    K = torch.empty(T, Hkv, 128, dtype=torch.bfloat16, device=dev)
+    V = torch.empty_like(K)
+    hs2.hs2_bridge_kv(H, Wk, Wv, K, V, sh)
+    del H
+    nr, nh, nv = synth.needle_scatter_torch(cfg, device=dev)
+    K[nr, nh] = nv
+    Q = synth.q_rows_torch(cfg, synth.TID_Q, device=dev)
+    O = torch.empty_like(Q)
+    lse = torch.empty(T, Hq, dtype=torch.float32, device=dev)
+    hs2.hs2_full_attn_lse(Q, K, V, O, lse, sh)
+    del O
+    ws = torch.empty(hs2.workspace_size(hs2.OP_SELECT, sh), dtype=torch.uint8, device=dev)
+    idx = torch.empty(T, Hkv, 1152, dtype=torch.int32, device=dev)
+    hs2.hs2_select_topk(Q, K, lse, idx, None, sh, ws)
+    torch.cuda.synchronize()
+    assert hs2.hs2_get_device_status() == hs2.OK
+    print(f"select-once: {cfg.name}", flush=True)
+
+
 def kernels_once(dev):
     import long_context_bridge_b200 as hs2
     T, Hq, Hkv, dm = 32768, 32, 4, 2048
@@ -391,10 +421,18 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--kernels-once", action="store_true",
                     help="run each hot kernel once at a moderate size (profiler driver) and exit")
+    ap.add_argument("--select-once", default=None, metavar="T,HQ,HKV",
+                    help="run full attention and one selection on the 128K recipe with these "
+                         "sizes (profiler driver) and exit")
     args = ap.parse_args()
-    if args.kernels_once:
+    if args.kernels_once or args.select_once:
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
-        kernels_once(torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0"))))
+        dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+        if args.select_once:
+            T_, hq_, hkv_ = (int(x) for x in args.select_once.split(","))
+            select_once(dev, T_, hq_, hkv_)
+        else:
+            kernels_once(dev)
         return
 
     rank = int(os.environ.get("RANK", "0"))
