@@ -44,8 +44,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                        __nv_bfloat16* __restrict__ V, int T, int dm, int Nkv) {
   using C = BridgeCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* smem = smem_align1024(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* accbar = empty + STAGES;
@@ -179,8 +178,7 @@ __global__ void __launch_bounds__(THREADS, 2)
                       uint8_t* __restrict__ Vc, float* __restrict__ scale, int T, int dm,
                       int Hkv) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* smem = smem_align1024(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + F_STAGES * F_STAGE_BYTES);
   uint64_t* empty = full + F_STAGES;
   uint64_t* accbar = empty + F_STAGES;

@@ -56,6 +56,14 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The dynamic shared memory from its first 1024-byte boundary on (the
+// alignment of 128-byte-swizzled tiles).  Written as an offset from the
+// array itself, so that the compiler still sees a shared-memory pointer and
+// issues shared loads, stores and atomics through it.
+__device__ __forceinline__ uint8_t* smem_align1024(uint8_t* raw) {
+  return raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);
+}
+
 // ---------------------------------------------------------------------------
 // mbarrier
 // ---------------------------------------------------------------------------

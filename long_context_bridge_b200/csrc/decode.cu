@@ -124,8 +124,7 @@ __global__ void __launch_bounds__((DP_WARPS + 1) * 32, 3)
   __shared__ uint64_t full[DSTAGES], empty[DSTAGES];
   __shared__ float sScale[DSTAGES][2][DSTAGE_KEYS];  // K and V scales of a stage's keys
   extern __shared__ uint8_t dsmem_raw[];
-  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* ring = smem_align1024(dsmem_raw);
 
   // the KV heads of a chunk are neighbours in the grid, so the 128-byte head
   // slices of the same cache rows are read at about the same time

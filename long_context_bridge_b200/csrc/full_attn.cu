@@ -71,8 +71,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                      float* __restrict__ lse, int T, int Hkv, float scale_log2, int q_begin) {
   constexpr int QT = TILE / G;  // queries per Q tile
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* smem = smem_align1024(smem_raw);
   Bars* bars = reinterpret_cast<Bars*>(smem + OFF_BAR);
   const int warp = warp_id(), lane = lane_id();
   const int nqb = (T + QT - 1) / QT;

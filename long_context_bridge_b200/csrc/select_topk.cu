@@ -72,7 +72,7 @@ constexpr int NSB = 4;          // S^T buffers in TMEM (128 columns each)
 constexpr uint32_t IDESC = idesc_bf16(128, 128, 0, 0);
 constexpr float kLog2e = 1.4426950408889634f;
 
-constexpr int kRefresh = 4;         // tiles between floor refreshes (a power of two)
+constexpr int kRefresh = 8;         // tiles between floor refreshes (a power of two)
 constexpr int kBoundaryCap = 1024;  // boundary-bin entries per final select in scratch
 constexpr int kSortWords = 2048 + 2 * kBoundaryCap;  // per-warp sort scratch (32-bit words)
 
@@ -354,8 +354,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   using Cfg = SelCfg<G>;
   constexpr int QT = Cfg::QT, QH = Cfg::QH, NB = Cfg::NB, BSHIFT = Cfg::BSHIFT;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* smem = smem_align1024(smem_raw);
   Misc<G>* ms = reinterpret_cast<Misc<G>*>(smem + OFF_K + kst * TILE_BYTES);
   Bars* br = &ms->bars;
   const int warp = warp_id(), lane = lane_id();
@@ -558,25 +557,48 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         // candidates at or above the floor go to this warp's sub-buffer of
         // the query, in position order; each append is counted by score bin
+        // (groups of up to four queries: their tests and ballots first, one
+        // warp-uniform test for a sub-buffer about to overflow, then the
+        // appends as predicated stores)
         const bool chk = !all_exist || t * TILE + TILE - 1 > last_free;
         const int dpos = j + w - q_begin - q0 - qb0;  // candidate of query qb0 + qq iff dpos <= qq
+        constexpr int QB = QH < 4 ? QH : 4;
 #pragma unroll
-        for (int qq = 0; qq < QH; ++qq) {
-          const uint32_t bits = __float_as_uint(sc[qq]);
-          bool p = bits >= fl[qq];
-          if (chk) p = p && dpos <= qq && qq < qvalid;
-          const uint32_t bal = __ballot_sync(0xffffffffu, p);
-          if (bal == 0) continue;
-          if (n[qq] + 32 > uint32_t(capw)) {
-            n[qq] = make_room<NB, BSHIFT>(qbuf + size_t(qq) * capw, n[qq], ms->floor_bits[qb0 + qq],
-                                          k, capw, lo, ms->dig[sw], lane);
-            if (lane == 0) ms->compacted[qb0 + qq] = 1;
+        for (int q4 = 0; q4 < QH; q4 += QB) {
+          bool p[QB];
+          uint32_t bal[QB];
+          bool full = false;
+#pragma unroll
+          for (int u = 0; u < QB; ++u) {
+            const int qq = q4 + u;
+            p[u] = __float_as_uint(sc[qq]) >= fl[qq];
+            if (chk) p[u] = p[u] && dpos <= qq && qq < qvalid;
+            bal[u] = __ballot_sync(0xffffffffu, p[u]);
+            full = full || (bal[u] != 0 && n[qq] + 32 > uint32_t(capw));
           }
-          if (p) {
-            qbuf[size_t(qq) * capw + n[qq] + __popc(bal & lt_mask)] = make_uint2(bits, uint32_t(j));
-            atomicAdd(&ms->hist[qb0 + qq][bin_of<NB, BSHIFT>(bits, lo)], 1u);
+          if (full) {
+#pragma unroll
+            for (int u = 0; u < QB; ++u) {
+              const int qq = q4 + u;
+              if (bal[u] != 0 && n[qq] + 32 > uint32_t(capw)) {
+                n[qq] = make_room<NB, BSHIFT>(qbuf + size_t(qq) * capw, n[qq],
+                                              ms->floor_bits[qb0 + qq], k, capw, lo, ms->dig[sw],
+                                              lane);
+                if (lane == 0) ms->compacted[qb0 + qq] = 1;
+              }
+            }
           }
-          n[qq] += __popc(bal);
+#pragma unroll
+          for (int u = 0; u < QB; ++u) {
+            const int qq = q4 + u;
+            if (p[u]) {
+              const uint32_t bits = __float_as_uint(sc[qq]);
+              qbuf[size_t(qq) * capw + n[qq] + __popc(bal[u] & lt_mask)] =
+                  make_uint2(bits, uint32_t(j));
+              atomicAdd(&ms->hist[qb0 + qq][bin_of<NB, BSHIFT>(bits, lo)], 1u);
+            }
+            n[qq] += __popc(bal[u]);
+          }
         }
         // raise the floors this warp owns to the highest bin with at least k
         // appended entries at or above it (any snapshot of the counts gives a
