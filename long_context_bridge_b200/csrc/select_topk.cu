@@ -14,36 +14,38 @@
 //   warps 2-17 scorers, four per TMEM lane quarter: thread = key (TMEM lane);
 //              scorer warp 4s + r takes the s-th quarter of the item's queries
 //              (TMEM columns 32s .. 32s + 31) for keys 32r .. 32r + 31.
-// Pruning before the exact scores: a candidate can only enter the top k if
-// its score reaches the query's floor F (below).  With y_h = log2 of head
-// h's probability over F, score / F = sum_h 2^y_h.  A pre-filter evaluates
-// that sum in half precision, two heads per instruction (FFMA2 for the y
-// pair, one conversion to f16x2, ex2.approx.f16x2, f16x2 adds); its error
-// bound is far inside the 3% margin it is compared with, so it drops no
-// candidate that reaches the floor.  The survivors' G logits are staged in
-// shared memory and their exact scores, sum_h exp2(s*scale*log2e - lse2) in
-// fp32, are computed 32 at a time by full warps.
+// Scores: every scorer thread computes, for its key and each of its warp's
+// queries, score = sum over the G heads of exp2(s * scale * log2 e - lse2_h)
+// in fp32 (pairs of heads per FFMA2, one ex2.approx per head, pairwise adds).
+// Candidates only enter the top k if their score reaches the query's floor F.
 // Streaming exact top-k without CTA barriers in the tile loop:
-//   * every scorer warp appends the survivors of its 32 keys whose exact
-//     score reaches the floor to its own per-query sub-buffer; the four warps
-//     of a query's quarter hold disjoint key sets;
+//   * every scorer warp appends the candidates of its 32 keys whose score
+//     reaches the floor to its own per-query sub-buffer; the four warps of a
+//     query's quarter hold disjoint key sets;
 //   * every append is also counted in a per-query histogram of score bins
 //     (eighths of a binade below the largest possible score G) in shared
 //     memory; whatever snapshot of it a warp reads, the highest bin with at
 //     least k appended entries at or above it bounds the k-th best score from
 //     below, so that bin's lower edge is a valid floor.  One warp owns each
-//     query's floor, which only rises;
+//     query's floor, which only rises; it is refreshed every few tiles;
+//   * speculative floor: an item starts from 0.9 of the smallest k-th best
+//     score of the CTA's previous item of the same KV head (items run from
+//     the latest positions backwards, and earlier queries' k-th best scores
+//     are mostly larger).  Under it the histograms are not kept.  A query
+//     that ends with fewer than k buffered entries shows the guess was too
+//     high; the item is then listed and recomputed without speculation by a
+//     second launch, so the result never depends on the guess;
 //   * a sub-buffer about to overflow drops its entries below the floor, or,
 //     if that is not enough, keeps its own exact k best;
 //   * at the end of the item one warp per query selects the k best of the
 //     union of the four sub-buffers on the 64-bit key
 //     (score bits << 32 | ~position), larger score first and equal scores to
 //     the smaller position: the append histogram gives the k-th best's bin
-//     (a counting pass rebuilds it if entries were dropped), one pass takes
-//     every entry above that bin and lists the bin's own entries, an exact
-//     radix select over that short list settles the rest (over every entry
-//     if the list is too long), and the chosen positions are sorted
-//     ascending by a bitonic sort held lane-major in registers.
+//     (a counting pass rebuilds it if entries were dropped or not counted),
+//     one pass takes every entry above that bin and lists the bin's own
+//     entries, an exact radix select over that short list settles the rest
+//     (over every entry if the list is too long), and the chosen positions
+//     are sorted ascending by a bitonic sort held lane-major in registers.
 // Items whose every query has at most k candidates skip the scoring: all
 // candidates are selected.
 #include <cstddef>
@@ -497,9 +499,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       // CTA's previous item of this head (earlier-processed items lie at
       // later positions, whose k-th best scores are not larger)
       const uint32_t spec = speculate && ms->spec_g == g ? ms->spec_bits : 0u;
+      // with a speculative floor the histograms are not kept (the floor is
+      // close to the final k-th best already): the final select counts
       for (int i = tid; i < QT; i += SCORERS) {
         ms->floor_bits[i] = spec;
-        ms->compacted[i] = 0;
+        ms->compacted[i] = spec != 0u;
       }
       for (int i = tid; i < QT * NB; i += SCORERS) (&ms->hist[0][0])[i] = 0;
       const int qb0 = half * QH;        // this warp's queries: qb0 .. qb0 + QH - 1
@@ -595,7 +599,7 @@ __global__ void __launch_bounds__(THREADS, 1)
               const uint32_t bits = __float_as_uint(sc[qq]);
               qbuf[size_t(qq) * capw + n[qq] + __popc(bal[u] & lt_mask)] =
                   make_uint2(bits, uint32_t(j));
-              atomicAdd(&ms->hist[qb0 + qq][bin_of<NB, BSHIFT>(bits, lo)], 1u);
+              if (spec == 0u) atomicAdd(&ms->hist[qb0 + qq][bin_of<NB, BSHIFT>(bits, lo)], 1u);
             }
             n[qq] += __popc(bal[u]);
           }
@@ -603,7 +607,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         // raise the floors this warp owns to the highest bin with at least k
         // appended entries at or above it (any snapshot of the counts gives a
         // valid floor), then take up every floor of its queries
-        if ((t & (kRefresh - 1)) == kRefresh - 1) {
+        if (spec == 0u && (t & (kRefresh - 1)) == kRefresh - 1) {
           for (int q = half * QH + sub; q < (half + 1) * QH; q += 4) {
             uint32_t above, inbin;
             const int fb = hist_cross<NB>(ms->hist[q], uint32_t(k), lane, above, inbin);
