@@ -84,7 +84,8 @@ enum {
   HS2_OP_SELECT = 2,
   HS2_OP_SPARSE = 3,
   HS2_OP_BLOCK_PREFILL = 4,
-  HS2_OP_BLOCK_DECODE = 5
+  HS2_OP_BLOCK_DECODE = 5,
+  HS2_OP_SPARSE_PLAN = 6  /* bytes of a plan for hs2_sparse_plan (size_t(-1): no plan path) */
 };
 
 /*
@@ -210,6 +211,39 @@ hs2_status hs2_sparse_attn_layers(int32_t n_layers, const hs2_bf16* const* Q,
                                   const hs2_bf16* K, const hs2_bf16* V, const int32_t* idx,
                                   hs2_bf16* const* O, float* const* lse,
                                   const hs2_shape* shape, void* stream);
+
+/*
+ * Sparse attention in two calls, over the union of neighbouring queries'
+ * lists (same operation as hs2_sparse_attn; no counterpart on the pages).
+ * The lists of P = 128 / G consecutive query rows of one KV head overlap
+ * heavily (their recent windows almost entirely), so each distinct listed row
+ * can be gathered once for all of them.
+ *
+ * hs2_sparse_plan: from idx [T, n_kv_heads, k_global + window] (as written by
+ * hs2_select_topk, any order within a list), per (P query rows, KV head) the
+ * ascending union of their lists and, per union row, which of the P queries
+ * list it.  plan: a DEVICE buffer of hs2_workspace_size(HS2_OP_SPARSE_PLAN,
+ * shape) bytes, 16-byte aligned, owned by the caller; it depends only on idx
+ * and the shape and serves every sparse layer that shares idx.  An entry
+ * outside [-1, T), or one listed twice in a row's list, is used at most once
+ * and reported as HS2_ERR_BAD_INDEX by the next hs2_get_device_status().
+ *
+ * hs2_sparse_attn_planned: what hs2_sparse_attn(Q, K, V, idx, O, lse) writes
+ * for the idx the plan was built from, up to fp32 rounding order (the union
+ * rows are attended with a tcgen05 tile per 128 of them; rows a query does
+ * not list get probability exactly 0).  plan must come from hs2_sparse_plan
+ * with the same shape on the same stream (or a synchronised one).
+ *
+ * Both: HS2_ERR_UNSUPPORTED unless G = n_q_heads / n_kv_heads is 8 or 16,
+ * P * (k_global + window) <= 18432 and T * n_kv_heads < 2^31;
+ * HS2_ERR_WORKSPACE if plan_bytes is short.  hs2_block_prefill and
+ * hs2_block_prefill_rows take this path by themselves where it applies.
+ */
+hs2_status hs2_sparse_plan(const int32_t* idx, const hs2_shape* shape, void* plan,
+                           size_t plan_bytes, void* stream);
+hs2_status hs2_sparse_attn_planned(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V,
+                                   const void* plan, hs2_bf16* O, float* lse,
+                                   const hs2_shape* shape, void* stream);
 
 /*
  * The whole block at prefill: bridge (if H != NULL), full attention, selection

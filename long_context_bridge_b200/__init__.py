@@ -17,7 +17,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libhs2.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_BAD_INDEX = range(7)
-OP_BRIDGE, OP_FULL_ATTN, OP_SELECT, OP_SPARSE, OP_BLOCK_PREFILL, OP_BLOCK_DECODE = range(6)
+OP_BRIDGE, OP_FULL_ATTN, OP_SELECT, OP_SPARSE, OP_BLOCK_PREFILL, OP_BLOCK_DECODE, OP_SPARSE_PLAN = range(7)
 
 
 class HS2Error(RuntimeError):
@@ -55,6 +55,8 @@ def _load(path: str = LIB_PATH):
         "hs2_select_topk_noalloc": [P, P, P, P, P, SP, P],
         "hs2_sparse_attn": [P, P, P, P, P, P, SP, P],
         "hs2_sparse_attn_layers": [I32, PP, P, P, P, PP, PP, SP, P],
+        "hs2_sparse_plan": [P, SP, P, SZ, P],
+        "hs2_sparse_attn_planned": [P, P, P, P, P, P, SP, P],
         "hs2_block_prefill": [P, I32, P, P, P, P, P, P, P, P, I32, PP, PP, SP, P, SZ, P],
         "hs2_block_decode": [I32, C.POINTER(C.c_int64), P, P, P, P, P, P, P, P, I32, PP, PP, SP,
                              P, SZ, P],
@@ -88,7 +90,7 @@ def _load(path: str = LIB_PATH):
 _lib = _load()
 
 EXPORTED = ["hs2_bridge_kv", "hs2_bridge_kv_fp8", "hs2_full_attn_lse", "hs2_select_topk", "hs2_select_topk_noalloc",
-            "hs2_sparse_attn", "hs2_sparse_attn_layers",
+            "hs2_sparse_attn", "hs2_sparse_attn_layers", "hs2_sparse_plan", "hs2_sparse_attn_planned",
             "hs2_block_prefill", "hs2_block_decode", "hs2_workspace_size",
             "hs2_get_device_status", "hs2_status_string", "hs2_kernel_launches",
             "hs2_debug_set_wait_budget", "hs2_debug_read_probe", "hs2_block_prefill_rows",
@@ -176,6 +178,19 @@ def hs2_sparse_attn(Q, K, V, idx, O, lse, shape: Shape, stream=None):
                                 _ptr(idx, I32T, "idx"), _ptr(O, BF16, "O"),
                                 _ptr(lse, F32, "lse", True), C.byref(shape), _stream(stream)),
            "hs2_sparse_attn")
+
+
+def hs2_sparse_plan(idx, shape: Shape, plan, stream=None):
+    nbytes = plan.numel() * plan.element_size()
+    _check(_lib.hs2_sparse_plan(_ptr(idx, I32T, "idx"), C.byref(shape), _ptr(plan, U8, "plan"),
+                                nbytes, _stream(stream)), "hs2_sparse_plan")
+
+
+def hs2_sparse_attn_planned(Q, K, V, plan, O, lse, shape: Shape, stream=None):
+    _check(_lib.hs2_sparse_attn_planned(_ptr(Q, BF16, "Q"), _ptr(K, BF16, "K"), _ptr(V, BF16, "V"),
+                                        _ptr(plan, U8, "plan"), _ptr(O, BF16, "O"),
+                                        _ptr(lse, F32, "lse", True), C.byref(shape),
+                                        _stream(stream)), "hs2_sparse_attn_planned")
 
 
 def _ptr_array(ts, dtype, what):

@@ -6,6 +6,7 @@
 #include <algorithm>
 #include <atomic>
 #include <mutex>
+#include <map>
 #include <set>
 #include <utility>
 
@@ -64,15 +65,18 @@ bool make_tmap_3d(CUtensorMap* map, const void* base, uint64_t dim_x, uint64_t d
 }
 
 cudaError_t ensure_smem_attr(const void* func, int bytes) {
+  // the largest size set so far per (kernel, device): raised when a launch
+  // needs more (a kernel's dynamic size may depend on its arguments)
   static std::mutex mu;
-  static std::set<std::pair<const void*, int>> done;
+  static std::map<std::pair<const void*, int>, int> done;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lock(mu);
-  if (done.count({func, dev})) return cudaSuccess;
+  const auto it = done.find({func, dev});
+  if (it != done.end() && it->second >= bytes) return cudaSuccess;
   e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess) done.insert({func, dev});
+  if (e == cudaSuccess) done[{func, dev}] = bytes;
   return e;
 }
 
@@ -119,6 +123,63 @@ hs2_status cuda_status(cudaError_t e) {
     if (!(cond)) return HS2_ERR_INVALID_ARG;      \
   } while (0)
 
+// The block calls build and use the union plan slab by slab, so that their
+// workspace does not grow with T beyond the selection's.
+constexpr int64_t kPlanSlabRows = 32768;
+
+bool union_path(const hs2_shape* s, int64_t kv_rows) {
+  return sparse_union_supported(s->T, s->n_q_heads, s->n_kv_heads, s->k_global + s->window,
+                                kv_rows);
+}
+
+size_t block_prefill_bytes(const hs2_shape* s) {
+  size_t need = select_workspace_bytes(s->T, s->n_q_heads, s->n_kv_heads, s->k_global, s->window);
+  if (union_path(s, s->T)) {
+    const UnionPlan pl = union_plan_layout(s->T, s->n_q_heads, s->n_kv_heads,
+                                           s->k_global + s->window, 0,
+                                           std::min<int64_t>(s->T, kPlanSlabRows), nullptr);
+    need = std::max(need, pl.bytes);
+  }
+  return need;
+}
+
+// The sparse layers of a block: over the union plan, slab by slab, where the
+// shape allows it; else one list per (row, KV head).
+hs2_status block_sparse_layers(const hs2_shape* s, int64_t kv_rows, const hs2_bf16* K,
+                               const hs2_bf16* V, const int32_t* idx, int32_t n_sparse,
+                               const hs2_bf16* const* Q_sparse, hs2_bf16* const* O_sparse,
+                               void* ws, cudaStream_t st) {
+  SparseArgs a{};
+  a.K = K;
+  a.V = V;
+  a.idx = idx;
+  a.T = s->T;
+  a.Hq = s->n_q_heads;
+  a.Hkv = s->n_kv_heads;
+  a.scale = s->scale;
+  a.kw = s->k_global + s->window;
+  a.kv_rows = kv_rows;
+  if (!union_path(s, kv_rows)) {
+    for (int l = 0; l < n_sparse; ++l) {
+      a.Q = Q_sparse[l];
+      a.O = O_sparse[l];
+      HS2_TRY(cuda_status(launch_sparse(a, st)));
+    }
+    return HS2_OK;
+  }
+  for (int64_t r0 = 0; r0 < s->T; r0 += kPlanSlabRows) {
+    const int64_t rows = std::min(kPlanSlabRows, s->T - r0);
+    const UnionPlan pl = union_plan_layout(s->T, a.Hq, a.Hkv, a.kw, r0, rows, ws);
+    HS2_TRY(cuda_status(launch_sparse_plan(a, pl, st)));
+    for (int l = 0; l < n_sparse; ++l) {
+      a.Q = Q_sparse[l];
+      a.O = O_sparse[l];
+      HS2_TRY(cuda_status(launch_sparse_union(a, pl, st)));
+    }
+  }
+  return HS2_OK;
+}
+
 
 }  // namespace
 
@@ -147,6 +208,7 @@ hs2_status hs2_get_device_status(void* stream) {
   v |= status_full_attn(true);
   v |= status_select(true);
   v |= status_sparse(true);
+  v |= status_sparse_union(true);
   v |= status_decode(true);
   if (v == ~0u) return HS2_ERR_CUDA;
   if (v & DEV_TIMEOUT) return HS2_ERR_TIMEOUT;
@@ -171,21 +233,28 @@ hs2_status hs2_debug_set_wait_budget(int64_t cycles) {
   cudaError_t e = budget_bridge(c);
   if (e == cudaSuccess) e = budget_full_attn(c);
   if (e == cudaSuccess) e = budget_select(c);
+  if (e == cudaSuccess) e = budget_sparse_union(c);
   if (e == cudaSuccess) e = budget_decode(c);
   return cuda_status(e);
 }
 
 size_t hs2_workspace_size(int32_t op, const hs2_shape* s, int32_t batch, int32_t d_model) {
   (void)d_model;
-  const bool sel = op == HS2_OP_SELECT || op == HS2_OP_BLOCK_PREFILL || op == HS2_OP_BLOCK_DECODE;
+  const bool sel = op == HS2_OP_SELECT || op == HS2_OP_BLOCK_PREFILL ||
+                   op == HS2_OP_BLOCK_DECODE || op == HS2_OP_SPARSE_PLAN;
   if (check_shape(s, sel) != HS2_OK) return size_t(-1);
   switch (op) {
     case HS2_OP_BRIDGE:
     case HS2_OP_FULL_ATTN:
     case HS2_OP_SPARSE: return 0;
     case HS2_OP_SELECT:
-    case HS2_OP_BLOCK_PREFILL:
       return select_workspace_bytes(s->T, s->n_q_heads, s->n_kv_heads, s->k_global, s->window);
+    case HS2_OP_BLOCK_PREFILL: return block_prefill_bytes(s);
+    case HS2_OP_SPARSE_PLAN:
+      if (!union_path(s, s->T)) return size_t(-1);
+      return union_plan_layout(s->T, s->n_q_heads, s->n_kv_heads, s->k_global + s->window, 0,
+                               s->T, nullptr)
+          .bytes;
     case HS2_OP_BLOCK_DECODE:
       if (batch <= 0 || batch > kDecodeMaxBatch || int64_t(batch) * s->T > INT32_MAX)
         return size_t(-1);
@@ -319,6 +388,47 @@ hs2_status hs2_sparse_attn_layers(int32_t n_layers, const hs2_bf16* const* Q,
   return HS2_OK;
 }
 
+hs2_status hs2_sparse_plan(const int32_t* idx, const hs2_shape* s, void* plan,
+                           size_t plan_bytes, void* stream) {
+  HS2_TRY(check_shape(s, true));
+  HS2_NEED(idx && aligned16(idx));
+  if (!union_path(s, s->T)) return HS2_ERR_UNSUPPORTED;
+  SparseArgs a{};
+  a.idx = idx;
+  a.T = s->T;
+  a.Hq = s->n_q_heads;
+  a.Hkv = s->n_kv_heads;
+  a.kw = s->k_global + s->window;
+  a.kv_rows = s->T;
+  const UnionPlan pl = union_plan_layout(s->T, a.Hq, a.Hkv, a.kw, 0, s->T, plan);
+  if (plan == nullptr || plan_bytes < pl.bytes || !aligned16(plan)) return HS2_ERR_WORKSPACE;
+  return cuda_status(launch_sparse_plan(a, pl, static_cast<cudaStream_t>(stream)));
+}
+
+hs2_status hs2_sparse_attn_planned(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V,
+                                   const void* plan, hs2_bf16* O, float* lse, const hs2_shape* s,
+                                   void* stream) {
+  HS2_TRY(check_shape(s, true));
+  HS2_NEED(Q && K && V && plan && O);
+  HS2_NEED(aligned16(Q) && aligned16(K) && aligned16(V) && aligned16(plan) && aligned16(O));
+  if (!union_path(s, s->T)) return HS2_ERR_UNSUPPORTED;
+  SparseArgs a{};
+  a.Q = Q;
+  a.K = K;
+  a.V = V;
+  a.O = O;
+  a.lse = lse;
+  a.T = s->T;
+  a.Hq = s->n_q_heads;
+  a.Hkv = s->n_kv_heads;
+  a.scale = s->scale;
+  a.kw = s->k_global + s->window;
+  a.kv_rows = s->T;
+  const UnionPlan pl = union_plan_layout(s->T, a.Hq, a.Hkv, a.kw, 0, s->T,
+                                         const_cast<void*>(plan));
+  return cuda_status(launch_sparse_union(a, pl, static_cast<cudaStream_t>(stream)));
+}
+
 hs2_status hs2_block_prefill(const hs2_bf16* H, int32_t d_model, const hs2_bf16* W_k,
                              const hs2_bf16* W_v, hs2_bf16* K, hs2_bf16* V,
                              const hs2_bf16* Q_full, hs2_bf16* O_full, float* lse, int32_t* idx,
@@ -328,15 +438,15 @@ hs2_status hs2_block_prefill(const hs2_bf16* H, int32_t d_model, const hs2_bf16*
   HS2_TRY(check_shape(s, true));
   HS2_NEED(n_sparse >= 0 && (n_sparse == 0 || (Q_sparse && O_sparse)));
   for (int l = 0; l < n_sparse; ++l) HS2_NEED(Q_sparse[l] && O_sparse[l]);
-  const size_t need =
-      select_workspace_bytes(s->T, s->n_q_heads, s->n_kv_heads, s->k_global, s->window);
+  const size_t need = block_prefill_bytes(s);
   if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws))) return HS2_ERR_WORKSPACE;
+  for (int l = 0; l < n_sparse; ++l)
+    HS2_NEED(aligned16(Q_sparse[l]) && aligned16(O_sparse[l]));
   if (H != nullptr) HS2_TRY(hs2_bridge_kv(H, d_model, W_k, W_v, K, V, s, stream));
   HS2_TRY(hs2_full_attn_lse(Q_full, K, V, O_full, lse, s, stream));
   HS2_TRY(hs2_select_topk(Q_full, K, lse, idx, nullptr, s, ws, ws_bytes, stream));
-  for (int l = 0; l < n_sparse; ++l)
-    HS2_TRY(hs2_sparse_attn(Q_sparse[l], K, V, idx, O_sparse[l], nullptr, s, stream));
-  return HS2_OK;
+  return block_sparse_layers(s, s->T, K, V, idx, n_sparse, Q_sparse, O_sparse, ws,
+                             static_cast<cudaStream_t>(stream));
 }
 
 hs2_status hs2_block_prefill_rows(int64_t q_begin, const hs2_bf16* K, const hs2_bf16* V,
@@ -353,8 +463,12 @@ hs2_status hs2_block_prefill_rows(int64_t q_begin, const hs2_bf16* K, const hs2_
   HS2_NEED(n_sparse >= 0 && (n_sparse == 0 || (Q_sparse && O_sparse)));
   for (int l = 0; l < n_sparse; ++l)
     HS2_NEED(Q_sparse[l] && O_sparse[l] && aligned16(Q_sparse[l]) && aligned16(O_sparse[l]));
-  const size_t need =
-      select_workspace_bytes(s->T, s->n_q_heads, s->n_kv_heads, s->k_global, s->window);
+  size_t need = select_workspace_bytes(s->T, s->n_q_heads, s->n_kv_heads, s->k_global, s->window);
+  if (union_path(s, q_begin + s->T))
+    need = std::max(need, union_plan_layout(s->T, s->n_q_heads, s->n_kv_heads,
+                                            s->k_global + s->window, 0,
+                                            std::min<int64_t>(s->T, kPlanSlabRows), nullptr)
+                              .bytes);
   if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws))) return HS2_ERR_WORKSPACE;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   AttnArgs fa{Q_full, K, V, O_full, lse, s->T, s->n_q_heads, s->n_kv_heads, s->scale, q_begin};
@@ -362,22 +476,7 @@ hs2_status hs2_block_prefill_rows(int64_t q_begin, const hs2_bf16* K, const hs2_
   SelectArgs sa{Q_full, K, lse, idx, nullptr, s->T, s->n_q_heads, s->n_kv_heads, s->scale,
                 s->k_global, s->window, ws, ws_bytes, q_begin};
   HS2_TRY(cuda_status(launch_select(sa, st)));
-  for (int l = 0; l < n_sparse; ++l) {
-    SparseArgs a{};
-    a.Q = Q_sparse[l];
-    a.K = K;
-    a.V = V;
-    a.idx = idx;
-    a.O = O_sparse[l];
-    a.T = s->T;
-    a.Hq = s->n_q_heads;
-    a.Hkv = s->n_kv_heads;
-    a.scale = s->scale;
-    a.kw = s->k_global + s->window;
-    a.kv_rows = q_begin + s->T;
-    HS2_TRY(cuda_status(launch_sparse(a, st)));
-  }
-  return HS2_OK;
+  return block_sparse_layers(s, q_begin + s->T, K, V, idx, n_sparse, Q_sparse, O_sparse, ws, st);
 }
 
 hs2_status hs2_block_decode(int32_t batch, const int64_t* seq_len, const hs2_bf16* q_full,

@@ -16,12 +16,14 @@ unsigned status_bridge(bool clear);
 unsigned status_full_attn(bool clear);
 unsigned status_select(bool clear);
 unsigned status_sparse(bool clear);
+unsigned status_sparse_union(bool clear);
 unsigned status_decode(bool clear);
 
 // spin budget (cycles) of the bounded waits in each kernel file (testing)
 cudaError_t budget_bridge(long long cycles);
 cudaError_t budget_full_attn(long long cycles);
 cudaError_t budget_select(long long cycles);
+cudaError_t budget_sparse_union(long long cycles);
 cudaError_t budget_decode(long long cycles);
 
 // Tensor maps (bf16, 128-byte swizzle, zero fill out of bounds).
@@ -126,6 +128,31 @@ struct SparseArgs {
   float* rec;       // decode, nullable: write softmax-state records instead of O
 };
 cudaError_t launch_sparse(const SparseArgs& a, cudaStream_t stream);
+
+// Sparse attention over the union of the lists of P = 128 / G consecutive
+// query rows (sparse_union.cu).  A plan covers query blocks qb0 .. qb0+nqb-1
+// (rows qb0*P ..) of every KV head; entry (g, b) = g * nqb + b holds
+// uinfo[entry].x union rows at urow/umask[entry * cap ..] (ascending
+// positions; bit q of a mask: the row is on the list of query row
+// (qb0 + b) * P + q); bit q of uinfo[entry].y: that query's list is not empty.
+constexpr int kUnionMaxEntries = 18432;  // most list entries (P * (k + w)) per item
+struct UnionPlan {
+  int qb0, nqb;
+  int64_t cap;
+  size_t bytes;
+  uint2* uinfo;
+  int32_t* urow;
+  uint32_t* umask;
+};
+bool sparse_union_supported(int64_t T, int Hq, int Hkv, int kw, int64_t kv_rows);
+// layout of a plan for query rows row0 .. row0 + rows - 1 (row0 a multiple of
+// 128) at base (null: sizes only)
+UnionPlan union_plan_layout(int64_t T, int Hq, int Hkv, int kw, int64_t row0, int64_t rows,
+                            void* base);
+// a.idx, a.T, a.Hq, a.Hkv, a.kw, a.kv_rows
+cudaError_t launch_sparse_plan(const SparseArgs& a, const UnionPlan& pl, cudaStream_t stream);
+// a.Q, a.K, a.V, a.O, a.lse, a.T, a.Hq, a.Hkv, a.scale, a.kv_rows
+cudaError_t launch_sparse_union(const SparseArgs& a, const UnionPlan& pl, cudaStream_t stream);
 
 // Fused sparse layers (bf16 K/V): the Q, O and (nullable) lse of each layer
 constexpr int kMaxFusedLayers = 3;
