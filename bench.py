@@ -338,14 +338,15 @@ def bench_decode(hs2, dev, steps, warmup):
 # ---------------------------------------------------------------------------
 # one launch of each hot kernel at a moderate size (for profiler captures)
 # ---------------------------------------------------------------------------
-def select_once(dev, T, Hq, Hkv):
-    """Full attention and one selection launch on the 128K workload's recipe
-    (bridge from H, needles planted, queries mixed with the needle direction)
-    with fewer heads, so that the same key-stream lengths fit a profiler's
-    multi-pass capture (about 1.3 GB on the device at T = 131072, 8/1 heads)."""
+def block_once(dev, T, Hq, Hkv):
+    """Full attention, one selection, the union plan and one sparse layer over
+    it, on the 128K workload's recipe (bridge from H, needles planted, queries
+    mixed with the needle direction) with fewer heads, so that the same
+    key-stream lengths fit a profiler's multi-pass capture (about 2 GB on the
+    device at T = 131072, 8/1 heads)."""
     import long_context_bridge_b200 as hs2
     base = synth.CONFIGS["C3"]
-    cfg = synth.BlockConfig(f"select T={T} {Hq}q/{Hkv}kv", base.number, T, Hq, Hkv,
+    cfg = synth.BlockConfig(f"block T={T} {Hq}q/{Hkv}kv", base.number, T, Hq, Hkv,
                             d_model=base.d_model, n_needles=base.n_needles, q_mix=True)
     H, Wk, Wv = synth.bridge_inputs_torch(cfg, device=dev)
     sh = hs2.Shape.make(T, Hq, Hkv)
@@ -359,13 +360,17 @@ def select_once(dev, T, Hq, Hkv):
     O = torch.empty_like(Q)
     lse = torch.empty(T, Hq, dtype=torch.float32, device=dev)
     hs2.hs2_full_attn_lse(Q, K, V, O, lse, sh)
-    del O
     ws = torch.empty(hs2.workspace_size(hs2.OP_SELECT, sh), dtype=torch.uint8, device=dev)
     idx = torch.empty(T, Hkv, 1152, dtype=torch.int32, device=dev)
     hs2.hs2_select_topk(Q, K, lse, idx, None, sh, ws)
+    del ws
+    plan = torch.empty(hs2.workspace_size(hs2.OP_SPARSE_PLAN, sh), dtype=torch.uint8, device=dev)
+    hs2.hs2_sparse_plan(idx, sh, plan)
+    Qs = synth.q_rows_torch(cfg, synth.TID_QS0, device=dev)
+    hs2.hs2_sparse_attn_planned(Qs, K, V, plan, O, None, sh)
     torch.cuda.synchronize()
     assert hs2.hs2_get_device_status() == hs2.OK
-    print(f"select-once: {cfg.name}", flush=True)
+    print(f"block-once: {cfg.name}", flush=True)
 
 
 def kernels_once(dev):
@@ -387,7 +392,12 @@ def kernels_once(dev):
     ws = torch.empty(hs2.workspace_size(hs2.OP_SELECT, sh), dtype=torch.uint8, device=dev)
     idx = torch.empty(T, Hkv, 1152, dtype=torch.int32, device=dev)
     hs2.hs2_select_topk(Q, K, lse, idx, None, sh, ws)
-    hs2.hs2_sparse_attn(g(synth.TID_QS0, T * Hq * 128).view(T, Hq, 128), K, V, idx, O, None, sh)
+    Qs = g(synth.TID_QS0, T * Hq * 128).view(T, Hq, 128)
+    plan = torch.empty(hs2.workspace_size(hs2.OP_SPARSE_PLAN, sh), dtype=torch.uint8, device=dev)
+    hs2.hs2_sparse_plan(idx, sh, plan)
+    hs2.hs2_sparse_attn_planned(Qs, K, V, plan, O, None, sh)
+    hs2.hs2_sparse_attn(Qs, K, V, idx, O, None, sh)
+    del plan
     K8 = torch.empty(T, Hkv, 128, dtype=torch.uint8, device=dev)
     hs2.hs2_bridge_kv_fp8(H, Wk, Wv, K8, torch.empty_like(K8),
                           torch.empty(T, Hkv, dtype=torch.float32, device=dev),
@@ -405,8 +415,9 @@ def kernels_once(dev):
                          torch.empty(B, Hkv, 1152, dtype=torch.int32, device=dev), q[1:], os_, shd, wsd)
     torch.cuda.synchronize()
     assert hs2.hs2_get_device_status() == hs2.OK
-    print("kernels-once: 32K block (bridge, full attention, selection, one sparse layer, "
-          "bridge into the FP8 cache) and one decode step of 8 x 262144 tokens", flush=True)
+    print("kernels-once: 32K block (bridge, full attention, selection, the union plan and one "
+          "sparse layer over it, the per-list sparse kernel, bridge into the FP8 cache) and one "
+          "decode step of 8 x 262144 tokens", flush=True)
 
 
 # ---------------------------------------------------------------------------
@@ -421,16 +432,16 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--kernels-once", action="store_true",
                     help="run each hot kernel once at a moderate size (profiler driver) and exit")
-    ap.add_argument("--select-once", default=None, metavar="T,HQ,HKV",
-                    help="run full attention and one selection on the 128K recipe with these "
-                         "sizes (profiler driver) and exit")
+    ap.add_argument("--block-once", default=None, metavar="T,HQ,HKV",
+                    help="run full attention, one selection, the union plan and one sparse "
+                         "layer on the 128K recipe with these sizes (profiler driver) and exit")
     args = ap.parse_args()
-    if args.kernels_once or args.select_once:
+    if args.kernels_once or args.block_once:
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
         dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
-        if args.select_once:
-            T_, hq_, hkv_ = (int(x) for x in args.select_once.split(","))
-            select_once(dev, T_, hq_, hkv_)
+        if args.block_once:
+            T_, hq_, hkv_ = (int(x) for x in args.block_once.split(","))
+            block_once(dev, T_, hq_, hkv_)
         else:
             kernels_once(dev)
         return
@@ -481,9 +492,12 @@ def main():
     lse = torch.empty(T, Hq, dtype=torch.float32, device=dev)
     idx = torch.empty(T, Hkv, cfg.k_global + cfg.window, dtype=torch.int32, device=dev)
     ws = torch.empty(hs2.workspace_size(hs2.OP_BLOCK_PREFILL, shape), dtype=torch.uint8, device=dev)
+    # the sparse layers run over the union plan of the selection's lists
+    # (built once per block, shared by the layers)
+    plan = torch.empty(hs2.workspace_size(hs2.OP_SPARSE_PLAN, shape), dtype=torch.uint8, device=dev)
     nr, nh, nv = inp["needle_rows"], inp["needle_heads"], inp["needle_vals"]
 
-    names = ["bridge_kv", "full_attn_lse", "select_topk", "sparse_attn"]
+    names = ["bridge_kv", "full_attn_lse", "select_topk", "sparse_plan", "sparse_attn"]
     ev = {n: [] for n in names}
 
     def step(record=False):
@@ -500,16 +514,19 @@ def main():
         e3 = mark() if record else None
         hs2.hs2_select_topk(inp["Q"], K, lse, idx, None, shape, ws)
         e4 = mark() if record else None
+        hs2.hs2_sparse_plan(idx, shape, plan)
+        e5 = mark() if record else None
         spans = []
         for l in range(cfg.n_sparse):
             a = mark() if record else None
-            hs2.hs2_sparse_attn(inp["Qs"][l], K, V, idx, Os[l], None, shape)
+            hs2.hs2_sparse_attn_planned(inp["Qs"][l], K, V, plan, Os[l], None, shape)
             b = mark() if record else None
             spans.append((a, b))
         if record:
             ev["bridge_kv"].append((e0, e1))
             ev["full_attn_lse"].append((e2, e3))
             ev["select_topk"].append((e3, e4))
+            ev["sparse_plan"].append((e4, e5))
             ev["sparse_attn"].extend(spans)
 
     for _ in range(args.warmup):
@@ -517,6 +534,13 @@ def main():
     torch.cuda.synchronize()
     st = hs2.hs2_get_device_status()
     assert st == hs2.OK, f"device status {st}"
+    # union sizes of the plan (item = 128/G query rows x KV head), for the
+    # sparse kernels' byte and FLOP counts
+    P = 128 // (Hq // Hkv)
+    n_items = -(-T // P) * Hkv
+    u = plan[:n_items * 8].view(torch.int32).view(n_items, 2)[:, 0].long()
+    union_rows = int(u.sum())
+    union_chunks = int(torch.clamp((u + 127) // 128, min=1).sum())
 
     def barrier():
         if pg:
@@ -594,9 +618,10 @@ def main():
             with torch.cuda.stream(copy):
                 hidx.copy_(idx, non_blocking=True)
                 hlse.copy_(lse, non_blocking=True)
+            hs2.hs2_sparse_plan(idx, shape, plan)
             comp.wait_event(qs_in)
             for l in range(cfg.n_sparse):
-                hs2.hs2_sparse_attn(dQs[l], K, V, idx, Os[l], None, shape)
+                hs2.hs2_sparse_attn_planned(dQs[l], K, V, plan, Os[l], None, shape)
                 after(comp, copy)
                 with torch.cuda.stream(copy):
                     hOs[l].copy_(Os[l], non_blocking=True)
@@ -617,8 +642,8 @@ def main():
         e2e = {"value": job_throughput(T, world, ms_e2e), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
                "note": "hs2_bridge_kv, needle rows planted, hs2_full_attn_lse, hs2_select_topk, "
-                       "hs2_sparse_attn x 3 with pinned-host inputs and outputs copied on a "
-                       "second stream, overlapped with compute"}
+                       "hs2_sparse_plan, hs2_sparse_attn_planned x 3 with pinned-host inputs and "
+                       "outputs copied on a second stream, overlapped with compute"}
 
     if rank != 0:
         if pg:
@@ -627,6 +652,8 @@ def main():
 
     hbm, tfl, src = peaks()
     work = algorithmic(cfg)
+    kw_ = cfg.k_global + cfg.window
+    work["sparse_plan"] = ("hbm", float(T) * Hkv * kw_ * 4 + union_rows * 8.0 + n_items * 8.0)
     dom = max(names, key=lambda n: kern_ms[n])
     bound, amount = work[dom]
     secs = kern_ms[dom] / 1e3
@@ -653,13 +680,21 @@ def main():
                                          else (a / s_ / 1e9) / SPEC_HBM_GBS)
     l2_gbs = read_peak_gbs(hs2, dev, 48 << 20, 40)
     hbm_read_gbs = read_peak_gbs(hs2, dev, 2 << 30, 2)
-    sp_gbs = per_kernel["sparse_attn"]["GB/s"]
-    per_kernel["sparse_attn"]["frac_of_l2_read"] = sp_gbs / l2_gbs
-    per_kernel["sparse_attn"]["dram_bytes"] = traffic_from_profiles("sparse_attn")
-    per_kernel["sparse_attn"]["note"] = (
-        "algorithmic bytes (every gathered row counted once per list) over time; the gathered "
-        "rows come mostly from L2 (their DRAM bytes, from ncu, are a few percent of them), so "
-        "the HBM fraction can exceed 1 and the L2 read peak (frac_of_l2_read) is the bound")
+    sp_s = kern_ms["sparse_attn"] / 1e3
+    union_bytes = union_rows * 2 * 128 * 2.0 + T * Hq * 128 * 2 * 2
+    union_flops = union_chunks * 128.0 * 128 * (144 + 128) * 2
+    per_kernel["sparse_attn"].update({
+        "union_rows_per_item": union_rows / n_items,
+        "union_GB/s": union_bytes / sp_s / 1e9,
+        "union_frac_of_l2_read": union_bytes / sp_s / 1e9 / l2_gbs,
+        "executed_TFLOP/s": union_flops / sp_s / 1e12,
+        "executed_frac_of_bf16": union_flops / sp_s / 1e12 / tfl,
+        "dram_bytes": traffic_from_profiles("sparse_attn"),
+        "note": "GB/s and frac: the method's bytes (every list's rows counted once per list, "
+                "1152 per (row, KV head)) over time; the kernel gathers each distinct row of "
+                "128/G neighbouring queries' lists once (union_rows_per_item) and runs masked "
+                "tcgen05 tiles over them, so the list-byte fraction exceeds 1; union_GB/s and "
+                "executed_TFLOP/s are what it moves and computes"})
     probes = {"l2_read_gbs": l2_gbs, "hbm_read_gbs": hbm_read_gbs,
               "how": "hs2_debug_read_probe: 16-byte loads through L2 by 4 CTAs per SM over a "
                      "48 MiB buffer (40 passes) and a 2 GiB buffer (2 passes)"}
@@ -679,11 +714,12 @@ def main():
     fused = {"metric": "3 sparse layers in one pass over the gathered rows, ms @128K",
              "value": fused_ms, "unit": "ms", "separate_ms": kern_ms["sparse_attn"] * cfg.n_sparse,
              "GB/s": cfg.n_sparse * sp / (fused_ms / 1e3) / 1e9,
-             "note": "algorithmic bytes of the three separate layers over the fused time; "
+             "note": "per-list kernel (hs2_sparse_attn_layers); algorithmic bytes of the three "
+                     "layers over the fused time; separate_ms: the step's three planned layers; "
                      "not in the step (a model's layer l+1 queries depend on layer l)"}
     dec = None
     if not args.no_decode:
-        del inp, K, V, O, Os, lse, idx, ws
+        del inp, K, V, O, Os, lse, idx, ws, plan
         torch.cuda.empty_cache()
         dec = bench_decode(hs2, dev, args.steps, args.warmup)
     f1 = bench_bridge_fp8(hs2, dev, args.steps, args.warmup) if not args.no_decode else None
