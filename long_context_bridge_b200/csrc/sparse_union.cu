@@ -394,16 +394,22 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (isV) ++nv; else ++nk;
       }
     };
-    auto fetch_k = [&](int c) {
+    // a chunk's position and mask of this thread's row, loaded one chunk
+    // ahead so that their latency hides behind a softmax
+    int nxt_pos = 0;
+    uint32_t nxt_msk = 0u;
+    auto load_row = [&](int c) {
       const int u = c * TILE + row;
       const bool in = u < U[X];
-      pos = in ? urow[base[X] + u] : 0;
-      const uint32_t msk = in ? umask[base[X] + u] : 0u;
+      nxt_pos = in ? urow[base[X] + u] : 0;
+      nxt_msk = in ? umask[base[X] + u] : 0u;
+    };
+    auto fetch_k = [&]() {  // chunk of nxt_pos / nxt_msk: its mask tile and K rows
       uint32_t w[8];
 #pragma unroll
       for (int c2 = 0; c2 < 8; ++c2) {
-        const uint32_t lo = ((msk >> (2 * c2)) & 1u) ? 0u : masked_bits;
-        const uint32_t hi = ((msk >> (2 * c2 + 1)) & 1u) ? 0u : masked_bits;
+        const uint32_t lo = ((nxt_msk >> (2 * c2)) & 1u) ? 0u : masked_bits;
+        const uint32_t hi = ((nxt_msk >> (2 * c2 + 1)) & 1u) ? 0u : masked_bits;
         w[c2] = lo | (hi << 16);
       }
       *reinterpret_cast<uint4*>(smem + OFF_X + sw128_off(row, 2 + 2 * X)) =
@@ -412,9 +418,14 @@ __global__ void __launch_bounds__(THREADS, 1)
           make_uint4(w[4], w[5], w[6], w[7]);
       fence_proxy_async_smem();
       __syncwarp();
+      pos = nxt_pos;
       gather(false);
     };
-    if (n > 0) fetch_k(0);
+    if (n > 0) {
+      load_row(0);
+      fetch_k();
+      if (n > 1) load_row(1);
+    }
     float m_use = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
@@ -422,7 +433,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_after();
       if (ok) {
         gather(true);                  // V(j): pos still holds chunk j's rows
-        if (j + 1 < n) fetch_k(j + 1);
+        if (j + 1 < n) {
+          fetch_k();                   // K(j + 1)
+          if (j + 2 < n) load_row(j + 2);
+        }
       }
       float x[128];
 #pragma unroll
