@@ -534,9 +534,9 @@ def main():
     torch.cuda.synchronize()
     st = hs2.hs2_get_device_status()
     assert st == hs2.OK, f"device status {st}"
-    # union sizes of the plan (item = 128/G query rows x KV head), for the
-    # sparse kernels' byte and FLOP counts
-    P = 128 // (Hq // Hkv)
+    # union sizes of the plan (item = 256/G query rows x KV head: two 128-row
+    # tiles), for the sparse kernels' byte and FLOP counts
+    P = 256 // (Hq // Hkv)
     n_items = -(-T // P) * Hkv
     u = plan[:n_items * 8].view(torch.int32).view(n_items, 2)[:, 0].long()
     union_rows = int(u.sum())
@@ -682,7 +682,7 @@ def main():
     hbm_read_gbs = read_peak_gbs(hs2, dev, 2 << 30, 2)
     sp_s = kern_ms["sparse_attn"] / 1e3
     union_bytes = union_rows * 2 * 128 * 2.0 + T * Hq * 128 * 2 * 2
-    union_flops = union_chunks * 128.0 * 128 * (144 + 128) * 2
+    union_flops = union_chunks * 2 * 128.0 * 128 * (144 + 128) * 2  # both tiles per chunk
     per_kernel["sparse_attn"].update({
         "union_rows_per_item": union_rows / n_items,
         "union_GB/s": union_bytes / sp_s / 1e9,
@@ -692,7 +692,7 @@ def main():
         "dram_bytes": traffic_from_profiles("sparse_attn"),
         "note": "GB/s and frac: the method's bytes (every list's rows counted once per list, "
                 "1152 per (row, KV head)) over time; the kernel gathers each distinct row of "
-                "128/G neighbouring queries' lists once (union_rows_per_item) and runs masked "
+                "256/G neighbouring queries' lists once (union_rows_per_item) and runs masked "
                 "tcgen05 tiles over them, so the list-byte fraction exceeds 1; union_GB/s and "
                 "executed_TFLOP/s are what it moves and computes"})
     probes = {"l2_read_gbs": l2_gbs, "hbm_read_gbs": hbm_read_gbs,

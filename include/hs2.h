@@ -215,9 +215,10 @@ hs2_status hs2_sparse_attn_layers(int32_t n_layers, const hs2_bf16* const* Q,
 /*
  * Sparse attention in two calls, over the union of neighbouring queries'
  * lists (same operation as hs2_sparse_attn; no counterpart on the pages).
- * The lists of P = 128 / G consecutive query rows of one KV head overlap
+ * The lists of P = 256 / G consecutive query rows of one KV head overlap
  * heavily (their recent windows almost entirely), so each distinct listed row
- * can be gathered once for all of them.
+ * can be gathered once for all of them (two 128-row tensor-core tiles of
+ * (query, head) rows share it).
  *
  * hs2_sparse_plan: from idx [T, n_kv_heads, k_global + window] (as written by
  * hs2_select_topk, any order within a list), per (P query rows, KV head) the
@@ -235,7 +236,7 @@ hs2_status hs2_sparse_attn_layers(int32_t n_layers, const hs2_bf16* const* Q,
  * with the same shape on the same stream (or a synchronised one).
  *
  * Both: HS2_ERR_UNSUPPORTED unless G = n_q_heads / n_kv_heads is 8 or 16,
- * P * (k_global + window) <= 18432 and T * n_kv_heads < 2^31;
+ * P * (k_global + window) <= 36864 and T * n_kv_heads < 2^31;
  * HS2_ERR_WORKSPACE if plan_bytes is short.  hs2_block_prefill and
  * hs2_block_prefill_rows take this path by themselves where it applies.
  */

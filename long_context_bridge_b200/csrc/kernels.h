@@ -129,13 +129,13 @@ struct SparseArgs {
 };
 cudaError_t launch_sparse(const SparseArgs& a, cudaStream_t stream);
 
-// Sparse attention over the union of the lists of P = 128 / G consecutive
-// query rows (sparse_union.cu).  A plan covers query blocks qb0 .. qb0+nqb-1
-// (rows qb0*P ..) of every KV head; entry (g, b) = g * nqb + b holds
-// uinfo[entry].x union rows at urow/umask[entry * cap ..] (ascending
-// positions; bit q of a mask: the row is on the list of query row
+// Sparse attention over the union of the lists of P = 256 / G consecutive
+// query rows, two 128-row tiles (sparse_union.cu).  A plan covers query
+// blocks qb0 .. qb0+nqb-1 (rows qb0*P ..) of every KV head; entry (g, b) =
+// g * nqb + b holds uinfo[entry].x union rows at urow/umask[entry * cap ..]
+// (ascending positions; bit q of a mask: the row is on the list of query row
 // (qb0 + b) * P + q); bit q of uinfo[entry].y: that query's list is not empty.
-constexpr int kUnionMaxEntries = 18432;  // most list entries (P * (k + w)) per item
+constexpr int kUnionMaxEntries = 36864;  // most list entries (P * (k + w)) per item
 struct UnionPlan {
   int qb0, nqb;
   int64_t cap;

@@ -8,34 +8,35 @@
 // heavily (the recent windows almost entirely, the top-k sets largely), so
 // this path gathers each distinct row once for a group of queries:
 //
-//   item = P = 128/G consecutive query rows x one KV head = 128 (query, head)
-//          rows, the M of one tcgen05 tile.
+//   item = P = 256/G consecutive query rows x one KV head = two tcgen05 tiles
+//          of 128 (query, head) rows, A (the first 128/G queries) and B.
 //
 // Plan (sparse_plan_kernel, one CTA per item): the union U of the item's P
 // lists, ascending, and per union row a mask of the queries whose list holds
 // it.  Positions are marked in a shared-memory bitmap one window of 2^17
 // positions at a time; a block scan of the words' bit counts gives every
-// position its rank in the union, so the masks are set with one shared
-// atomic per list entry.  The order of a list does not matter; an entry
+// position its rank in the union, so the masks (in the plan, zeroed first)
+// are set with one atomic per list entry.  The order of a list does not matter; an entry
 // outside [-1, kv_rows) or repeated within its list is reported as
 // DEV_BAD_INDEX and used at most once.
 //
-// Attention (sparse_union_kernel): full_attn.cu's structure on gathered tiles.
-// A CTA owns two items, A and B, and ping-pongs between them:
-//   warp 0     the two Q tiles (TMA)
+// Attention (sparse_union_kernel): full_attn.cu's structure on gathered
+// tiles.  A CTA owns one item; its two Q tiles share every K/V chunk:
+//   warp 0     the Q tiles, then K chunk j (128 union rows, gathered four
+//              rows per TMA, tile::gather4 with 128 B swizzle) and the
+//              chunk's mask tiles into a two-stage ring
+//   warp 10    the V chunks into a two-stage ring
 //   warp 1     TMEM owner; one lane issues per chunk
 //                PV_A(j) S_A(j+1) PV_B(j) S_B(j+1)
 //              S = Q K^T over the 128 dims plus one more K step of 16:
-//              a one-hot of each row's query (A side) against the chunk's
-//              mask tile (B side: 0 where the query's list holds the union
-//              row, -B where it does not, B = 2^e with B * scale * log2 e in
-//              [2^13, 2^14)), so a row's base-2 logits of rows not on its
-//              list drop by at least 2^13 and their probabilities underflow
-//              to exactly 0; P stays in TMEM for PV
-//   warps 2-9  per item, a warpgroup that fetches the item's chunks (128
-//              union rows of K and of V gathered four rows per TMA,
-//              tile::gather4 with 128 B swizzle, plus the chunk's mask tile)
-//              and runs the softmax, one thread per (query, head) row: the
+//              a one-hot of each row's query within its tile (A side)
+//              against the chunk's mask tile for that tile's queries (B side:
+//              0 where the query's list holds the union row, -B where it
+//              does not, B = 2^e with B * scale * log2 e in [2^13, 2^14)),
+//              so a row's base-2 logits of rows not on its list drop by at
+//              least 2^13 and their probabilities underflow to exactly 0;
+//              P stays in TMEM for PV
+//   warps 2-9  softmax of A and of B, one thread per (query, head) row: the
 //              online base-2 softmax of full_attn.cu.  Chunks seen before a
 //              row's first listed key add finite values (logits within
 //              rounding of each other) that the rescale by 2^(-2^13 or less)
@@ -54,6 +55,8 @@ HS2_BUDGET_SETTER(budget_sparse_union)
 
 namespace {
 
+constexpr int TILE = 128;  // union rows per chunk, rows per Q tile
+
 // ----------------------------------------------------------------------------
 // plan
 // ----------------------------------------------------------------------------
@@ -68,21 +71,21 @@ __global__ void __launch_bounds__(PLAN_THREADS)
     sparse_plan_kernel(const int32_t* __restrict__ idx, int T, int Hkv, int kw, int kv_rows,
                        int nqb, int qb0, int64_t cap, uint2* __restrict__ uinfo,
                        int32_t* __restrict__ urow, uint32_t* __restrict__ umask) {
-  static_assert(PLAN_WARPS % P == 0, "warps per query");
-  constexpr int WPQ = PLAN_WARPS / P;  // warps sharing one query's list
+  static_assert(P % PLAN_WARPS == 0 && P <= 32, "queries per item");
   __shared__ uint32_t bitmap[kWinWords];
   __shared__ uint32_t prefix[kWinWords];
   __shared__ uint32_t wsum[PLAN_WARPS];
   __shared__ int max_pos_s;
   __shared__ uint32_t total_s;
   __shared__ uint32_t qmask_s;  // queries with at least one usable entry
-  extern __shared__ uint32_t masks[];  // [P * kw]: query masks of the window's union rows
   const int item = blockIdx.x;         // plan entry: (KV head, query block) of this launch
   const int g = item / nqb, qb = qb0 + item % nqb;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int q = warp / WPQ, part = warp % WPQ;
-  const int64_t row = int64_t(qb) * P + q;
-  const int32_t* list = row < T ? idx + (row * Hkv + g) * kw : nullptr;
+  // warp w takes the lists of queries w, w + 16, ... of the item
+  auto list_of = [&](int q) -> const int32_t* {
+    const int64_t row = int64_t(qb) * P + q;
+    return row < T ? idx + (row * Hkv + g) * kw : nullptr;
+  };
   int32_t* out_row = urow + item * cap;
   uint32_t* out_mask = umask + item * cap;
 
@@ -90,11 +93,14 @@ __global__ void __launch_bounds__(PLAN_THREADS)
     max_pos_s = -1;
     qmask_s = 0;
   }
-  for (int i = threadIdx.x; i < P * kw; i += PLAN_THREADS) masks[i] = 0;
-  // the largest listed position (windows past it hold nothing)
-  int mp = -1;
-  if (list != nullptr) {
-    for (int e = part * 32 + lane; e < kw; e += 32 * WPQ) {
+  __syncthreads();
+  // the largest listed position (windows past it hold nothing), and which
+  // queries have entries
+  for (int q = warp; q < P; q += PLAN_WARPS) {
+    const int32_t* list = list_of(q);
+    if (list == nullptr) continue;
+    int mp = -1;
+    for (int e = lane; e < kw; e += 32) {
       const int j = list[e];
       if (j >= 0 && j < kv_rows) {
         mp = max(mp, j);
@@ -102,13 +108,12 @@ __global__ void __launch_bounds__(PLAN_THREADS)
         set_dev_status(DEV_BAD_INDEX);
       }
     }
-  }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mp = max(mp, __shfl_xor_sync(0xffffffffu, mp, o));
-  __syncthreads();
-  if (lane == 0 && mp >= 0) {
-    atomicMax(&max_pos_s, mp);
-    atomicOr(&qmask_s, 1u << q);
+    for (int o = 16; o > 0; o >>= 1) mp = max(mp, __shfl_xor_sync(0xffffffffu, mp, o));
+    if (lane == 0 && mp >= 0) {
+      atomicMax(&max_pos_s, mp);
+      atomicOr(&qmask_s, 1u << q);
+    }
   }
   __syncthreads();
   const int max_pos = max_pos_s;
@@ -118,8 +123,10 @@ __global__ void __launch_bounds__(PLAN_THREADS)
     for (int i = threadIdx.x; i < kWinWords; i += PLAN_THREADS) bitmap[i] = 0;
     __syncthreads();
     const int64_t W1 = min(W0 + kWinSpan, int64_t(kv_rows));
-    if (list != nullptr) {
-      for (int e = part * 32 + lane; e < kw; e += 32 * WPQ) {
+    for (int q = warp; q < P; q += PLAN_WARPS) {
+      const int32_t* list = list_of(q);
+      if (list == nullptr) continue;
+      for (int e = lane; e < kw; e += 32) {
         const int j = list[e];
         if (j >= W0 && j < W1) atomicOr(&bitmap[(j - W0) >> 5], 1u << (j & 31));
       }
@@ -169,23 +176,23 @@ __global__ void __launch_bounds__(PLAN_THREADS)
     }
     __syncthreads();
     const uint32_t total = total_s;
+    for (uint32_t i = threadIdx.x; i < total; i += PLAN_THREADS) out_mask[ubase + i] = 0u;
+    __syncthreads();
     // each entry's rank in the window's union marks its query there
-    if (list != nullptr) {
-      for (int e = part * 32 + lane; e < kw; e += 32 * WPQ) {
+    for (int q = warp; q < P; q += PLAN_WARPS) {
+      const int32_t* list = list_of(q);
+      if (list == nullptr) continue;
+      for (int e = lane; e < kw; e += 32) {
         const int j = list[e];
         if (j >= W0 && j < W1) {
           const int wd = (j - W0) >> 5;
           const uint32_t r = prefix[wd] + __popc(bitmap[wd] & ((1u << (j & 31)) - 1u));
-          const uint32_t old = atomicOr(&masks[r], 1u << q);
+          const uint32_t old = atomicOr(&out_mask[ubase + r], 1u << q);
           if (old & (1u << q)) set_dev_status(DEV_BAD_INDEX);  // listed twice
         }
       }
     }
     __syncthreads();
-    for (uint32_t i = threadIdx.x; i < total; i += PLAN_THREADS) {
-      out_mask[ubase + i] = masks[i];
-      masks[i] = 0;
-    }
     ubase += total;
     __syncthreads();
   }
@@ -195,16 +202,21 @@ __global__ void __launch_bounds__(PLAN_THREADS)
 // ----------------------------------------------------------------------------
 // attention over the union
 // ----------------------------------------------------------------------------
-constexpr int THREADS = 320;               // Q loader, MMA, two softmax warpgroups
-constexpr int TILE = 128;                  // union rows per chunk, rows per Q tile
+constexpr int THREADS = 352;   // K loader, MMA, two softmax warpgroups, V loader
+constexpr int LOADER_V = 10;
+constexpr int NST = 2;                     // K / V ring stages
 constexpr int CHUNK = TILE * 128;          // bytes of one 64-column half tile
 constexpr int TILE_BYTES = 2 * CHUNK;      // 128 rows x 128 dims bf16
-constexpr int OFF_Q = 0;                   // Q_A, Q_B
-constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;  // K_A, K_B
-constexpr int OFF_V = OFF_K + 2 * TILE_BYTES;  // V_A, V_B
-constexpr int OFF_X = OFF_V + 2 * TILE_BYTES;  // 128 rows x 128 B: one-hot, mask_A, mask_B
-constexpr int OFF_BAR = OFF_X + CHUNK;
+constexpr int OFF_Q = 0;                              // Q_A, Q_B
+constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;         // NST stages
+constexpr int OFF_V = OFF_K + NST * TILE_BYTES;       // NST stages
+// NST extra tiles (128 rows x 128 B, swizzled): 16-column blocks 1 and 2 of
+// stage s hold the mask tiles of tiles A and B for the chunk in stage s;
+// block 0 of stage 0 holds the one-hot of each row's query within its tile
+constexpr int OFF_X = OFF_V + NST * TILE_BYTES;
+constexpr int OFF_BAR = OFF_X + NST * CHUNK;
 constexpr int SMEM = OFF_BAR + 512 + 1024;
+static_assert(SMEM <= 232448, "shared memory per CTA");
 constexpr uint32_t IDESC_S = idesc_bf16(128, 128, 0, 0);   // Q K^T: both K-major
 constexpr uint32_t IDESC_O = idesc_bf16(128, 128, 0, 1);   // P V: V is MN-major
 constexpr float kLog2e = 1.4426950408889634f;
@@ -214,11 +226,11 @@ constexpr uint16_t kBf16One = 0x3F80;      // 1.0
 
 struct Bars {
   uint64_t q_full;
-  uint64_t k_full[2], v_full[2];  // per item: the chunk's gathers have landed
-  uint64_t s_full[2];
-  uint64_t p_full[2];   // 128 arrivals
-  uint64_t o_done[2];
-  uint64_t drain;
+  uint64_t k_full[NST], k_empty[NST], v_full[NST], v_empty[NST];
+  uint64_t s_full[2];   // per Q tile
+  uint64_t p_full[2];   // per Q tile (128 arrivals)
+  uint64_t o_done[2];   // per Q tile (last PV)
+  uint64_t drain;       // the MMA issuer's final commit
   uint32_t tmem_slot;
 };
 
@@ -231,6 +243,21 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int cc) {
   return uint32_t(r) * 128u + (uint32_t(cc ^ (r & 7)) << 4);
 }
 
+// mask tile entries of one union row for the 16 queries of a tile (bits of m)
+__device__ __forceinline__ void mask_row16(uint8_t* x_tile, int r, int block, uint32_t m,
+                                           uint32_t masked_bits) {
+  uint32_t w[8];
+#pragma unroll
+  for (int c2 = 0; c2 < 8; ++c2) {
+    const uint32_t lo = ((m >> (2 * c2)) & 1u) ? 0u : masked_bits;
+    const uint32_t hi = ((m >> (2 * c2 + 1)) & 1u) ? 0u : masked_bits;
+    w[c2] = lo | (hi << 16);
+  }
+  *reinterpret_cast<uint4*>(x_tile + sw128_off(r, 2 * block)) = make_uint4(w[0], w[1], w[2], w[3]);
+  *reinterpret_cast<uint4*>(x_tile + sw128_off(r, 2 * block + 1)) =
+      make_uint4(w[4], w[5], w[6], w[7]);
+}
+
 template <int G>
 __global__ void __launch_bounds__(THREADS, 1)
     sparse_union_kernel(const __grid_constant__ CUtensorMap tmQ,
@@ -240,39 +267,35 @@ __global__ void __launch_bounds__(THREADS, 1)
                         const uint32_t* __restrict__ umask, int64_t cap,
                         __nv_bfloat16* __restrict__ O, float* __restrict__ lse, int T, int Hkv,
                         int nqb, int qb0, float scale_log2, uint32_t masked_bits) {
-  constexpr int P = TILE / G;  // queries per item
+  constexpr int QT = TILE / G;   // queries per Q tile
+  constexpr int P = 2 * QT;      // queries per item
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_align1024(smem_raw);
   Bars* bars = reinterpret_cast<Bars*>(smem + OFF_BAR);
   const int warp = warp_id(), lane = lane_id();
-  const int npair = (nqb + 1) / 2;
-  const int pr = npair - 1 - int(blockIdx.x);  // latest (largest) items first
+  const int lq = nqb - 1 - int(blockIdx.x);  // latest (largest) items first
   const int g = blockIdx.y;
-  int qb[2], U[2], n_c[2];
-  uint32_t qmask[2];
-  int64_t base[2];
-#pragma unroll
-  for (int X = 0; X < 2; ++X) {
-    const int lq = 2 * pr + X;  // query block within this launch
-    qb[X] = qb0 + lq;
-    const bool exists = lq < nqb;
-    base[X] = (int64_t(g) * nqb + lq) * cap;
-    const uint2 info = exists ? uinfo[int64_t(g) * nqb + lq] : make_uint2(0u, 0u);
-    U[X] = int(info.x);
-    qmask[X] = info.y;
-    // an item with an empty union still runs one chunk (all masked) to write its rows
-    n_c[X] = exists ? max(1, (U[X] + TILE - 1) / TILE) : 0;
-  }
-  const int n_max = max(n_c[0], n_c[1]);
+  const int qb = qb0 + lq;
+  const int64_t entry = int64_t(g) * nqb + lq;
+  const int64_t base = entry * cap;
+  const uint2 info = uinfo[entry];
+  const int U = int(info.x);
+  const uint32_t qmask = info.y;
+  // an item with an empty union still runs one chunk (all masked) to write its rows
+  const int n = max(1, (U + TILE - 1) / TILE);
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bars->k_full[s], 32);  // the item's 32 gather issuers
-      mbar_init(&bars->v_full[s], 32);
-      mbar_init(&bars->s_full[s], 1);
-      mbar_init(&bars->p_full[s], 128);
-      mbar_init(&bars->o_done[s], 1);
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
+    }
+    for (int X = 0; X < 2; ++X) {
+      mbar_init(&bars->s_full[X], 1);
+      mbar_init(&bars->p_full[X], 128);
+      mbar_init(&bars->o_done[X], 1);
     }
     mbar_init(&bars->drain, 1);
     fence_barrier_init();
@@ -282,7 +305,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     tc_fence_before();
   }
   if (warp >= 2 && warp < 6) {
-    // one-hot of each row's query: 16-column block 0 of the extra tile
+    // one-hot of each row's query within its tile (block 0 of the stage-0 extra tile)
     const int r = threadIdx.x - 64;
     const int qcol = r / G;
     uint32_t w[8];
@@ -300,58 +323,129 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_slot;
 
-  if (warp == 0) {
-    if (lane == 0) {
-      // ------------------------------ Q tiles --------------------------------
+  if (warp == 0 || warp == LOADER_V) {
+    // ------------------------------- loaders -------------------------------
+    // lane l gathers union rows 4l .. 4l+3 of each chunk (both 64-column
+    // halves); the K loader also writes those rows of the chunk's mask tiles.
+    // Each lane's positions and masks are loaded one chunk ahead.
+    const bool isV = warp == LOADER_V;
+    if (!isV && lane == 0) {
       prefetch_tmap(&tmQ);
-      prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
-      const int nq = n_c[1] > 0 ? 2 : 1;
-      mbar_arrive_expect_tx(&bars->q_full, nq * TILE_BYTES);
-      for (int X = 0; X < nq; ++X)
+      mbar_arrive_expect_tx(&bars->q_full, 2 * TILE_BYTES);
+      for (int X = 0; X < 2; ++X)
         for (int c = 0; c < 2; ++c)
           tma_load_3d(smem + OFF_Q + X * TILE_BYTES + c * CHUNK, &tmQ, &bars->q_full, c * 64,
-                      g * G, qb[X] * P);
-      drain_phase(&bars->q_full, 1);
+                      g * G, qb * P + X * QT);
+    }
+    if (lane == 0) prefetch_tmap(isV ? &tmV : &tmK);
+    int4 np = make_int4(0, 0, 0, 0);
+    uint4 nm = make_uint4(0u, 0u, 0u, 0u);
+    auto load_rows = [&](int j) {
+      const int u0 = j * TILE + 4 * lane;
+      np = *reinterpret_cast<const int4*>(urow + base + u0);
+      if (!isV) nm = *reinterpret_cast<const uint4*>(umask + base + u0);
+    };
+    load_rows(0);
+    int issued = 0;
+    bool ok = true;
+    for (int j = 0; j < n && ok; ++j) {
+      const int s = j % NST;
+      int pos[4] = {np.x, np.y, np.z, np.w};
+      uint32_t msk[4] = {nm.x, nm.y, nm.z, nm.w};
+      if (j + 1 < n) load_rows(j + 1);
+      const int u0 = j * TILE + 4 * lane;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (u0 + i >= U) {  // past the union: row 0, masked for every query
+          pos[i] = 0;
+          msk[i] = 0u;
+        }
+      }
+      uint64_t* full = isV ? &bars->v_full[s] : &bars->k_full[s];
+      bool w_ok = true;
+      if (lane == 0 && j >= NST)
+        w_ok = mbar_wait(isV ? &bars->v_empty[s] : &bars->k_empty[s], ((j / NST) - 1) & 1);
+      if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
+      if (!isV) {
+        uint8_t* x_tile = smem + OFF_X + s * CHUNK;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          mask_row16(x_tile, 4 * lane + i, 1, msk[i] & 0xFFFFu, masked_bits);          // tile A
+          mask_row16(x_tile, 4 * lane + i, 2, (msk[i] >> QT) & 0xFFFFu, masked_bits);  // tile B
+        }
+        fence_proxy_async_smem();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive_expect_tx(full, TILE_BYTES);
+      __syncwarp();
+      uint8_t* dst = smem + (isV ? OFF_V : OFF_K) + s * TILE_BYTES + (4 * lane) * 128;
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
+        tma_gather4(dst + c * CHUNK, isV ? &tmV : &tmK, full, c * 64, pos[0] * Hkv + g,
+                    pos[1] * Hkv + g, pos[2] * Hkv + g, pos[3] * Hkv + g);
+      issued = j + 1;
+    }
+    // every issued copy lands before the CTA can exit
+    if (lane == 0) {
+      if (!isV) drain_phase(&bars->q_full, 1);
+      for (int s = 0; s < NST; ++s)
+        drain_phase(isV ? &bars->v_full[s] : &bars->k_full[s],
+                    issued > s ? uint32_t((issued - 1 - s) / NST + 1) : 0u);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------ MMA issuer -----------------------------
       bool ok = mbar_wait(&bars->q_full, 0);
-      const uint32_t sX = smem_u32(smem + OFF_X);
-      auto issue_s = [&](int X, int j) -> bool {
-        if (!mbar_wait(&bars->k_full[X], j & 1)) return false;
-        tc_fence_after();
+      const uint32_t sX0 = smem_u32(smem + OFF_X);
+      auto issue_s = [&](int X, int j) {
+        const int s = j % NST;
         const uint32_t sQ = smem_u32(smem + OFF_Q + X * TILE_BYTES);
-        const uint32_t sK = smem_u32(smem + OFF_K + X * TILE_BYTES);
+        const uint32_t sK = smem_u32(smem + OFF_K + s * TILE_BYTES);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
           mma_ss(tmem + X * 256, kmajor_desc(sQ, ks), kmajor_desc(sK, ks), IDESC_S, ks > 0);
         // the list masks: one-hot(query) . mask row
-        mma_ss(tmem + X * 256, sdesc_sw128(sX, 16, 1024), sdesc_sw128(sX + 32 * (1 + X), 16, 1024),
-               IDESC_S, 1);
+        mma_ss(tmem + X * 256, sdesc_sw128(sX0, 16, 1024),
+               sdesc_sw128(sX0 + s * CHUNK + 32 * (1 + X), 16, 1024), IDESC_S, 1);
         mma_commit(&bars->s_full[X]);
-        return true;
       };
       auto issue_pv = [&](int X, int j) -> bool {
-        if (!mbar_wait(&bars->v_full[X], j & 1)) return false;
         if (!mbar_wait(&bars->p_full[X], j & 1)) return false;
         tc_fence_after();
-        const uint32_t sV = smem_u32(smem + OFF_V + X * TILE_BYTES);
+        const uint32_t sV = smem_u32(smem + OFF_V + (j % NST) * TILE_BYTES);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
           const uint64_t bd = sdesc_sw128(sV + ks * 16 * 128, CHUNK, 1024);
           mma_ts(tmem + X * 256 + 128, tmem + X * 256 + ks * 8, bd, IDESC_O, (j > 0 || ks > 0));
         }
-        if (j == n_c[X] - 1) mma_commit(&bars->o_done[X]);
+        if (j == n - 1) mma_commit(&bars->o_done[X]);
         return true;
       };
-      for (int X = 0; X < 2 && ok; ++X)
-        if (n_c[X] > 0) ok = issue_s(X, 0);
-      for (int j = 0; j < n_max && ok; ++j) {
-        for (int X = 0; X < 2 && ok; ++X) {
-          if (j < n_c[X]) ok = issue_pv(X, j);
-          if (ok && j + 1 < n_c[X]) ok = issue_s(X, j + 1);
+      if (ok) {
+        ok = mbar_wait(&bars->k_full[0], 0);
+        tc_fence_after();
+        if (ok) {
+          issue_s(0, 0);
+          issue_s(1, 0);
+          mma_commit(&bars->k_empty[0]);
+        }
+      }
+      for (int j = 0; j < n && ok; ++j) {
+        const int s = j % NST;
+        const bool next = j + 1 < n;
+        if (!mbar_wait(&bars->v_full[s], (j / NST) & 1)) { ok = false; break; }
+        if (!issue_pv(0, j)) { ok = false; break; }
+        if (next) {
+          const int s1 = (j + 1) % NST;
+          if (!mbar_wait(&bars->k_full[s1], ((j + 1) / NST) & 1)) { ok = false; break; }
+          tc_fence_after();
+          issue_s(0, j + 1);
+        }
+        if (!issue_pv(1, j)) { ok = false; break; }
+        mma_commit(&bars->v_empty[s]);
+        if (next) {
+          issue_s(1, j + 1);
+          mma_commit(&bars->k_empty[(j + 1) % NST]);
         }
       }
       mma_drain(&bars->drain);  // no MMA outlives the TMEM
@@ -361,83 +455,16 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int X = (warp - 2) >> 2;
     const int sub = warp & 3;
     const int row = sub * 32 + lane;            // TMEM lane == tile row
-    const int qi = qb[X] * P + row / G;         // query row
+    const int qin = X * QT + row / G;           // query within the item
+    const int qi = qb * P + qin;                // query row
     const int h = g * G + row % G;              // query head
     const uint32_t lane_addr = uint32_t(sub * 32) << 16;
     const uint32_t tS = tmem + lane_addr + X * 256, tO = tS + 128;
-    const int n = n_c[X];
-    // This warpgroup also fetches its item's chunks: thread `row` loads union
-    // row `row` of a chunk's position and mask and writes the row's mask
-    // tile entries; every fourth thread gathers its group of four rows (both
-    // 64-column halves) with two TMA gathers.  K and the mask tile of chunk
-    // j + 1 and V of chunk j go out as soon as S(j) is complete (which also
-    // means PV(j - 1) is: the MMAs complete in issue order), so they overlap
-    // this chunk's softmax.
-    const bool issuer = (lane & 3) == 0;
-    uint8_t* const k_dst = smem + OFF_K + X * TILE_BYTES + (row & ~3) * 128;
-    uint8_t* const v_dst = smem + OFF_V + X * TILE_BYTES + (row & ~3) * 128;
-    int pos = 0;
-    uint32_t nk = 0, nv = 0;  // this thread's K and V gathers issued (issuers)
-    auto gather = [&](bool isV) {
-      const int p0 = __shfl_sync(0xffffffffu, pos, lane & ~3);
-      const int p1 = __shfl_sync(0xffffffffu, pos, (lane & ~3) + 1);
-      const int p2 = __shfl_sync(0xffffffffu, pos, (lane & ~3) + 2);
-      const int p3 = __shfl_sync(0xffffffffu, pos, (lane & ~3) + 3);
-      if (issuer) {
-        uint64_t* full = isV ? &bars->v_full[X] : &bars->k_full[X];
-        const CUtensorMap* map = isV ? &tmV : &tmK;
-        uint8_t* dst = isV ? v_dst : k_dst;
-        mbar_arrive_expect_tx(full, 2 * 4 * 128);
-        for (int c = 0; c < 2; ++c)
-          tma_gather4(dst + c * CHUNK, map, full, c * 64, p0 * Hkv + g, p1 * Hkv + g,
-                      p2 * Hkv + g, p3 * Hkv + g);
-        if (isV) ++nv; else ++nk;
-      }
-    };
-    // a chunk's position and mask of this thread's row, loaded one chunk
-    // ahead so that their latency hides behind a softmax
-    int nxt_pos = 0;
-    uint32_t nxt_msk = 0u;
-    auto load_row = [&](int c) {
-      const int u = c * TILE + row;
-      const bool in = u < U[X];
-      nxt_pos = in ? urow[base[X] + u] : 0;
-      nxt_msk = in ? umask[base[X] + u] : 0u;
-    };
-    auto fetch_k = [&]() {  // chunk of nxt_pos / nxt_msk: its mask tile and K rows
-      uint32_t w[8];
-#pragma unroll
-      for (int c2 = 0; c2 < 8; ++c2) {
-        const uint32_t lo = ((nxt_msk >> (2 * c2)) & 1u) ? 0u : masked_bits;
-        const uint32_t hi = ((nxt_msk >> (2 * c2 + 1)) & 1u) ? 0u : masked_bits;
-        w[c2] = lo | (hi << 16);
-      }
-      *reinterpret_cast<uint4*>(smem + OFF_X + sw128_off(row, 2 + 2 * X)) =
-          make_uint4(w[0], w[1], w[2], w[3]);
-      *reinterpret_cast<uint4*>(smem + OFF_X + sw128_off(row, 3 + 2 * X)) =
-          make_uint4(w[4], w[5], w[6], w[7]);
-      fence_proxy_async_smem();
-      __syncwarp();
-      pos = nxt_pos;
-      gather(false);
-    };
-    if (n > 0) {
-      load_row(0);
-      fetch_k();
-      if (n > 1) load_row(1);
-    }
     float m_use = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       ok = ok && mbar_wait(&bars->s_full[X], j & 1);
       tc_fence_after();
-      if (ok) {
-        gather(true);                  // V(j): pos still holds chunk j's rows
-        if (j + 1 < n) {
-          fetch_k();                   // K(j + 1)
-          if (j + 2 < n) load_row(j + 2);
-        }
-      }
       float x[128];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
@@ -500,38 +527,31 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_arrive(&bars->p_full[X]);
     }
     // epilogue: O / l and lse (a row of a query with an empty list: 0, -inf)
-    if (n > 0) {
-      ok = ok && mbar_wait(&bars->o_done[X], 0);
-      tc_fence_after();
-      const bool empty = ((qmask[X] >> (row / G)) & 1u) == 0u;
-      const float inv = empty ? 0.f : 1.f / l;
-      const bool store = ok && qi < T;
-      __nv_bfloat16* dst = O + (size_t(qi) * (Hkv * G) + h) * 128;
+    ok = ok && mbar_wait(&bars->o_done[X], 0);
+    tc_fence_after();
+    const bool empty = ((qmask >> qin) & 1u) == 0u;
+    const float inv = empty ? 0.f : 1.f / l;
+    const bool store = ok && qi < T;
+    __nv_bfloat16* dst = O + (size_t(qi) * (Hkv * G) + h) * 128;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tO + c * 32, r);
-        tmem_wait_ld();
-        if (store) {
+    for (int c = 0; c < 4; ++c) {
+      uint32_t r[32];
+      tmem_ld32(tO + c * 32, r);
+      tmem_wait_ld();
+      if (store) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint4 v;
-            v.x = pack_bf16x2(__uint_as_float(r[8 * q + 0]) * inv, __uint_as_float(r[8 * q + 1]) * inv);
-            v.y = pack_bf16x2(__uint_as_float(r[8 * q + 2]) * inv, __uint_as_float(r[8 * q + 3]) * inv);
-            v.z = pack_bf16x2(__uint_as_float(r[8 * q + 4]) * inv, __uint_as_float(r[8 * q + 5]) * inv);
-            v.w = pack_bf16x2(__uint_as_float(r[8 * q + 6]) * inv, __uint_as_float(r[8 * q + 7]) * inv);
-            reinterpret_cast<uint4*>(dst + c * 32)[q] = v;
-          }
+        for (int q = 0; q < 4; ++q) {
+          uint4 v;
+          v.x = pack_bf16x2(__uint_as_float(r[8 * q + 0]) * inv, __uint_as_float(r[8 * q + 1]) * inv);
+          v.y = pack_bf16x2(__uint_as_float(r[8 * q + 2]) * inv, __uint_as_float(r[8 * q + 3]) * inv);
+          v.z = pack_bf16x2(__uint_as_float(r[8 * q + 4]) * inv, __uint_as_float(r[8 * q + 5]) * inv);
+          v.w = pack_bf16x2(__uint_as_float(r[8 * q + 6]) * inv, __uint_as_float(r[8 * q + 7]) * inv);
+          reinterpret_cast<uint4*>(dst + c * 32)[q] = v;
         }
       }
-      if (store && lse != nullptr)
-        lse[size_t(qi) * (Hkv * G) + h] = empty ? -INFINITY : (m_use + __log2f(l)) * kLn2;
     }
-    // every gather this thread issued has landed before the CTA can exit
-    if (issuer) {
-      drain_phase(&bars->k_full[X], nk);
-      drain_phase(&bars->v_full[X], nv);
-    }
+    if (store && lse != nullptr)
+      lse[size_t(qi) * (Hkv * G) + h] = empty ? -INFINITY : (m_use + __log2f(l)) * kLn2;
   }
   tc_fence_before();
   __syncthreads();
@@ -541,7 +561,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-int union_p(int Hq, int Hkv) { return Hkv > 0 ? TILE / (Hq / Hkv) : 0; }
+// queries per plan item (two Q tiles)
+int union_p(int Hq, int Hkv) { return Hkv > 0 ? 2 * TILE / (Hq / Hkv) : 0; }
 
 // bf16 bits of -B, B = 2^e the power of two with B * scale * log2 e in
 // [2^13, 2^14): far enough below every listed logit, near enough that
@@ -556,10 +577,10 @@ uint32_t masked_bf16_bits(float scale) {
 
 template <int G>
 cudaError_t launch_union_g(const SparseArgs& a, const UnionPlan& pl, cudaStream_t stream) {
-  constexpr int P = TILE / G;
+  constexpr int QT = TILE / G;
   CUtensorMap tmQ, tmK, tmV;
-  // Q [T, Hq, 128]: box 64 dims x G heads x P tokens -> 128 rows of 128 B
-  if (!make_tmap_3d(&tmQ, a.Q, 128, a.Hq, a.T, 256, uint64_t(a.Hq) * 256, 64, G, P))
+  // Q [T, Hq, 128]: box 64 dims x G heads x QT tokens -> 128 rows of 128 B
+  if (!make_tmap_3d(&tmQ, a.Q, 128, a.Hq, a.T, 256, uint64_t(a.Hq) * 256, 64, G, QT))
     return cudaErrorInvalidValue;
   // K, V as [kv_rows * Hkv] rows of 128 dims: box 64 dims x 1 row, gathered
   // four rows at a time
@@ -568,7 +589,7 @@ cudaError_t launch_union_g(const SparseArgs& a, const UnionPlan& pl, cudaStream_
   if (!make_tmap_2d(&tmV, a.V, 128, rows, 256, 64, 1)) return cudaErrorInvalidValue;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(sparse_union_kernel<G>), SMEM);
   if (e != cudaSuccess) return e;
-  const dim3 grid(unsigned((pl.nqb + 1) / 2), unsigned(a.Hkv));
+  const dim3 grid(unsigned(pl.nqb), unsigned(a.Hkv));
   sparse_union_kernel<G><<<grid, THREADS, SMEM, stream>>>(
       tmQ, tmK, tmV, pl.uinfo, pl.urow, pl.umask, pl.cap, reinterpret_cast<__nv_bfloat16*>(a.O),
       a.lse, int(a.T), a.Hkv, pl.nqb, pl.qb0, a.scale * kLog2e, masked_bf16_bits(a.scale));
@@ -578,11 +599,8 @@ cudaError_t launch_union_g(const SparseArgs& a, const UnionPlan& pl, cudaStream_
 
 template <int P>
 cudaError_t launch_plan_p(const SparseArgs& a, const UnionPlan& pl, cudaStream_t stream) {
-  const int dyn = P * a.kw * int(sizeof(uint32_t));
-  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(sparse_plan_kernel<P>), dyn);
-  if (e != cudaSuccess) return e;
   const unsigned items = unsigned(pl.nqb) * unsigned(a.Hkv);
-  sparse_plan_kernel<P><<<items, PLAN_THREADS, dyn, stream>>>(
+  sparse_plan_kernel<P><<<items, PLAN_THREADS, 0, stream>>>(
       a.idx, int(a.T), a.Hkv, a.kw, int(a.kv_rows), pl.nqb, pl.qb0, pl.cap, pl.uinfo, pl.urow,
       pl.umask);
   count_launch();
@@ -595,7 +613,7 @@ bool sparse_union_supported(int64_t T, int Hq, int Hkv, int kw, int64_t kv_rows)
   if (Hkv <= 0 || Hq % Hkv != 0) return false;
   const int G = Hq / Hkv;
   if (G != 8 && G != 16) return false;
-  const int P = TILE / G;
+  const int P = union_p(Hq, Hkv);
   return kw >= 1 && int64_t(P) * kw <= kUnionMaxEntries && T >= 1 && T <= INT32_MAX &&
          kv_rows >= T && kv_rows * Hkv <= INT32_MAX;
 }
@@ -623,8 +641,8 @@ UnionPlan union_plan_layout(int64_t T, int Hq, int Hkv, int kw, int64_t row0, in
 
 cudaError_t launch_sparse_plan(const SparseArgs& a, const UnionPlan& pl, cudaStream_t stream) {
   switch (union_p(a.Hq, a.Hkv)) {
+    case 32: return launch_plan_p<32>(a, pl, stream);
     case 16: return launch_plan_p<16>(a, pl, stream);
-    case 8: return launch_plan_p<8>(a, pl, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -1,6 +1,6 @@
 """Sparse attention over the union plan (hs2_sparse_plan, then
 hs2_sparse_attn_planned) against the oracle's sparse attention on the same
-lists.  Item = P = 128/G consecutive query rows of one KV head: the cases
+lists.  Item = P = 256/G consecutive query rows of one KV head: the cases
 cover G = 8 and 16, ragged T (a partial last item), unions of one to several
 128-row chunks, lists in scrambled order, rows whose list is empty, and
 entries that are out of range or repeated (reported as bad and used at most
@@ -81,8 +81,8 @@ def test_planned_sparse_scrambled_lists_and_empty_rows(hs2, orc):
             idx[r, g] = idx[r, g, rng.permutation(k + w)]
     empty = [3, 700, 701, 1499]
     idx[empty, 1] = -1
-    idx[1024:1040, 0] = -1   # every list of one item (P = 16 rows) of KV head 0
-    idx[1200:1208, 0] = -1   # half of another item
+    idx[1024:1056, 0] = -1   # every list of one item (P = 32 rows) of KV head 0
+    idx[1200:1216, 0] = -1   # the first of the two tiles of another item
     O, lse, st = run_planned(hs2, Qs, K, V, idx, T, Hq, Hkv, k, w)
     assert st == hs2.OK
     Oo, lo = orc.sparse_attn(kv, Qs, idx, sc)
@@ -95,7 +95,7 @@ def test_planned_sparse_scrambled_lists_and_empty_rows(hs2, orc):
     Oh = host_f64(O)
     for r in empty:
         assert np.all(Oh[r, G:2 * G] == 0.0) and np.all(got_l[r, G:2 * G] == -np.inf)
-    for a, b in [(1024, 1040), (1200, 1208)]:
+    for a, b in [(1024, 1056), (1200, 1216)]:
         assert np.all(Oh[a:b, :G] == 0.0) and np.all(got_l[a:b, :G] == -np.inf)
 
 
