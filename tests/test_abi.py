@@ -131,3 +131,37 @@ def test_workspace_size_queries(hs2):
     assert hs2.workspace_size(hs2.OP_SPARSE, s) == 0
     with pytest.raises(hs2.HS2Error):
         hs2.workspace_size(hs2.OP_FULL_ATTN, hs2.Shape.make(32768, 16, 2, head_dim=96))
+
+
+def test_sparse_plan_sizes_and_host_checks(hs2):
+    """The union plan's size follows its layout (per item of 256/G query rows:
+    a (count, mask) pair, then positions and masks for (256/G)(k+w) entries
+    rounded up to 128, per KV head), and the two plan calls reject unsupported
+    shapes, missing buffers and a short plan on the host."""
+    L = _raw(hs2)
+    ok_ptr = C.c_void_p(0x10000)
+    for T, hq, hkv, k, w in ((131072, 32, 4, 1024, 128), (1000, 16, 1, 2048, 256), (700, 32, 2, 64, 16)):
+        P = 256 // (hq // hkv)
+        s = hs2.Shape.make(T, hq, hkv, k_global=k, window=w)
+        items = -(-T // P) * hkv
+        cap = -(-(P * (k + w)) // 128) * 128
+        want = -(-(items * 8) // 256) * 256 + 2 * items * cap * 4
+        assert hs2.workspace_size(hs2.OP_SPARSE_PLAN, s) == want
+        # a plan one byte short
+        assert L.hs2_sparse_plan(ok_ptr, C.byref(s), ok_ptr, want - 1, None) == hs2.ERR_WORKSPACE
+        assert L.hs2_sparse_plan(None, C.byref(s), ok_ptr, want, None) == hs2.ERR_INVALID_ARG
+        assert L.hs2_sparse_attn_planned(ok_ptr, ok_ptr, ok_ptr, None, ok_ptr, None, C.byref(s),
+                                         None) == hs2.ERR_INVALID_ARG
+    # no plan path: G outside {8, 16}, or (256/G)(k + w) above 36864
+    for hq, hkv, k, w in ((8, 2, 64, 16), (8, 1, 1024, 256), (64, 4, 2048, 512)):
+        s = hs2.Shape.make(4096, hq, hkv, k_global=k, window=w)
+        with pytest.raises(hs2.HS2Error):
+            hs2.workspace_size(hs2.OP_SPARSE_PLAN, s)
+        assert L.hs2_sparse_plan(ok_ptr, C.byref(s), ok_ptr, 1 << 40, None) == hs2.ERR_UNSUPPORTED
+        assert L.hs2_sparse_attn_planned(ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr, None, C.byref(s),
+                                         None) == hs2.ERR_UNSUPPORTED
+    # the block prefill's workspace covers a plan slab (32768 rows) as well as the selection
+    s = hs2.Shape.make(131072, 32, 4)
+    slab_items = 32768 // 32 * 4
+    slab = -(-(slab_items * 8) // 256) * 256 + 2 * slab_items * 1152 * 32 * 4
+    assert hs2.workspace_size(hs2.OP_BLOCK_PREFILL, s) >= slab
