@@ -342,7 +342,7 @@ def block_once(dev, T, Hq, Hkv):
     """Full attention, one selection, the union plan and one sparse layer over
     it, on the 128K workload's recipe (bridge from H, needles planted, queries
     mixed with the needle direction) with fewer heads, so that the same
-    key-stream lengths fit a profiler's multi-pass capture (about 2 GB on the
+    key-stream lengths fit a profiler's multi-pass capture (a few GB on the
     device at T = 131072, 8/1 heads)."""
     import long_context_bridge_b200 as hs2
     base = synth.CONFIGS["C3"]
